@@ -1,0 +1,142 @@
+"""fp64 CPU oracle of the DiG token mixer (GLA recurrence, backward, SREM, epilogue).
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+package.  It shares no code with the CUDA path and never imports it.
+
+Every function takes numpy arrays (any float dtype; they are widened to fp64)
+in the layouts documented in ``oracle.c`` and returns fp64 arrays.
+
+Parity status of each function (what pins it is in tests/test_oracle_pins.py):
+  gla_fwd        pinned: brute-force quadratic form, alpha==1 causal linear
+                 attention, alpha->0 diagonal case, constant-gate closed form,
+                 causality and linearity
+  gla_bwd        pinned: central finite differences of a scalar loss, and the
+                 reverse-cumsum identity for d log(alpha)
+  srem_dwconv    pinned: scipy.signal.correlate2d, identity kernel = pure
+                 permutation, all-ones kernel on a constant grid (9/6/4)
+  epilogue       pinned: unit RMS of the normalised row, Swish(0) = 0,
+                 positive scale invariance
+  scan_index     pinned: bijection, inverse restores the grid, transpose on
+                 square grids, a hand-derived 3x4 fixture
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        L = ctypes.c_long
+        lib.oracle_scan_index.restype = L
+        lib.oracle_scan_index.argtypes = [ctypes.c_int, L, L, L]
+        lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+        lib.oracle_gla_fwd.restype = ctypes.c_int
+        lib.oracle_gla_fwd.argtypes = [dp, dp, dp, dp, ctypes.c_int, ctypes.c_double, dp,
+                                       L, L, L, L, L, L, L, ctypes.c_int]
+        lib.oracle_gla_bwd.restype = ctypes.c_int
+        lib.oracle_gla_bwd.argtypes = [dp, dp, dp, dp, ctypes.c_int, ctypes.c_double, dp,
+                                       dp, dp, dp, dp, L, L, L, L, L, L, L, ctypes.c_int]
+        lib.oracle_epilogue.restype = ctypes.c_int
+        lib.oracle_epilogue.argtypes = [dp, dp, dp, ctypes.c_double, dp, L, L]
+        lib.oracle_srem_dwconv.restype = ctypes.c_int
+        lib.oracle_srem_dwconv.argtypes = [dp, dp, dp, dp, L, L, L, L, ctypes.c_int]
+        _lib = lib
+    return _lib
+
+
+def _f64(a):
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    _load().oracle_set_num_threads(int(n))
+
+
+def scan_index(mode: int, grid_h: int, grid_w: int) -> np.ndarray:
+    """perm[t] = grid index (row * grid_w + col) visited at scan position t."""
+    lib = _load()
+    L = grid_h * grid_w
+    out = np.array([lib.oracle_scan_index(mode, grid_h, grid_w, t) for t in range(L)],
+                   dtype=np.int64)
+    if L and out.min() < 0:
+        raise ValueError("bad scan mode %r" % (mode,))
+    return out
+
+
+def gla_fwd(q, k, v, z, inv_tau, grid_h, grid_w, mode):
+    """o [B,L,H,dv] of the GLA recurrence.  q,k [B,L,H,dk]; v [B,L,H,dv];
+    z [B,L,Hz,dk] gate logits with Hz in {1, H}."""
+    q, k, v, z = _f64(q), _f64(k), _f64(v), _f64(z)
+    B, L, H, dk = q.shape
+    dv = v.shape[3]
+    gh = z.shape[2]
+    o = np.zeros((B, L, H, dv), dtype=np.float64)
+    rc = _load().oracle_gla_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(z), gh, float(inv_tau), _ptr(o),
+                                B, H, L, dk, dv, grid_h, grid_w, int(mode))
+    if rc:
+        raise ValueError("oracle_gla_fwd rejected the arguments (rc=%d)" % rc)
+    return o
+
+
+def gla_bwd(q, k, v, z, inv_tau, dO, grid_h, grid_w, mode):
+    """(dq, dk, dv, dlogalpha) of sum(o * dO); dlogalpha is shaped like z."""
+    q, k, v, z, dO = _f64(q), _f64(k), _f64(v), _f64(z), _f64(dO)
+    B, L, H, dk = q.shape
+    dv = v.shape[3]
+    gh = z.shape[2]
+    dq = np.zeros_like(q)
+    dkk = np.zeros_like(k)
+    dvv = np.zeros_like(v)
+    dla = np.zeros_like(z)
+    rc = _load().oracle_gla_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(z), gh, float(inv_tau), _ptr(dO),
+                                _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dla),
+                                B, H, L, dk, dv, grid_h, grid_w, int(mode))
+    if rc:
+        raise ValueError("oracle_gla_bwd rejected the arguments (rc=%d)" % rc)
+    return dq, dkk, dvv, dla
+
+
+def epilogue(o, r, gamma=None, eps=1e-5):
+    """y = Swish(r) * RMSNorm_dv(o) * gamma over the last axis."""
+    o, r = _f64(o), _f64(r)
+    dv = o.shape[-1]
+    rows = o.size // dv if dv else 0
+    g = None if gamma is None else _f64(gamma)
+    y = np.zeros_like(o)
+    rc = _load().oracle_epilogue(_ptr(o), _ptr(r), _ptr(g), float(eps), _ptr(y), rows, dv)
+    if rc:
+        raise ValueError("oracle_epilogue rejected the arguments")
+    return y
+
+
+def srem_dwconv(x, w, bias, mode):
+    """x [B,Hg,Wg,C] grid order; w [C,3,3]; bias [C] or None -> y [B,L,C] in scan order."""
+    x, w = _f64(x), _f64(w)
+    B, Hg, Wg, C = x.shape
+    bb = None if bias is None else _f64(bias)
+    y = np.zeros((B, Hg * Wg, C), dtype=np.float64)
+    rc = _load().oracle_srem_dwconv(_ptr(x), _ptr(w), _ptr(bb), _ptr(y), B, Hg, Wg, C, int(mode))
+    if rc:
+        raise ValueError("oracle_srem_dwconv rejected the arguments")
+    return y

@@ -1,0 +1,285 @@
+/*
+ * oracle.c -- plain, slow, step-by-step fp64 reference of the DiG token mixer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test-suite, the smoke check and the CPU
+ * baseline leg of the benchmark may load this library.  It shares no code,
+ * header, table or constant with the CUDA path in gated_linear_attention_fwd_b200/.
+ *
+ * Sources ("DiG: Scalable and Efficient Diffusion Models with Gated Linear
+ * Attention", the docswell study-group slides, page 2 of the reference set):
+ *   - GLA recurrence: slide "Gated Linear Attention Transformer (GLA) の導入",
+ *     eq. (5)-(8).  The gate is read as alpha_t = sigmoid(z_t)^(1/tau) with the
+ *     value gate beta fixed to 1, the state is S_t = diag(alpha_t) S_{t-1} + k_t^T v_t
+ *     and the output is the row-vector product o_t = q_t S_t (S includes token t).
+ *   - Output gate and norm: same slide, eq. (9)-(10), with the norm read as
+ *     RMSNorm over d_v (Fig. 4 labels it "RMS Norm").
+ *   - SREM: slide "SREM (Spatial Reorient & Enhancement Module) の導入": a 3x3
+ *     depthwise conv on the 2-D token grid followed by a transpose / flip of the
+ *     scan order.
+ * Every reading of a garbled or silent passage is listed in the design doc.
+ *
+ * Layouts (all fp64, row-major, tokens in grid row-major order g = row*Wg + col):
+ *   q, k        [B][L][H][dk]
+ *   v, o, dO    [B][L][H][dv]
+ *   z, dlogalpha [B][L][Hz][dk]   (Hz = gate_heads, 1 or H)
+ *   x (conv in) [B][Hg][Wg][C];  conv out y [B][L][C] in scan order
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Scan order: grid index visited at scan position t (DiG scanning directions;
+ * the four modes are row-major forward / reversed and column-major forward /
+ * reversed).  Returns -1 for a bad mode. */
+long oracle_scan_index(int mode, long Hg, long Wg, long t)
+{
+    long L = Hg * Wg;
+    switch (mode) {
+    case 0: return t;                                   /* row-major, forward   */
+    case 1: return L - 1 - t;                           /* row-major, reversed  */
+    case 2: return (t % Hg) * Wg + t / Hg;              /* column-major forward */
+    case 3: { long u = L - 1 - t; return (u % Hg) * Wg + u / Hg; } /* col, reversed */
+    default: return -1;
+    }
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+/* log(sigmoid(x)) evaluated without overflow. */
+static double log_sigmoid(double x)
+{
+    return (x < 0.0 ? x : 0.0) - log1p(exp(-fabs(x)));
+}
+
+static int check_shape(long B, long H, long L, long dk, long dv, long Hg, long Wg,
+                       int mode, int gate_heads)
+{
+    if (B < 0 || H <= 0 || L < 0 || dk <= 0 || dv <= 0) return 1;
+    if (Hg * Wg != L) return 1;
+    if (mode < 0 || mode > 3) return 1;
+    if (gate_heads != 1 && gate_heads != H) return 1;
+    return 0;
+}
+
+/* Forward recurrence, one token at a time in scan order. */
+int oracle_gla_fwd(const double *q, const double *k, const double *v, const double *z,
+                   int gate_heads, double inv_tau, double *o,
+                   long B, long H, long L, long dk, long dv, long Hg, long Wg, int mode)
+{
+    if (check_shape(B, H, L, dk, dv, Hg, Wg, mode, gate_heads)) return 1;
+    long n = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < n; ++bh) {
+        long b = bh / H, h = bh % H, hz = (gate_heads == 1) ? 0 : h;
+        double *S = (double *)calloc((size_t)(dk * dv), sizeof(double));
+        double *alpha = (double *)malloc((size_t)dk * sizeof(double));
+        for (long t = 0; t < L; ++t) {
+            long g = oracle_scan_index(mode, Hg, Wg, t);
+            const double *qt = q + ((b * L + g) * H + h) * dk;
+            const double *kt = k + ((b * L + g) * H + h) * dk;
+            const double *vt = v + ((b * L + g) * H + h) * dv;
+            const double *zt = z + ((b * L + g) * gate_heads + hz) * dk;
+            double *ot = o + ((b * L + g) * H + h) * dv;
+            for (long c = 0; c < dk; ++c) alpha[c] = exp(inv_tau * log_sigmoid(zt[c]));
+            /* S_t = diag(alpha_t) S_{t-1} + k_t^T v_t */
+            for (long c = 0; c < dk; ++c)
+                for (long j = 0; j < dv; ++j)
+                    S[c * dv + j] = alpha[c] * S[c * dv + j] + kt[c] * vt[j];
+            /* o_t = q_t S_t */
+            for (long j = 0; j < dv; ++j) {
+                double acc = 0.0;
+                for (long c = 0; c < dk; ++c) acc += qt[c] * S[c * dv + j];
+                ot[j] = acc;
+            }
+        }
+        free(S);
+        free(alpha);
+    }
+    return 0;
+}
+
+/* Backward of the recurrence: a reverse sweep over the scan order carrying
+ * dS = dLoss/dS_t.  The forward states are rebuilt from checkpoints taken every
+ * CK steps.  dlogalpha is the gradient with respect to log(alpha_t); with one
+ * shared gate (gate_heads == 1) it is summed over heads. */
+#define CK 64
+int oracle_gla_bwd(const double *q, const double *k, const double *v, const double *z,
+                   int gate_heads, double inv_tau, const double *dO,
+                   double *dq, double *dk_out, double *dv_out, double *dlogalpha,
+                   long B, long H, long L, long dk, long dv, long Hg, long Wg, int mode)
+{
+    if (check_shape(B, H, L, dk, dv, Hg, Wg, mode, gate_heads)) return 1;
+    long n = B * H;
+    long nblk = (L + CK - 1) / CK;
+    /* per-head dlogalpha, reduced over heads afterwards in a fixed order */
+    double *dla_h = (double *)calloc((size_t)(B * H * L * dk) + 1, sizeof(double));
+    if (!dla_h) return 2;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < n; ++bh) {
+        long b = bh / H, h = bh % H, hz = (gate_heads == 1) ? 0 : h;
+        size_t ssz = (size_t)(dk * dv);
+        double *ckpt = (double *)calloc(ssz * (size_t)(nblk + 1), sizeof(double));
+        double *blk = (double *)malloc(ssz * CK * sizeof(double));
+        double *S = (double *)calloc(ssz, sizeof(double));
+        double *dS = (double *)calloc(ssz, sizeof(double));
+        double *alpha = (double *)malloc((size_t)dk * sizeof(double));
+        /* forward sweep: ckpt[m] = state before the first token of block m */
+        for (long t = 0; t < L; ++t) {
+            if (t % CK == 0) memcpy(ckpt + (size_t)(t / CK) * ssz, S, ssz * sizeof(double));
+            long g = oracle_scan_index(mode, Hg, Wg, t);
+            const double *kt = k + ((b * L + g) * H + h) * dk;
+            const double *vt = v + ((b * L + g) * H + h) * dv;
+            const double *zt = z + ((b * L + g) * gate_heads + hz) * dk;
+            for (long c = 0; c < dk; ++c) {
+                double a = exp(inv_tau * log_sigmoid(zt[c]));
+                for (long j = 0; j < dv; ++j) S[c * dv + j] = a * S[c * dv + j] + kt[c] * vt[j];
+            }
+        }
+        /* reverse sweep */
+        for (long m = nblk - 1; m >= 0; --m) {
+            long t0 = m * CK, t1 = (t0 + CK < L) ? t0 + CK : L;
+            /* rebuild S_t for t in [t0, t1) */
+            memcpy(S, ckpt + (size_t)m * ssz, ssz * sizeof(double));
+            for (long t = t0; t < t1; ++t) {
+                long g = oracle_scan_index(mode, Hg, Wg, t);
+                const double *kt = k + ((b * L + g) * H + h) * dk;
+                const double *vt = v + ((b * L + g) * H + h) * dv;
+                const double *zt = z + ((b * L + g) * gate_heads + hz) * dk;
+                for (long c = 0; c < dk; ++c) {
+                    double a = exp(inv_tau * log_sigmoid(zt[c]));
+                    for (long j = 0; j < dv; ++j) S[c * dv + j] = a * S[c * dv + j] + kt[c] * vt[j];
+                }
+                memcpy(blk + (size_t)(t - t0) * ssz, S, ssz * sizeof(double));
+            }
+            for (long t = t1 - 1; t >= t0; --t) {
+                long g = oracle_scan_index(mode, Hg, Wg, t);
+                const double *qt = q + ((b * L + g) * H + h) * dk;
+                const double *kt = k + ((b * L + g) * H + h) * dk;
+                const double *vt = v + ((b * L + g) * H + h) * dv;
+                const double *zt = z + ((b * L + g) * gate_heads + hz) * dk;
+                const double *dot = dO + ((b * L + g) * H + h) * dv;
+                const double *St = blk + (size_t)(t - t0) * ssz;
+                const double *Sp = (t > t0) ? blk + (size_t)(t - 1 - t0) * ssz
+                                            : ckpt + (size_t)m * ssz;
+                double *dqt = dq + ((b * L + g) * H + h) * dk;
+                double *dkt = dk_out + ((b * L + g) * H + h) * dk;
+                double *dvt = dv_out + ((b * L + g) * H + h) * dv;
+                double *dlat = dla_h + ((b * H + h) * L + g) * dk;
+                for (long c = 0; c < dk; ++c) alpha[c] = exp(inv_tau * log_sigmoid(zt[c]));
+                /* dS_t = q_t^T dO_t + (carried gradient from S_{t+1}) */
+                for (long c = 0; c < dk; ++c)
+                    for (long j = 0; j < dv; ++j) dS[c * dv + j] += qt[c] * dot[j];
+                /* dq_t = dO_t S_t^T */
+                for (long c = 0; c < dk; ++c) {
+                    double acc = 0.0;
+                    for (long j = 0; j < dv; ++j) acc += dot[j] * St[c * dv + j];
+                    dqt[c] = acc;
+                }
+                /* dk_t = v_t dS_t^T,  dv_t = k_t dS_t */
+                for (long c = 0; c < dk; ++c) {
+                    double acc = 0.0;
+                    for (long j = 0; j < dv; ++j) acc += dS[c * dv + j] * vt[j];
+                    dkt[c] = acc;
+                }
+                for (long j = 0; j < dv; ++j) {
+                    double acc = 0.0;
+                    for (long c = 0; c < dk; ++c) acc += kt[c] * dS[c * dv + j];
+                    dvt[j] = acc;
+                }
+                /* dLoss/dlog(alpha_t)[c] = alpha_t[c] * sum_j dS_t[c,j] S_{t-1}[c,j] */
+                for (long c = 0; c < dk; ++c) {
+                    double acc = 0.0;
+                    for (long j = 0; j < dv; ++j) acc += dS[c * dv + j] * Sp[c * dv + j];
+                    dlat[c] = alpha[c] * acc;
+                }
+                /* gradient carried to S_{t-1} */
+                for (long c = 0; c < dk; ++c)
+                    for (long j = 0; j < dv; ++j) dS[c * dv + j] *= alpha[c];
+            }
+        }
+        free(ckpt); free(blk); free(S); free(dS); free(alpha);
+    }
+    /* scatter / reduce per-head values into the gate layout */
+    for (long b = 0; b < B; ++b)
+        for (long g = 0; g < L; ++g) {
+            if (gate_heads == 1) {
+                double *dst = dlogalpha + (b * L + g) * dk;
+                for (long c = 0; c < dk; ++c) {
+                    double acc = 0.0;
+                    for (long h = 0; h < H; ++h) acc += dla_h[((b * H + h) * L + g) * dk + c];
+                    dst[c] = acc;
+                }
+            } else {
+                for (long h = 0; h < H; ++h)
+                    memcpy(dlogalpha + ((b * L + g) * H + h) * dk,
+                           dla_h + ((b * H + h) * L + g) * dk, (size_t)dk * sizeof(double));
+            }
+        }
+    free(dla_h);
+    return 0;
+}
+
+/* y = Swish(r) * RMSNorm(o) * gamma, the norm taken over the d_v features of
+ * one (token, head) row (slide eq. (9)-(10)).  gamma may be NULL (all ones). */
+int oracle_epilogue(const double *o, const double *r, const double *gamma, double eps,
+                    double *y, long rows, long dv)
+{
+    if (rows < 0 || dv <= 0) return 1;
+#pragma omp parallel for schedule(static)
+    for (long i = 0; i < rows; ++i) {
+        const double *oi = o + i * dv, *ri = r + i * dv;
+        double ms = 0.0;
+        for (long j = 0; j < dv; ++j) ms += oi[j] * oi[j];
+        double inv = 1.0 / sqrt(ms / (double)dv + eps);
+        for (long j = 0; j < dv; ++j) {
+            double sw = ri[j] / (1.0 + exp(-ri[j]));
+            y[i * dv + j] = sw * oi[j] * inv * (gamma ? gamma[j] : 1.0);
+        }
+    }
+    return 0;
+}
+
+/* SREM: 3x3 depthwise cross-correlation with zero "same" padding on the grid,
+ * result written in scan order: y[b][t][ch] = conv(x)[b][grid(t)][ch]. */
+int oracle_srem_dwconv(const double *x, const double *w, const double *bias, double *y,
+                       long B, long Hg, long Wg, long C, int mode)
+{
+    if (B < 0 || Hg < 0 || Wg < 0 || C <= 0 || mode < 0 || mode > 3) return 1;
+    long L = Hg * Wg;
+#pragma omp parallel for schedule(static)
+    for (long bt = 0; bt < B * L; ++bt) {
+        long b = bt / L, t = bt % L;
+        long g = oracle_scan_index(mode, Hg, Wg, t);
+        long r0 = g / Wg, c0 = g % Wg;
+        for (long ch = 0; ch < C; ++ch) {
+            double acc = bias ? bias[ch] : 0.0;
+            for (long di = -1; di <= 1; ++di)
+                for (long dj = -1; dj <= 1; ++dj) {
+                    long rr = r0 + di, cc = c0 + dj;
+                    if (rr < 0 || rr >= Hg || cc < 0 || cc >= Wg) continue;
+                    acc += w[ch * 9 + (di + 1) * 3 + (dj + 1)] * x[((b * Hg + rr) * Wg + cc) * C + ch];
+                }
+            y[(b * L + t) * C + ch] = acc;
+        }
+    }
+    return 0;
+}
