@@ -1,0 +1,247 @@
+// dig_api.cu -- the C ABI of libdig.so (include/dig.h): argument validation,
+// work decomposition, workspace layout, launches.  No allocation, no
+// synchronisation (except dig_read_status), no device state kept.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/dig.h"
+#include "dig_common.cuh"
+#include "gla.h"
+
+namespace dig {
+
+static thread_local char g_last_error[512] = "";
+
+static dig_status fail(dig_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+WsLayout ws_layout(int nseq, int nseg, int nchunks, int dk, int dv, bool backward) {
+  const size_t dkp = (size_t)((dk + 15) / 16 * 16);
+  const size_t nrec = (size_t)nseq * nseg;
+  WsLayout w{};
+  size_t off = sizeof(WsHeader);
+  w.flags = off;
+  off = align_up(off + nrec * 4, 256);
+  w.flags2 = off;
+  off = align_up(off + (backward ? nrec * 4 : 0), 256);
+  w.seg_gam = off;
+  off = align_up(off + nrec * dkp * 4, 256);
+  w.seg_S = off;
+  off = align_up(off + nrec * (size_t)dk * dv * 4, 256);
+  w.seg_H = off;
+  off = align_up(off + (backward ? nrec * (size_t)dk * dv * 4 : 0), 256);
+  w.chunk_S = off;
+  off = align_up(off + (backward ? (size_t)nseq * nchunks * dk * dv * 4 : 0), 256);
+  w.chunk_B = off;
+  off = align_up(off + (backward ? (size_t)nseq * nchunks * dkp * 4 : 0), 256);
+  w.total = off;
+  return w;
+}
+
+namespace {
+
+constexpr int kMaxDev = 64;
+int g_sms[kMaxDev];
+
+int device_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return 148;
+  if (g_sms[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    g_sms[dev] = n;
+  }
+  return g_sms[dev];
+}
+
+int chunk_len(int dtype) { return dtype == DIG_BF16 ? 128 : 64; }
+
+// Segments per sequence: enough CTAs to cover the SMs once (one resident CTA
+// per SM), never more than the sequence has chunks.
+int choose_nseg(int nseq, int nchunks) {
+  const int slots = device_sms();  // kernels run one CTA per SM
+  if (nseq >= slots || nchunks <= 1) return 1;
+  int nseg = slots / nseq;
+  if (nseg > nchunks) nseg = nchunks;
+  return nseg < 1 ? 1 : nseg;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+dig_status check_common(int B, int H, int L, int d_k, int d_v, int grid_h, int grid_w, int scan_mode, int dtype,
+                        int out_dtype, int gate_heads) {
+  if (B < 0 || H <= 0 || L < 0 || grid_h < 0 || grid_w < 0)
+    return fail(DIG_ERR_INVALID_ARGUMENT, "negative or zero size (B=%d H=%d L=%d grid=%dx%d)", B, H, L, grid_h, grid_w);
+  if ((long long)grid_h * grid_w != L)
+    return fail(DIG_ERR_INVALID_ARGUMENT, "L=%d is not grid_h*grid_w=%d*%d", L, grid_h, grid_w);
+  if (scan_mode < 0 || scan_mode > 3) return fail(DIG_ERR_INVALID_ARGUMENT, "scan_mode %d not in 0..3", scan_mode);
+  if ((dtype != DIG_F32 && dtype != DIG_BF16) || (out_dtype != DIG_F32 && out_dtype != DIG_BF16))
+    return fail(DIG_ERR_INVALID_ARGUMENT, "dtype %d / out_dtype %d not DIG_F32 or DIG_BF16", dtype, out_dtype);
+  if (gate_heads != 1 && gate_heads != H)
+    return fail(DIG_ERR_INVALID_ARGUMENT, "gate_heads=%d must be 1 or H=%d", gate_heads, H);
+  if (d_k <= 0 || d_v <= 0) return fail(DIG_ERR_INVALID_ARGUMENT, "head dims must be positive");
+  if (!gla_variant_built(d_k, d_v))
+    return fail(DIG_ERR_UNSUPPORTED, "(d_k, d_v) = (%d, %d) is not built (supported: (32,64), (36,72), (64,64))", d_k,
+                d_v);
+  if ((long long)B * L * H * (d_k > d_v ? d_k : d_v) >= (1ll << 40))
+    return fail(DIG_ERR_INVALID_ARGUMENT, "tensor too large");
+  return DIG_OK;
+}
+
+}  // namespace
+}  // namespace dig
+
+using namespace dig;
+
+extern "C" {
+
+int dig_gla_supported(int d_k, int d_v) { return gla_variant_built(d_k, d_v) ? 1 : 0; }
+
+size_t dig_gla_workspace_bytes(int B, int H, int L, int d_k, int d_v, int pass) {
+  if (B < 0 || H <= 0 || L < 0 || d_k <= 0 || d_v <= 0 || (pass != 0 && pass != 1)) return 0;
+  const int nseq = B * H;
+  // sized for the larger chunk count (fp32 inputs use shorter chunks)
+  const int nchunks = (L + 63) / 64;
+  const int nseg = choose_nseg(nseq > 0 ? nseq : 1, nchunks);
+  return ws_layout(nseq > 0 ? nseq : 1, nseg, nchunks, d_k, d_v, pass == 1).total;
+}
+
+dig_status dig_gla_fwd(const void* q, const void* k, const void* v, const float* z, int gate_heads, float inv_tau,
+                       void* o, const void* r, const float* gamma, float eps, void* y, int B, int H, int L, int d_k,
+                       int d_v, int grid_h, int grid_w, int scan_mode, int dtype, int out_dtype, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  dig_status st = check_common(B, H, L, d_k, d_v, grid_h, grid_w, scan_mode, dtype, out_dtype, gate_heads);
+  if (st != DIG_OK) return st;
+  if (!workspace) return fail(DIG_ERR_INVALID_ARGUMENT, "workspace is NULL");
+  if (!aligned16(workspace)) return fail(DIG_ERR_MISALIGNED, "workspace not 16-byte aligned");
+  if (B == 0 || L == 0) return DIG_OK;
+  if (!q || !k || !v || !z || !o) return fail(DIG_ERR_INVALID_ARGUMENT, "q, k, v, z and o must be non-NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(z) || !aligned16(o) || !aligned16(r) ||
+      !aligned16(gamma) || !aligned16(y))
+    return fail(DIG_ERR_MISALIGNED, "a tensor pointer is not 16-byte aligned");
+  const int C = chunk_len(dtype);
+  const int nseq = B * H;
+  const int nchunks = (L + C - 1) / C;
+  const int nseg = choose_nseg(nseq, nchunks);
+  const WsLayout lay = ws_layout(nseq, nseg, nchunks, d_k, d_v, false);
+  if (workspace_bytes < lay.total)
+    return fail(DIG_ERR_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, needs %zu", workspace_bytes, lay.total);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  GlaArgs a{};
+  a.q = q; a.k = k; a.v = v; a.z = z; a.r = r; a.gamma = gamma; a.o = o; a.y = y;
+  a.B = B; a.H = H; a.L = L; a.Hg = grid_h; a.Wg = grid_w; a.mode = scan_mode; a.gate_heads = gate_heads;
+  a.inv_tau = inv_tau; a.eps = eps;
+  a.nchunks = nchunks; a.nseg = nseg;
+  a.status = reinterpret_cast<uint32_t*>(ws);
+  a.done = reinterpret_cast<uint32_t*>(ws) + 1;
+  a.flags = reinterpret_cast<uint32_t*>(ws + lay.flags);
+  a.seg_gam = reinterpret_cast<float*>(ws + lay.seg_gam);
+  a.seg_S = reinterpret_cast<float*>(ws + lay.seg_S);
+  GlaVariant var{C, dtype == DIG_BF16 ? 1 : 2, d_k, d_v, dtype, out_dtype};
+  const cudaError_t e = launch_gla_fwd(var, a, nseq * nseg, nseg > 1, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "gla_fwd launch: %s", cudaGetErrorString(e));
+  return DIG_OK;
+}
+
+dig_status dig_gla_bwd(const void* q, const void* k, const void* v, const float* z, int gate_heads, float inv_tau,
+                       const void* dO, void* dq, void* dk, void* dv, float* dlog_alpha, int B, int H, int L, int d_k,
+                       int d_v, int grid_h, int grid_w, int scan_mode, int dtype, int out_dtype, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  dig_status st = check_common(B, H, L, d_k, d_v, grid_h, grid_w, scan_mode, dtype, out_dtype, gate_heads);
+  if (st != DIG_OK) return st;
+  if (!workspace) return fail(DIG_ERR_INVALID_ARGUMENT, "workspace is NULL");
+  if (!aligned16(workspace)) return fail(DIG_ERR_MISALIGNED, "workspace not 16-byte aligned");
+  if (B == 0 || L == 0) return DIG_OK;
+  if (!q || !k || !v || !z || !dO || !dq || !dk || !dv || !dlog_alpha)
+    return fail(DIG_ERR_INVALID_ARGUMENT, "all tensor pointers of the backward must be non-NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(z) || !aligned16(dO) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || !aligned16(dlog_alpha))
+    return fail(DIG_ERR_MISALIGNED, "a tensor pointer is not 16-byte aligned");
+  const int C = chunk_len(dtype);
+  const int nseq = B * H;
+  const int nchunks = (L + C - 1) / C;
+  const int nseg = choose_nseg(nseq, nchunks);
+  const WsLayout lay = ws_layout(nseq, nseg, nchunks, d_k, d_v, true);
+  if (workspace_bytes < lay.total)
+    return fail(DIG_ERR_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, needs %zu", workspace_bytes, lay.total);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (gate_heads == 1) {
+    // heads add their contributions into dlog_alpha
+    const cudaError_t e = cudaMemsetAsync(dlog_alpha, 0, (size_t)B * L * d_k * sizeof(float), s);
+    if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "dlog_alpha clear: %s", cudaGetErrorString(e));
+  }
+  GlaArgs a{};
+  a.q = q; a.k = k; a.v = v; a.z = z; a.dO = dO; a.dq = dq; a.dk = dk; a.dv = dv; a.dla = dlog_alpha;
+  a.B = B; a.H = H; a.L = L; a.Hg = grid_h; a.Wg = grid_w; a.mode = scan_mode; a.gate_heads = gate_heads;
+  a.inv_tau = inv_tau;
+  a.nchunks = nchunks; a.nseg = nseg;
+  a.status = reinterpret_cast<uint32_t*>(ws);
+  a.done = reinterpret_cast<uint32_t*>(ws) + 1;
+  a.flags = reinterpret_cast<uint32_t*>(ws + lay.flags);
+  a.flags2 = reinterpret_cast<uint32_t*>(ws + lay.flags2);
+  a.seg_gam = reinterpret_cast<float*>(ws + lay.seg_gam);
+  a.seg_S = reinterpret_cast<float*>(ws + lay.seg_S);
+  a.seg_H = reinterpret_cast<float*>(ws + lay.seg_H);
+  a.chunk_S = reinterpret_cast<float*>(ws + lay.chunk_S);
+  a.chunk_B = reinterpret_cast<float*>(ws + lay.chunk_B);
+  GlaVariant var{C, dtype == DIG_BF16 ? 1 : 2, d_k, d_v, dtype, out_dtype};
+  const cudaError_t e = launch_gla_bwd(var, a, nseq * nseg, nseg > 1, s);
+  if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "gla_bwd launch: %s", cudaGetErrorString(e));
+  return DIG_OK;
+}
+
+dig_status dig_srem_reorient_dwconv(const void* x, const float* w, const float* bias, void* y, int B, int grid_h,
+                                    int grid_w, int C, int scan_mode, int dtype, int out_dtype, void* stream) {
+  if (B < 0 || grid_h < 0 || grid_w < 0 || C <= 0)
+    return fail(DIG_ERR_INVALID_ARGUMENT, "bad size (B=%d grid=%dx%d C=%d)", B, grid_h, grid_w, C);
+  if (scan_mode < 0 || scan_mode > 3) return fail(DIG_ERR_INVALID_ARGUMENT, "scan_mode %d not in 0..3", scan_mode);
+  if ((dtype != DIG_F32 && dtype != DIG_BF16) || (out_dtype != DIG_F32 && out_dtype != DIG_BF16))
+    return fail(DIG_ERR_INVALID_ARGUMENT, "dtype %d / out_dtype %d not DIG_F32 or DIG_BF16", dtype, out_dtype);
+  if ((long long)B * grid_h * grid_w * C >= (1ll << 40)) return fail(DIG_ERR_INVALID_ARGUMENT, "tensor too large");
+  if (B == 0 || grid_h == 0 || grid_w == 0) return DIG_OK;
+  if (!x || !w || !y) return fail(DIG_ERR_INVALID_ARGUMENT, "x, w and y must be non-NULL");
+  if (!aligned16(x) || !aligned16(y) || !aligned16(w) || !aligned16(bias))
+    return fail(DIG_ERR_MISALIGNED, "a tensor pointer is not 16-byte aligned");
+  const cudaError_t e =
+      launch_srem(x, w, bias, y, B, grid_h, grid_w, C, scan_mode, dtype, out_dtype, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "srem launch: %s", cudaGetErrorString(e));
+  return DIG_OK;
+}
+
+dig_status dig_read_status(void* workspace, void* stream) {
+  if (!workspace) return fail(DIG_ERR_INVALID_ARGUMENT, "workspace is NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t host = 0;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemcpy(&host, workspace, sizeof(host), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && host != 0) e = cudaMemset(workspace, 0, sizeof(uint32_t));
+  if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "read status: %s", cudaGetErrorString(e));
+  return static_cast<dig_status>(host);
+}
+
+const char* dig_status_string(dig_status s) {
+  switch (s) {
+    case DIG_OK: return "ok";
+    case DIG_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case DIG_ERR_UNSUPPORTED: return "unsupported configuration";
+    case DIG_ERR_MISALIGNED: return "misaligned pointer";
+    case DIG_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case DIG_ERR_CUDA: return "CUDA error";
+    case DIG_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case DIG_ERR_GATE_RANGE: return "gate decay outside the chunked factorisation's range";
+    default: return "unknown status";
+  }
+}
+
+const char* dig_last_error(void) { return g_last_error; }
+
+}  // extern "C"

@@ -1,0 +1,149 @@
+"""Thin ctypes binding of libdig.so (include/dig.h).
+
+Argument marshalling only: tensors are passed as raw device pointers with their
+sizes and the current CUDA stream; every step of the computation runs in the
+library's sm_100a kernels.  Importing this module fails loudly when libdig.so
+has not been built -- there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdig.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "dig.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError("libdig.so is not built; run `python -m gated_linear_attention_fwd_b200.build` "
+                      "(or __graft_entry__.build()) first")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+DIG_OK = 0
+DIG_ERR_INVALID_ARGUMENT = 1
+DIG_ERR_UNSUPPORTED = 2
+DIG_ERR_MISALIGNED = 3
+DIG_ERR_WORKSPACE_TOO_SMALL = 4
+DIG_ERR_CUDA = 5
+DIG_ERR_DEVICE_TIMEOUT = 6
+DIG_ERR_GATE_RANGE = 7
+
+DIG_F32 = 0
+DIG_BF16 = 1
+
+SCAN_ROW_FWD, SCAN_ROW_REV, SCAN_COL_FWD, SCAN_COL_REV = 0, 1, 2, 3
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+_sz = ctypes.c_size_t
+
+lib.dig_gla_supported.restype = _i
+lib.dig_gla_supported.argtypes = [_i, _i]
+lib.dig_gla_workspace_bytes.restype = _sz
+lib.dig_gla_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
+lib.dig_gla_fwd.restype = _i
+lib.dig_gla_fwd.argtypes = [_vp, _vp, _vp, _vp, _i, _f, _vp, _vp, _vp, _f, _vp,
+                            _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]
+lib.dig_gla_bwd.restype = _i
+lib.dig_gla_bwd.argtypes = [_vp, _vp, _vp, _vp, _i, _f, _vp, _vp, _vp, _vp, _vp,
+                            _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]
+lib.dig_srem_reorient_dwconv.restype = _i
+lib.dig_srem_reorient_dwconv.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
+lib.dig_read_status.restype = _i
+lib.dig_read_status.argtypes = [_vp, _vp]
+lib.dig_status_string.restype = ctypes.c_char_p
+lib.dig_status_string.argtypes = [_i]
+lib.dig_last_error.restype = ctypes.c_char_p
+lib.dig_last_error.argtypes = []
+
+
+class DigError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib.dig_last_error().decode(errors="replace")
+        super().__init__("%s: %s (%d)%s" % (where, lib.dig_status_string(status).decode(), status,
+                                            (": " + msg) if msg else ""))
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/dig.h declares."""
+    src = open(HEADER_PATH).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dig_[a-z0-9_]+)\s*\(", src)))
+
+
+def _code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return DIG_F32
+    if dt == torch.bfloat16:
+        return DIG_BF16
+    raise TypeError("unsupported dtype %s (float32 or bfloat16)" % dt)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(st, where):
+    if st != DIG_OK:
+        raise DigError(st, where)
+
+
+def gla_workspace_bytes(B, H, L, d_k, d_v, backward=False) -> int:
+    return int(lib.dig_gla_workspace_bytes(B, H, L, d_k, d_v, 1 if backward else 0))
+
+
+def new_workspace(B, H, L, d_k, d_v, backward=False, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace (uint8) sized for dig_gla_fwd / dig_gla_bwd."""
+    n = gla_workspace_bytes(B, H, L, d_k, d_v, backward)
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def dig_gla_fwd(q, k, v, z, inv_tau, o, grid_h, grid_w, scan_mode, workspace,
+                r=None, gamma=None, eps=1e-5, y=None, stream=None):
+    """q,k [B,L,H,dk]; v,o [B,L,H,dv]; z [B,L,gate_heads,dk] fp32 (see include/dig.h)."""
+    B, L, H, dk = q.shape
+    dv = v.shape[3]
+    st = lib.dig_gla_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(z), z.shape[2], float(inv_tau), _ptr(o),
+                         _ptr(r), _ptr(gamma), float(eps), _ptr(y),
+                         B, H, L, dk, dv, grid_h, grid_w, scan_mode, _code(q.dtype), _code(o.dtype),
+                         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "dig_gla_fwd")
+
+
+def dig_gla_bwd(q, k, v, z, inv_tau, dO, dq, dk, dv, dlog_alpha, grid_h, grid_w, scan_mode, workspace,
+                stream=None):
+    B, L, H, d_k = q.shape
+    d_v = v.shape[3]
+    st = lib.dig_gla_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(z), z.shape[2], float(inv_tau), _ptr(dO),
+                         _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlog_alpha),
+                         B, H, L, d_k, d_v, grid_h, grid_w, scan_mode, _code(q.dtype), _code(dq.dtype),
+                         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "dig_gla_bwd")
+
+
+def dig_srem_reorient_dwconv(x, w, bias, y, scan_mode, stream=None):
+    """x [B,Hg,Wg,C] grid order; w [C,3,3] fp32; bias [C] fp32 or None; y [B,L,C] scan order."""
+    B, Hg, Wg, C = x.shape
+    st = lib.dig_srem_reorient_dwconv(_ptr(x), _ptr(w), _ptr(bias), _ptr(y), B, Hg, Wg, C, scan_mode,
+                                      _code(x.dtype), _code(y.dtype), _stream(stream))
+    _check(st, "dig_srem_reorient_dwconv")
+
+
+def dig_read_status(workspace, stream=None) -> int:
+    return int(lib.dig_read_status(_ptr(workspace), _stream(stream)))

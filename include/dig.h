@@ -1,0 +1,140 @@
+/*
+ * dig.h -- C ABI of the B200 (sm_100a) DiG token mixer: chunkwise Gated Linear
+ * Attention forward and backward, and the SREM reorient + 3x3 depthwise conv.
+ *
+ * Source of the operations ("DiG: Scalable and Efficient Diffusion Models with
+ * Gated Linear Attention"; docswell study-group slides, page 2 of the reference
+ * set, and the volcengine translation of the paper, page 3):
+ *   GLA        slide "Gated Linear Attention Transformer (GLA) の導入", eq. (5)-(8):
+ *              alpha_t = sigmoid(z_t)^(1/tau)        (gate, per key channel)
+ *              S_t = diag(alpha_t) S_{t-1} + k_t^T v_t   (S_0 = 0, d_k x d_v)
+ *              o_t = q_t S_t
+ *   epilogue   same slide, eq. (9)-(10): y_t = Swish(r_t) * RMSNorm(o_t) * gamma
+ *              (the projections X W_r and W_O are outside this library)
+ *   chunking   slide "計算効率の分析" / paper "Efficiency Analysis": the sequence is
+ *              split into chunks that fit on-chip memory
+ *   SREM       slide "SREM (Spatial Reorient & Enhancement Module) の導入" and the
+ *              paper's "DiG Block" section: 3x3 depthwise conv on the 2-D token grid
+ *              and one of four scan orders (transpose / flip)
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *     never allocates, frees or keeps device memory, and never synchronises
+ *     (except dig_read_status).  Work is enqueued on `stream` (a cudaStream_t;
+ *     NULL = legacy default stream) and the call returns without waiting.
+ *   - Tensors are dense, row-major, tokens in GRID row-major order
+ *     (token g = row * grid_w + col, L = grid_h * grid_w).  Pointers must be
+ *     16-byte aligned.
+ *   - Element types: `dtype` is the storage type of q, k, v, dO, r and of the
+ *     conv input x (DIG_F32 or DIG_BF16); `out_dtype` is the storage type of o,
+ *     y, dq, dk, dv and the conv output.  z, dlog_alpha, gamma, the conv weights
+ *     and bias are always fp32.  Arithmetic is fp32 (tensor-core products in tf32
+ *     with fp32 accumulation; three-term split tf32 when dtype == DIG_F32).
+ *   - Errors in the arguments are reported synchronously and nothing is
+ *     launched.  A failed launch returns DIG_ERR_CUDA.  Conditions found on the
+ *     device (a bounded wait that ran out, a gate outside the supported range)
+ *     are recorded in a status word inside the workspace; read it with
+ *     dig_read_status.  dig_last_error() gives a message for the last failure
+ *     of the calling thread.
+ */
+#ifndef DIG_H_
+#define DIG_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int dig_status;
+enum {
+  DIG_OK = 0,
+  DIG_ERR_INVALID_ARGUMENT = 1,   /* bad shape, pointer, mode or dtype             */
+  DIG_ERR_UNSUPPORTED = 2,        /* valid but not built (head dims, see below)      */
+  DIG_ERR_MISALIGNED = 3,         /* a pointer is not 16-byte aligned                */
+  DIG_ERR_WORKSPACE_TOO_SMALL = 4,
+  DIG_ERR_CUDA = 5,               /* a CUDA call failed (launch, attribute query)    */
+  DIG_ERR_DEVICE_TIMEOUT = 6,     /* device status: a bounded inter-CTA wait ran out  */
+  DIG_ERR_GATE_RANGE = 7          /* device status: a chunk's gate decay left the
+                                     exponent range of the chunked factorisation      */
+};
+
+/* Scan orders (DiG scanning directions; layer l of the model uses mode l % 4).
+ * Scan position t visits grid token g = pi(t):
+ *   ROW_FWD  pi(t) = t                    ROW_REV  pi(t) = L-1-t
+ *   COL_FWD  pi(t) = (t % grid_h) * grid_w + t / grid_h
+ *   COL_REV  pi(t) = COL_FWD(L-1-t)                                          */
+enum { DIG_SCAN_ROW_FWD = 0, DIG_SCAN_ROW_REV = 1, DIG_SCAN_COL_FWD = 2, DIG_SCAN_COL_REV = 3 };
+
+enum { DIG_F32 = 0, DIG_BF16 = 1 };
+
+/* Head dimensions built into this library: (d_k, d_v) in
+ * {(32,64), (36,72), (64,64)}; any other pair returns DIG_ERR_UNSUPPORTED. */
+int dig_gla_supported(int d_k, int d_v);
+
+/* Bytes of device workspace dig_gla_fwd (pass = 0) or dig_gla_bwd (pass = 1)
+ * needs for this shape on the current device.  The workspace must be
+ * zero-filled before its first use; every call that ends with status DIG_OK
+ * leaves it ready for the next call (no re-zeroing needed).  After a device
+ * status other than DIG_OK, zero it again.  Calls that may run concurrently
+ * need separate workspaces.  Returns 0 for invalid shapes. */
+size_t dig_gla_workspace_bytes(int B, int H, int L, int d_k, int d_v, int pass);
+
+/* GLA forward (slide eq. (5)-(8), chunkwise).
+ *   q, k   [B, L, H, d_k]   dtype        queries / keys (no extra 1/sqrt(d) scale)
+ *   v      [B, L, H, d_v]   dtype
+ *   z      [B, L, gate_heads, d_k] fp32  gate logits; alpha = exp(inv_tau*logsigmoid(z));
+ *                                        gate_heads is 1 (one gate shared by all heads)
+ *                                        or H
+ *   o      [B, L, H, d_v]   out_dtype    o_t = q_t S_t, written at the token's grid slot
+ *   r      [B, L, H, d_v]   dtype        optional (NULL): output-gate input
+ *   gamma  [d_v] fp32                    optional (NULL = ones): RMSNorm weight
+ *   y      [B, L, H, d_v]   out_dtype    optional: Swish(r) * o / sqrt(mean(o^2)+eps) * gamma;
+ *                                        written only when both r and y are non-NULL
+ * The recurrence runs in the scan order `scan_mode` over the grid_h x grid_w
+ * grid; no reordered copy of any tensor is written. */
+dig_status dig_gla_fwd(const void *q, const void *k, const void *v, const float *z,
+                       int gate_heads, float inv_tau, void *o,
+                       const void *r, const float *gamma, float eps, void *y,
+                       int B, int H, int L, int d_k, int d_v, int grid_h, int grid_w,
+                       int scan_mode, int dtype, int out_dtype,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/* GLA backward: gradients of sum(o * dO) for the forward above.
+ *   dO          [B, L, H, d_v]  dtype
+ *   dq, dk      [B, L, H, d_k]  out_dtype
+ *   dv          [B, L, H, d_v]  out_dtype
+ *   dlog_alpha  [B, L, gate_heads, d_k] fp32: dLoss/dlog(alpha), summed over heads
+ *               when gate_heads == 1.  The gradient of the logits is
+ *               dz = dlog_alpha * inv_tau * sigmoid(-z) (left to the caller).
+ * When gate_heads == 1 the heads' contributions to dlog_alpha are added with
+ * floating-point atomics, so its last bits may differ between runs. */
+dig_status dig_gla_bwd(const void *q, const void *k, const void *v, const float *z,
+                       int gate_heads, float inv_tau, const void *dO,
+                       void *dq, void *dk, void *dv, float *dlog_alpha,
+                       int B, int H, int L, int d_k, int d_v, int grid_h, int grid_w,
+                       int scan_mode, int dtype, int out_dtype,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/* SREM reorient + 3x3 depthwise conv (zero "same" padding, cross-correlation as
+ * in a depthwise nn.Conv2d):
+ *   x     [B, grid_h, grid_w, C] dtype, grid order
+ *   w     [C, 3, 3] fp32;  bias [C] fp32 or NULL
+ *   y     [B, L, C] out_dtype, in SCAN order: y[b, t] = conv(x)[b, pi(t)]
+ * With the identity kernel (centre tap 1) this is exactly the reorient
+ * permutation. */
+dig_status dig_srem_reorient_dwconv(const void *x, const float *w, const float *bias, void *y,
+                                    int B, int grid_h, int grid_w, int C, int scan_mode,
+                                    int dtype, int out_dtype, void *stream);
+
+/* Synchronises `stream`, returns the device status word kept in `workspace`
+ * (DIG_OK, DIG_ERR_DEVICE_TIMEOUT or DIG_ERR_GATE_RANGE) and clears it. */
+dig_status dig_read_status(void *workspace, void *stream);
+
+const char *dig_status_string(dig_status s);
+const char *dig_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DIG_H_ */
