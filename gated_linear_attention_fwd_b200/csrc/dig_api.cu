@@ -62,7 +62,8 @@ int device_sms() {
   return g_sms[dev];
 }
 
-int chunk_len(int dtype) { return dtype == DIG_BF16 ? 128 : 64; }
+// Tokens per chunk: forward 128 (bf16 inputs) / 64 (fp32); backward 64 / 32.
+int chunk_len(int dtype, bool backward) { return (dtype == DIG_BF16 ? 128 : 64) >> (backward ? 1 : 0); }
 
 // Segments per sequence: enough CTAs to cover the SMs once (one resident CTA
 // per SM), never more than the sequence has chunks.
@@ -108,8 +109,8 @@ int dig_gla_supported(int d_k, int d_v) { return gla_variant_built(d_k, d_v) ? 1
 size_t dig_gla_workspace_bytes(int B, int H, int L, int d_k, int d_v, int pass) {
   if (B < 0 || H <= 0 || L < 0 || d_k <= 0 || d_v <= 0 || (pass != 0 && pass != 1)) return 0;
   const int nseq = B * H;
-  // sized for the larger chunk count (fp32 inputs use shorter chunks)
-  const int nchunks = (L + 63) / 64;
+  // sized for the largest chunk count (fp32 inputs use shorter chunks)
+  const int nchunks = pass == 1 ? (L + 31) / 32 : (L + 63) / 64;
   const int nseg = choose_nseg(nseq > 0 ? nseq : 1, nchunks);
   return ws_layout(nseq > 0 ? nseq : 1, nseg, nchunks, d_k, d_v, pass == 1).total;
 }
@@ -127,7 +128,7 @@ dig_status dig_gla_fwd(const void* q, const void* k, const void* v, const float*
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(z) || !aligned16(o) || !aligned16(r) ||
       !aligned16(gamma) || !aligned16(y))
     return fail(DIG_ERR_MISALIGNED, "a tensor pointer is not 16-byte aligned");
-  const int C = chunk_len(dtype);
+  const int C = chunk_len(dtype, false);
   const int nseq = B * H;
   const int nchunks = (L + C - 1) / C;
   const int nseg = choose_nseg(nseq, nchunks);
@@ -165,7 +166,7 @@ dig_status dig_gla_bwd(const void* q, const void* k, const void* v, const float*
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(z) || !aligned16(dO) || !aligned16(dq) ||
       !aligned16(dk) || !aligned16(dv) || !aligned16(dlog_alpha))
     return fail(DIG_ERR_MISALIGNED, "a tensor pointer is not 16-byte aligned");
-  const int C = chunk_len(dtype);
+  const int C = chunk_len(dtype, true);
   const int nseq = B * H;
   const int nchunks = (L + C - 1) / C;
   const int nseg = choose_nseg(nseq, nchunks);

@@ -1,0 +1,115 @@
+// gla_common.cuh -- device helpers shared by the GLA forward and backward
+// kernels: compile-time sizes, split-term bf16 operand stores, prefetch vectors,
+// the base-2 gate, and the tensor-core issue loop.
+#pragma once
+#include <cstring>
+#include <type_traits>
+
+#include "dig_common.cuh"
+#include "sm100.cuh"
+
+namespace dig {
+
+__host__ __device__ constexpr int cround(int x, int m) { return (x + m - 1) / m * m; }
+__host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
+__host__ __device__ constexpr int pow2ceil(int x) {
+  int p = 32;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+// Store one operand value as NT bf16 terms (term i in copy i).
+template <int NT>
+__device__ __forceinline__ void st_op(uint8_t* base, int copy_bytes, uint32_t off, float x) {
+#pragma unroll
+  for (int i = 0; i < NT; ++i) {
+    const __nv_bfloat16 hb = __float2bfloat16_rn(x);
+    *reinterpret_cast<__nv_bfloat16*>(base + i * copy_bytes + off) = hb;
+    x -= __bfloat162float(hb);
+  }
+}
+// Four consecutive K values of one row (8 bytes per term, same core-matrix row).
+template <int NT>
+__device__ __forceinline__ void st_op4(uint8_t* base, int copy_bytes, uint32_t off, float x0, float x1, float x2,
+                                       float x3) {
+#pragma unroll
+  for (int i = 0; i < NT; ++i) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(x0, x1);
+    const __nv_bfloat162 b = __floats2bfloat162_rn(x2, x3);
+    uint2 u;
+    u.x = *reinterpret_cast<const uint32_t*>(&a);
+    u.y = *reinterpret_cast<const uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(base + i * copy_bytes + off) = u;
+    x0 -= __low2float(a);
+    x1 -= __high2float(a);
+    x2 -= __low2float(b);
+    x3 -= __high2float(b);
+  }
+}
+
+// Raw 4-element vectors as fetched from global memory (prefetched in registers).
+template <typename T>
+struct Raw4;
+template <>
+struct Raw4<__nv_bfloat16> {
+  using type = uint2;
+};
+template <>
+struct Raw4<float> {
+  using type = float4;
+};
+__device__ __forceinline__ void unpack4(const uint2& u, float* o) {
+  o[0] = __uint_as_float(u.x << 16);
+  o[1] = __uint_as_float(u.x & 0xFFFF0000u);
+  o[2] = __uint_as_float(u.y << 16);
+  o[3] = __uint_as_float(u.y & 0xFFFF0000u);
+}
+__device__ __forceinline__ void unpack4(const float4& u, float* o) {
+  o[0] = u.x;
+  o[1] = u.y;
+  o[2] = u.z;
+  o[3] = u.w;
+}
+template <typename R>
+__device__ __forceinline__ R zero4() {
+  R r;
+  memset(&r, 0, sizeof(R));
+  return r;
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+// Base-2 log decay of one gate logit: inv_tau * log2(sigmoid(z)), evaluated as
+// inv_tau * (min(z, 0) * log2(e) - log2(1 + 2^(-|z| log2(e)))).
+__device__ __forceinline__ float log2_decay(float z, float inv_tau) {
+  return inv_tau * (fminf(z, 0.f) * kLog2e - log2f(1.f + exp2f(-fabsf(z) * kLog2e)));
+}
+
+// Issues D (+)= A * B for operands stored as NA / NB bf16 terms: every term
+// pair (i, j) with i + j below max(NA, NB), KSTEPS K-steps each.  Descriptors
+// are formed once; later K-steps and terms only add to the start-address field
+// (shared-memory addresses stay below 2^18, so the 14-bit field never carries).
+template <int NA, int NB, int KSTEPS>
+__device__ __forceinline__ void mma_issue(uint32_t dtm, uint64_t a0, uint32_t a_term, uint32_t a_kstep, uint64_t b0,
+                                          uint32_t b_term, uint32_t b_kstep, uint32_t idesc, bool accumulate) {
+  constexpr int ORD = NA > NB ? NA : NB;
+  bool first = !accumulate;
+#pragma unroll
+  for (int i = 0; i < NA; ++i) {
+#pragma unroll
+    for (int j = 0; j < NB; ++j) {
+      if (i + j >= ORD) continue;
+#pragma unroll
+      for (int s = 0; s < KSTEPS; ++s) {
+        mma_bf16(dtm, a0 + (uint64_t)((i * a_term + s * a_kstep) >> 4), b0 + (uint64_t)((j * b_term + s * b_kstep) >> 4),
+                 idesc, first ? 0u : 1u);
+        first = false;
+      }
+    }
+  }
+}
+
+
+// The per-thread program.  Threads 0-127 own channel half 0, threads 128-255
+// half 1 (compile-time H); both halves run the same barrier sequence.
+
+}  // namespace dig

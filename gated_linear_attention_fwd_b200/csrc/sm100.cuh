@@ -3,16 +3,14 @@
 // (kind::tf32, one CTA), tcgen05.commit / tcgen05.ld, and the shared-memory
 // matrix descriptors of the canonical no-swizzle operand layouts.
 //
-// Operand layout used throughout (tf32 = 4-byte elements, no swizzle):
-//   an R x K operand stored "K-major" is a grid of 8-row x 16-byte core matrices;
-//   element (row, k) lives at byte
-//       (row / 8) * SBO + (k / 4) * LBO + (row % 8) * 16 + (k % 4) * 4
-//   LBO and SBO are free multiples of 16 bytes (chosen per buffer to avoid
-//   shared-memory bank conflicts).  One tf32 MMA consumes K = 8, i.e. two core
-//   matrices along K, so K-step s starts at base + 2 * s * LBO.
-//   Read transposed (rows become K, k becomes M/N) the same bytes form an
-//   "MN-major" operand whose descriptor swaps the two strides; its K-step s (8
-//   rows) starts at base + s * SBO.
+// Operand layout used throughout (no swizzle, "K-major"): an R x K operand is a
+// grid of 8-row x 16-byte core matrices; for 2-byte (bf16) elements, element
+// (row, k) lives at byte
+//     (row / 8) * SBO + (k / 8) * LBO + (row % 8) * 16 + (k % 8) * 2
+// (tf32: k / 4 and (k % 4) * 4).  LBO and SBO are free multiples of 16 bytes,
+// chosen per buffer to avoid shared-memory bank conflicts.  One MMA consumes
+// 32 bytes of K (16 bf16 or 8 tf32), i.e. two core matrices along K, so K-step s
+// starts at base + 2 * s * LBO.
 #pragma once
 #include <cstdint>
 
@@ -39,10 +37,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+      : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
 }
@@ -100,7 +98,24 @@ __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn, bool 
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// D[tmem] (+)= A * B, A: M x K, B: N x K (both from shared memory). One thread issues.
+// Instruction descriptor: kind::f16 with bf16 A and B, fp32 accumulator, dense, K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A * B, A: M x K, B: N x K (both bf16 in shared memory). One thread issues.
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A * B, A: M x K, B: N x K (both tf32 in shared memory). One thread issues.
 __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                          uint32_t accumulate) {
   asm volatile(
@@ -148,9 +163,13 @@ __device__ __forceinline__ float to_tf32(float x) {
   return __uint_as_float(r);
 }
 
-// Byte offset of element (row, k) in a K-major no-swizzle operand.
+// Byte offset of element (row, k) in a K-major no-swizzle operand of tf32.
 __host__ __device__ __forceinline__ uint32_t kmajor_off(uint32_t row, uint32_t k, uint32_t lbo, uint32_t sbo) {
   return (row >> 3) * sbo + (k >> 2) * lbo + (row & 7u) * 16u + (k & 3u) * 4u;
+}
+// Byte offset of element (row, k) in a K-major no-swizzle operand of bf16.
+__host__ __device__ __forceinline__ uint32_t kmaj16(uint32_t row, uint32_t k, uint32_t lbo, uint32_t sbo) {
+  return (row >> 3) * sbo + (k >> 3) * lbo + (row & 7u) * 16u + (k & 7u) * 2u;
 }
 
 }  // namespace dig
