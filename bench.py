@@ -1,0 +1,341 @@
+#!/usr/bin/env python
+"""Benchmark of the DiG GLA token mixer on B200.
+
+One step = the whole hot path over one batch of the DiG-S/2 1792x1792 workload
+(B=2, 112x112 token grid, L=12544, 6 heads, d_k=32, d_v=64, bf16 inputs):
+GLA forward with the fused Swish(r)*RMSNorm(o) epilogue, GLA backward
+(dq, dk, dv, dlog alpha) and the SREM reorient + 3x3 depthwise conv (C=384).
+Step i runs scan mode i % 4, as layer i of DiG would.  Inputs are resident in
+HBM; L2 is flushed (512 MiB write) before every step, outside the timed events.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 the script runs under torchrun, one rank per GPU, each rank an
+independent replica (the path has no data-path collective); time is the max over
+ranks.  Prints one JSON line on rank 0.
+"""
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gated_linear_attention_fwd_b200 import inputs  # noqa: E402
+
+METRIC = "GLA fwd+bwd tokens/s at L=4096/12544/16384; % of roofline (tensor/HBM)"
+WORKLOAD_INDEX = 3  # DiG-S/2 at 1792^2: the configuration that carries every hot-path step
+L2_FLUSH_BYTES = 512 << 20
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def algorithmic_bytes(w):
+    """Bytes each kernel must move once (inputs read once, outputs written once)."""
+    BL, H, dk, dv = w.B * w.L, w.H, w.dk, w.dv
+    e = 2  # bf16 storage
+    qk = BL * H * dk * e
+    vv = BL * H * dv * e
+    z = BL * dk * 4  # one gate shared by the heads, fp32
+    fwd = 2 * qk + vv + z + vv + 2 * vv        # q k v z r in; o y out
+    bwd = 2 * qk + vv + z + vv + 2 * qk + vv + z  # q k v z dO in; dq dk dv dlogalpha out
+    conv = 2 * BL * w.conv_C * e
+    return {"fwd": fwd, "bwd": bwd, "conv": conv}
+
+
+def _src_hash(names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "gated_linear_attention_fwd_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(kernel, srcs, scale):
+    """DRAM bytes per launch from the committed ncu capture, if the kernel is unchanged."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f).get(kernel)
+    if not d or d.get("source_sha") != _src_hash(srcs):
+        return None
+    return float(d["dram_bytes_per_launch"]) * scale
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+        finally:
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows]
+        mx = max(float(r[2]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        loaded = [s for s in sm if s > 0.5 * mx] or sm
+        return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def cpu_sample(w, x, steps=1):
+    """The fp64 oracle on batch element 0 (all heads): forward + epilogue + backward + conv."""
+    import oracle
+    sl = lambda a: a[:1]
+    t0 = time.perf_counter()
+    for i in range(steps):
+        mode = i % 4
+        o = oracle.gla_fwd(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["z"]), w.inv_tau, w.grid_h, w.grid_w, mode)
+        oracle.epilogue(o, sl(x["r"]))
+        oracle.gla_bwd(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["z"]), w.inv_tau, sl(x["dO"]), w.grid_h, w.grid_w,
+                       mode)
+        oracle.srem_dwconv(sl(x["x_conv"]), x["w_conv"], None, mode)
+    dt = time.perf_counter() - t0
+    return w.L * steps / dt, dt, min(w.H, oracle.num_threads())
+
+
+def run_reference(args, rank, world):
+    """The oracle, timed on the host cores, as the reference arm."""
+    w = inputs.WORKLOADS[WORKLOAD_INDEX]
+    if rank != 0:
+        return None
+    x = inputs.make_inputs(w)
+    cpu_sample(w, x, steps=args.warmup)
+    tps, dt, cores = cpu_sample(w, x, steps=args.steps)
+    sample = "oracle (fp64 C, OpenMP over heads) on batch element 0 of %s: fwd+epilogue+bwd+conv, %d tokens/step" % (
+        w.name, w.L)
+    line = {"impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": _config(w, world),
+            "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    return line
+
+
+def _config(w, world):
+    return {"workload": "%s: B=%d, %dx%d token grid (L=%d), H=%d, d_k=%d, d_v=%d, bf16 inputs; fwd + Swish*RMSNorm "
+                        "epilogue + bwd + SREM 3x3 dwconv (C=%d); scan mode cycles over the 4 DiG directions"
+                        % (w.name, w.B, w.grid_h, w.grid_w, w.L, w.H, w.dk, w.dv, w.conv_C),
+            "global_batch": w.B * world, "seq_len": w.L, "parallelism": "replicas x%d" % world,
+            "l2": "flushed (512 MiB write) before every step, outside the timed events"}
+
+
+def run_ours(args, rank, world, local_rank):
+    from gated_linear_attention_fwd_b200 import dig
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = inputs.WORKLOADS[WORKLOAD_INDEX]
+    x = inputs.make_inputs(w, seed=inputs.SEED_BASE + WORKLOAD_INDEX + rank)
+    bf = torch.bfloat16
+    t = lambda a, dt=bf: torch.from_numpy(a).to(dev).to(dt).contiguous()
+    B, L, H, dk, dv = w.B, w.L, w.H, w.dk, w.dv
+    q, k, v, r, dO, xc = t(x["q"]), t(x["k"]), t(x["v"]), t(x["r"]), t(x["dO"]), t(x["x_conv"])
+    z, wc = t(x["z"], torch.float32), t(x["w_conv"], torch.float32)
+    o = torch.empty(B, L, H, dv, device=dev, dtype=bf)
+    y = torch.empty_like(o)
+    dq, dk_, dv_ = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dla = torch.empty_like(z)
+    yc = torch.empty(B, L, w.conv_C, device=dev, dtype=bf)
+    ws_f = dig.new_workspace(B, H, L, dk, dv, device=dev)
+    ws_b = dig.new_workspace(B, H, L, dk, dv, backward=True, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i, ev=None):
+        mode = i % 4
+        if ev:
+            ev[0].record(stream)
+        dig.dig_gla_fwd(q, k, v, z, w.inv_tau, o, w.grid_h, w.grid_w, mode, ws_f, r=r, y=y)
+        if ev:
+            ev[1].record(stream)
+        dig.dig_gla_bwd(q, k, v, z, w.inv_tau, dO, dq, dk_, dv_, dla, w.grid_h, w.grid_w, mode, ws_b)
+        if ev:
+            ev[2].record(stream)
+        dig.dig_srem_reorient_dwconv(xc, wc, None, yc, mode)
+        if ev:
+            ev[3].record(stream)
+
+    for i in range(args.warmup):
+        flush.fill_(float(i))
+        step(i)
+    torch.cuda.synchronize()
+    for ws in (ws_f, ws_b):
+        st = dig.dig_read_status(ws)
+        if st != dig.DIG_OK:
+            raise RuntimeError("device status after warm-up: %s" % dig.lib.dig_status_string(st).decode())
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for i in range(args.steps):
+            flush.fill_(float(i))       # evict L2 (outside the events)
+            step(i, evs[i])
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(3)] for i in range(args.steps)])  # ms
+    step_ms = float(per.sum(axis=1).mean())
+    if world > 1:
+        tt = torch.tensor([step_ms], device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        step_ms = float(tt.item())
+    for ws in (ws_f, ws_b):
+        st = dig.dig_read_status(ws)
+        if st != dig.DIG_OK:
+            raise RuntimeError("device status after timing: %s" % dig.lib.dig_status_string(st).decode())
+
+    # end to end: the same step through the C ABI with pinned host buffers
+    host_in = {n: a.cpu().pin_memory() for n, a in (("q", q), ("k", k), ("v", v), ("z", z), ("r", r), ("dO", dO),
+                                                     ("x", xc), ("w", wc))}
+    outs = (o, y, dq, dk_, dv_, dla, yc)
+    host_out = [a.cpu().pin_memory() for a in outs]
+    dev_in = {"q": q, "k": k, "v": v, "z": z, "r": r, "dO": dO, "x": xc, "w": wc}
+    h2d = sum(a.numel() * a.element_size() for a in host_in.values())
+    d2h = sum(a.numel() * a.element_size() for a in outs)
+    e2e_steps = max(3, min(args.steps, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_ms = []
+    for i in range(e2e_steps + 1):
+        flush.fill_(float(i))
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for n_, hbuf in host_in.items():
+            dev_in[n_].copy_(hbuf, non_blocking=True)
+        step(i)
+        for hb, a in zip(host_out, outs):
+            hb.copy_(a, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        if i > 0:
+            e2e_ms.append(e0.elapsed_time(e1))
+    e2e_step_ms = float(np.mean(e2e_ms))
+    if world > 1:
+        tt = torch.tensor([e2e_step_ms], device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        e2e_step_ms = float(tt.item())
+
+    if rank != 0:
+        return None
+    hbm, tflops, peak_kind = _peaks()
+    algo = algorithmic_bytes(w)
+    t_f, t_b, t_c = [float(per[:, j].mean()) * 1e-3 for j in range(3)]
+    names = {"fwd": ("gla_fwd_kernel", ["gla_fwd.cu", "gla_common.cuh", "sm100.cuh", "dig_common.cuh"], t_f),
+             "bwd": ("gla_bwd_kernel", ["gla_bwd.cu", "gla_common.cuh", "sm100.cuh", "dig_common.cuh"], t_b),
+             "conv": ("srem_dwconv_kernel", ["srem.cu", "dig_common.cuh"], t_c)}
+    dom = max(names, key=lambda n: names[n][2])
+    kname, srcs, tdom = names[dom]
+    achieved = algo[dom] / tdom / 1e9
+    tokens = B * L * world
+    line = {
+        "metric": METRIC, "value": tokens / (step_ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": _config(w, world),
+        "roofline": {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": _traffic(kname, srcs, 1.0),
+                     "algorithmic_bytes": algo[dom], "peak_source": peak_kind,
+                     "step_frac": (sum(algo.values()) / hbm / 1e9) / (step_ms * 1e-3)},
+        "kernels_us": {"gla_fwd": t_f * 1e6, "gla_bwd": t_b * 1e6, "srem_dwconv": t_c * 1e6},
+        "e2e": {"value": tokens / (e2e_step_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        tps, dt, cores = cpu_sample(w, x, steps=1)
+        line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": "oracle (fp64 C) on batch element 0 of %s, all heads, one step "
+                                          "(fwd+epilogue+bwd+conv, %d tokens), %.1f s" % (w.name, w.L, dt)}
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        ap.error("--gpus %d but WORLD_SIZE=%d (launch N>1 with torchrun)" % (args.gpus, world))
+    if world > 1 and args.impl == "ours":
+        import datetime
+        torch.distributed.init_process_group(backend="nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, rank, world)
+        else:
+            line = run_ours(args, rank, world, local_rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1 and args.impl == "ours":
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,59 @@
+"""Run one DiG op a few times on a synthetic workload, for profilers (ncu).
+
+    python -m gated_linear_attention_fwd_b200.profile_driver --op bwd --workload 3 --iters 4
+
+Inputs are random tensors of the workload's shapes (values do not affect the
+timing of these kernels); the device status word is checked at the end.
+"""
+import argparse
+
+import torch
+
+from . import dig, inputs
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--op", choices=["fwd", "bwd", "conv"], default="fwd")
+    ap.add_argument("--workload", type=int, default=3)
+    ap.add_argument("--iters", type=int, default=4)
+    ap.add_argument("--mode", type=int, default=0)
+    ap.add_argument("--epilogue", action="store_true")
+    args = ap.parse_args()
+    w = inputs.WORKLOADS[args.workload]
+    B, L, H, dk, dv = w.B, w.L, w.H, w.dk, w.dv
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    g = torch.Generator(device="cuda").manual_seed(0)
+    rnd = lambda *s: torch.randn(*s, device="cuda", generator=g).to(dt)
+    if args.op == "conv":
+        C = w.conv_C or H * dv
+        x, wc = rnd(B, w.grid_h, w.grid_w, C), torch.randn(C, 3, 3, device="cuda", generator=g) * 0.1
+        y = torch.empty(B, L, C, device="cuda", dtype=dt)
+        for _ in range(args.iters):
+            dig.dig_srem_reorient_dwconv(x, wc, None, y, args.mode)
+        torch.cuda.synchronize()
+        print("ok")
+        return
+    q, k, v = rnd(B, L, H, dk), rnd(B, L, H, dk), rnd(B, L, H, dv)
+    z = 0.03 * torch.randn(B, L, 1, dk, device="cuda", generator=g)
+    if args.op == "fwd":
+        o = torch.empty(B, L, H, dv, device="cuda", dtype=dt)
+        r = rnd(B, L, H, dv) if args.epilogue else None
+        y = torch.empty_like(o) if args.epilogue else None
+        ws = dig.new_workspace(B, H, L, dk, dv)
+        for _ in range(args.iters):
+            dig.dig_gla_fwd(q, k, v, z, w.inv_tau, o, w.grid_h, w.grid_w, args.mode, ws, r=r, y=y)
+    else:
+        dO = rnd(B, L, H, dv)
+        dq, dkk, dvv, dla = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(z)
+        ws = dig.new_workspace(B, H, L, dk, dv, backward=True)
+        for _ in range(args.iters):
+            dig.dig_gla_bwd(q, k, v, z, w.inv_tau, dO, dq, dkk, dvv, dla, w.grid_h, w.grid_w, args.mode, ws)
+    st = dig.dig_read_status(ws)
+    if st != dig.DIG_OK:
+        raise SystemExit("device status %d" % st)
+    print("ok")
+
+
+if __name__ == "__main__":
+    main()
