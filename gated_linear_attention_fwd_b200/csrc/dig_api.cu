@@ -23,6 +23,9 @@ static dig_status fail(dig_status s, const char* fmt, ...) {
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Lets other entry points of the library report a message through dig_last_error.
+void set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+
 WsLayout ws_layout(int nseq, int nseg, int nchunks, int dk, int dv, bool backward) {
   const size_t dkp = (size_t)((dk + 15) / 16 * 16);
   const size_t nrec = (size_t)nseq * nseg;

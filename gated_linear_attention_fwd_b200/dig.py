@@ -49,6 +49,9 @@ lib.dig_gla_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
 lib.dig_gla_fwd.restype = _i
 lib.dig_gla_fwd.argtypes = [_vp, _vp, _vp, _vp, _i, _f, _vp, _vp, _vp, _f, _vp,
                             _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]
+lib.dig_gla_fwd_noalloc.restype = _i
+lib.dig_gla_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i, _f, _vp, _vp, _vp, _f, _vp,
+                                    _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp]
 lib.dig_gla_bwd.restype = _i
 lib.dig_gla_bwd.argtypes = [_vp, _vp, _vp, _vp, _i, _f, _vp, _vp, _vp, _vp, _vp,
                             _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]
@@ -124,6 +127,20 @@ def dig_gla_fwd(q, k, v, z, inv_tau, o, grid_h, grid_w, scan_mode, workspace,
                          B, H, L, dk, dv, grid_h, grid_w, scan_mode, _code(q.dtype), _code(o.dtype),
                          _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "dig_gla_fwd")
+
+
+def dig_gla_fwd_noalloc(q, k, v, z, inv_tau, o, grid_h, grid_w, scan_mode, r=None, gamma=None, eps=1e-5, y=None,
+                        device_status=None, stream=None):
+    """dig_gla_fwd on the library's built-in scratch (no workspace argument; for
+    callers that cannot allocate device memory).  device_status: optional int32
+    CUDA tensor receiving the call's device status word."""
+    B, L, H, dk = q.shape
+    dv = v.shape[3]
+    st = lib.dig_gla_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(z), z.shape[2], float(inv_tau), _ptr(o),
+                                 _ptr(r), _ptr(gamma), float(eps), _ptr(y),
+                                 B, H, L, dk, dv, grid_h, grid_w, scan_mode, _code(q.dtype), _code(o.dtype),
+                                 _ptr(device_status), _stream(stream))
+    _check(st, "dig_gla_fwd_noalloc")
 
 
 def dig_gla_bwd(q, k, v, z, inv_tau, dO, dq, dk, dv, dlog_alpha, grid_h, grid_w, scan_mode, workspace,

@@ -28,8 +28,9 @@
  *   - Element types: `dtype` is the storage type of q, k, v, dO, r and of the
  *     conv input x (DIG_F32 or DIG_BF16); `out_dtype` is the storage type of o,
  *     y, dq, dk, dv and the conv output.  z, dlog_alpha, gamma, the conv weights
- *     and bias are always fp32.  Arithmetic is fp32 (tensor-core products in tf32
- *     with fp32 accumulation; three-term split tf32 when dtype == DIG_F32).
+ *     and bias are always fp32.  Arithmetic is fp32: tensor-core products take
+ *     each operand as a sum of bf16 terms (two for bf16 inputs, three for fp32
+ *     inputs) and accumulate in fp32.
  *   - Errors in the arguments are reported synchronously and nothing is
  *     launched.  A failed launch returns DIG_ERR_CUDA.  Conditions found on the
  *     device (a bounded wait that ran out, a gate outside the supported range)
@@ -99,6 +100,30 @@ dig_status dig_gla_fwd(const void *q, const void *k, const void *v, const float 
                        int B, int H, int L, int d_k, int d_v, int grid_h, int grid_w,
                        int scan_mode, int dtype, int out_dtype,
                        void *workspace, size_t workspace_bytes, void *stream);
+
+/* Forward without a caller-allocated workspace, for callers that cannot call
+ * cudaMalloc (plug-ins hosted by a runtime that owns all device memory and
+ * forbids its extensions to allocate; host programs that link only this library
+ * and have no device allocator).  The paper has no counterpart: this is an
+ * interface convenience.  Same arguments and results as dig_gla_fwd, but the
+ * workspace is a 4 MiB scratch array built into the library (one per GPU that
+ * loads it, held until the process exits); nothing is allocated or freed.
+ *   - Shapes whose dig_gla_workspace_bytes(B, H, L, d_k, d_v, 0) exceeds 4 MiB
+ *     are rejected with DIG_ERR_WORKSPACE_TOO_SMALL (see dig_last_error).
+ *   - The first call on a device looks up the scratch array's device address
+ *     (with that device current); make that first call before any stream capture.
+ *   - Every call clears the scratch's status word and flags (a small memset on
+ *     `stream`) and shares the one array: calls that overlap on the GPU (other
+ *     streams, other threads) race on it and must not be issued.
+ *   - device_status (optional, device pointer): receives the call's device
+ *     status word (DIG_OK, DIG_ERR_DEVICE_TIMEOUT, DIG_ERR_GATE_RANGE) in
+ *     stream order. */
+dig_status dig_gla_fwd_noalloc(const void *q, const void *k, const void *v, const float *z,
+                               int gate_heads, float inv_tau, void *o,
+                               const void *r, const float *gamma, float eps, void *y,
+                               int B, int H, int L, int d_k, int d_v, int grid_h, int grid_w,
+                               int scan_mode, int dtype, int out_dtype,
+                               unsigned int *device_status, void *stream);
 
 /* GLA backward: gradients of sum(o * dO) for the forward above.
  *   dO          [B, L, H, d_v]  dtype
