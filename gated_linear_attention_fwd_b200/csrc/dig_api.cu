@@ -26,9 +26,11 @@ static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Lets other entry points of the library report a message through dig_last_error.
 void set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
 
-WsLayout ws_layout(int nseq, int nseg, int nchunks, int dk, int dv, bool backward) {
+WsLayout ws_layout(int B, int H, int gate_heads, int L, int nseg, int nchunks, int dk, int dv, bool backward) {
   const size_t dkp = (size_t)((dk + 15) / 16 * 16);
-  const size_t nrec = (size_t)nseq * nseg;
+  const size_t nseq = (size_t)B * H;
+  const size_t nrec = nseq * nseg;
+  const size_t nbz = (size_t)B * gate_heads;
   WsLayout w{};
   size_t off = sizeof(WsHeader);
   w.flags = off;
@@ -42,9 +44,13 @@ WsLayout ws_layout(int nseq, int nseg, int nchunks, int dk, int dv, bool backwar
   w.seg_H = off;
   off = align_up(off + (backward ? nrec * (size_t)dk * dv * 4 : 0), 256);
   w.chunk_S = off;
-  off = align_up(off + (backward ? (size_t)nseq * nchunks * dk * dv * 4 : 0), 256);
+  off = align_up(off + (backward ? nseq * nchunks * dk * dv * 4 : 0), 256);
   w.chunk_B = off;
-  off = align_up(off + (backward ? (size_t)nseq * nchunks * dkp * 4 : 0), 256);
+  off = align_up(off + (backward ? nseq * nchunks * dkp * 4 : 0), 256);
+  w.gEQ = off;
+  off = align_up(off + nbz * (size_t)L * dk * 4, 256);
+  w.gCH = off;
+  off = align_up(off + nbz * (size_t)nchunks * 4 * dk * 4, 256);
   w.total = off;
   return w;
 }
@@ -109,13 +115,14 @@ extern "C" {
 
 int dig_gla_supported(int d_k, int d_v) { return gla_variant_built(d_k, d_v) ? 1 : 0; }
 
-size_t dig_gla_workspace_bytes(int B, int H, int L, int d_k, int d_v, int pass) {
+size_t dig_gla_workspace_bytes(int B, int H, int gate_heads, int L, int d_k, int d_v, int pass) {
   if (B < 0 || H <= 0 || L < 0 || d_k <= 0 || d_v <= 0 || (pass != 0 && pass != 1)) return 0;
+  if (gate_heads != 1 && gate_heads != H) return 0;
   const int nseq = B * H;
   // sized for the largest chunk count (fp32 inputs use shorter chunks)
   const int nchunks = pass == 1 ? (L + 31) / 32 : (L + 63) / 64;
   const int nseg = choose_nseg(nseq > 0 ? nseq : 1, nchunks);
-  return ws_layout(nseq > 0 ? nseq : 1, nseg, nchunks, d_k, d_v, pass == 1).total;
+  return ws_layout(B > 0 ? B : 1, H, gate_heads, L, nseg, nchunks, d_k, d_v, pass == 1).total;
 }
 
 dig_status dig_gla_fwd(const void* q, const void* k, const void* v, const float* z, int gate_heads, float inv_tau,
@@ -135,7 +142,7 @@ dig_status dig_gla_fwd(const void* q, const void* k, const void* v, const float*
   const int nseq = B * H;
   const int nchunks = (L + C - 1) / C;
   const int nseg = choose_nseg(nseq, nchunks);
-  const WsLayout lay = ws_layout(nseq, nseg, nchunks, d_k, d_v, false);
+  const WsLayout lay = ws_layout(B, H, gate_heads, L, nseg, nchunks, d_k, d_v, false);
   if (workspace_bytes < lay.total)
     return fail(DIG_ERR_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, needs %zu", workspace_bytes, lay.total);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -149,8 +156,13 @@ dig_status dig_gla_fwd(const void* q, const void* k, const void* v, const float*
   a.flags = reinterpret_cast<uint32_t*>(ws + lay.flags);
   a.seg_gam = reinterpret_cast<float*>(ws + lay.seg_gam);
   a.seg_S = reinterpret_cast<float*>(ws + lay.seg_S);
+  a.gEQ = reinterpret_cast<float*>(ws + lay.gEQ);
+  a.gCH = reinterpret_cast<float*>(ws + lay.gCH);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_gla_gate(a, C, d_k, nchunks, a.gEQ, a.gCH, s);
+  if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "gla_gate launch: %s", cudaGetErrorString(e));
   GlaVariant var{C, dtype == DIG_BF16 ? 1 : 2, d_k, d_v, dtype, out_dtype};
-  const cudaError_t e = launch_gla_fwd(var, a, nseq * nseg, nseg > 1, static_cast<cudaStream_t>(stream));
+  e = launch_gla_fwd(var, a, nseq * nseg, nseg > 1, s);
   if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "gla_fwd launch: %s", cudaGetErrorString(e));
   return DIG_OK;
 }
@@ -173,7 +185,7 @@ dig_status dig_gla_bwd(const void* q, const void* k, const void* v, const float*
   const int nseq = B * H;
   const int nchunks = (L + C - 1) / C;
   const int nseg = choose_nseg(nseq, nchunks);
-  const WsLayout lay = ws_layout(nseq, nseg, nchunks, d_k, d_v, true);
+  const WsLayout lay = ws_layout(B, H, gate_heads, L, nseg, nchunks, d_k, d_v, true);
   if (workspace_bytes < lay.total)
     return fail(DIG_ERR_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, needs %zu", workspace_bytes, lay.total);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -197,8 +209,12 @@ dig_status dig_gla_bwd(const void* q, const void* k, const void* v, const float*
   a.seg_H = reinterpret_cast<float*>(ws + lay.seg_H);
   a.chunk_S = reinterpret_cast<float*>(ws + lay.chunk_S);
   a.chunk_B = reinterpret_cast<float*>(ws + lay.chunk_B);
+  a.gEQ = reinterpret_cast<float*>(ws + lay.gEQ);
+  a.gCH = reinterpret_cast<float*>(ws + lay.gCH);
+  cudaError_t e = launch_gla_gate(a, C, d_k, nchunks, a.gEQ, a.gCH, s);
+  if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "gla_gate launch: %s", cudaGetErrorString(e));
   GlaVariant var{C, dtype == DIG_BF16 ? 1 : 2, d_k, d_v, dtype, out_dtype};
-  const cudaError_t e = launch_gla_bwd(var, a, nseq * nseg, nseg > 1, s);
+  e = launch_gla_bwd(var, a, nseq * nseg, nseg > 1, s);
   if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "gla_bwd launch: %s", cudaGetErrorString(e));
   return DIG_OK;
 }

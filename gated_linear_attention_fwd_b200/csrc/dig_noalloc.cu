@@ -14,7 +14,7 @@
 
 namespace {
 
-constexpr size_t kScratchBytes = 4u << 20;  // 4 MiB per device
+constexpr size_t kScratchBytes = 16u << 20;  // 16 MiB per device
 constexpr size_t kClearBytes = 256 + 16384;  // header + the flag words of up to 4096 segments
 constexpr int kMaxDevices = 64;
 
@@ -49,7 +49,7 @@ extern "C" dig_status dig_gla_fwd_noalloc(const void* q, const void* k, const vo
     }
     scratch = g_scratch_ptr[dev];
   }
-  const size_t need = dig_gla_workspace_bytes(B, H, L, d_k, d_v, 0);
+  const size_t need = dig_gla_workspace_bytes(B, H, gate_heads, L, d_k, d_v, 0);
   if (need > kScratchBytes) {
     char msg[200];
     snprintf(msg, sizeof(msg),

@@ -40,6 +40,9 @@ struct GlaArgs {
   float* seg_H;      // [nseq * nseg][DV][DK] segment state gradient (backward scan record)
   float* chunk_S;    // [nseq * nchunks][DV][DK] in-segment state entering each chunk (backward)
   float* chunk_B;    // [nseq * nchunks][DKP] in-segment log decay before each chunk (backward)
+  // gate factors shared by the heads (written by the gate kernel)
+  float* gEQ;        // [B * gate_heads][L (scan order)][DK]   2^(b - r)
+  float* gCH;        // [B * gate_heads][nchunks][4][DK]       2^r, 2^(Gamma-r), 2^Gamma, Gamma
 };
 
 // Kernel-variant selection: chunk length, split count, head dims, types.
@@ -52,9 +55,13 @@ struct GlaVariant {
 
 // Workspace layout for a given decomposition (bytes from the workspace start).
 struct WsLayout {
-  size_t flags, flags2, seg_gam, seg_S, seg_H, chunk_S, chunk_B, total;
+  size_t flags, flags2, seg_gam, seg_S, seg_H, chunk_S, chunk_B, gEQ, gCH, total;
 };
-WsLayout ws_layout(int nseq, int nseg, int nchunks, int dk, int dv, bool backward);
+WsLayout ws_layout(int B, int H, int gate_heads, int L, int nseg, int nchunks, int dk, int dv, bool backward);
+
+// Gate factors of every chunk (see gla_gate.cu); launched before the GLA kernels.
+cudaError_t launch_gla_gate(const GlaArgs& a, int chunk, int dk, int nchunks, float* EQ, float* CH,
+                            cudaStream_t s);
 
 // Launch helpers; return cudaSuccess or the launch error.  `coop` requests a
 // cooperative launch (all CTAs co-resident; needed when nseg > 1).

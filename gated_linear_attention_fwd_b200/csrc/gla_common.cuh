@@ -47,6 +47,68 @@ __device__ __forceinline__ void st_op4(uint8_t* base, int copy_bytes, uint32_t o
   }
 }
 
+// Shared-space stores of split bf16 terms: `saddr` is a shared-memory address
+// (cvta), term i goes to saddr + i * copy_bytes.
+template <int NT>
+__device__ __forceinline__ void sts_op4(uint32_t saddr, uint32_t copy_bytes, const float* x) {
+  float r[4] = {x[0], x[1], x[2], x[3]};
+#pragma unroll
+  for (int i = 0; i < NT; ++i) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(r[0], r[1]);
+    const __nv_bfloat162 b = __floats2bfloat162_rn(r[2], r[3]);
+    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(saddr + i * copy_bytes),
+                 "r"(*reinterpret_cast<const uint32_t*>(&a)), "r"(*reinterpret_cast<const uint32_t*>(&b))
+                 : "memory");
+    r[0] -= __low2float(a);
+    r[1] -= __high2float(a);
+    r[2] -= __low2float(b);
+    r[3] -= __high2float(b);
+  }
+}
+template <int NT>
+__device__ __forceinline__ void sts_op8(uint32_t saddr, uint32_t copy_bytes, const float* x) {
+  float r[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) r[j] = x[j];
+#pragma unroll
+  for (int i = 0; i < NT; ++i) {
+    __nv_bfloat162 h[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) h[j] = __floats2bfloat162_rn(r[2 * j], r[2 * j + 1]);
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(saddr + i * copy_bytes),
+                 "r"(*reinterpret_cast<const uint32_t*>(&h[0])), "r"(*reinterpret_cast<const uint32_t*>(&h[1])),
+                 "r"(*reinterpret_cast<const uint32_t*>(&h[2])), "r"(*reinterpret_cast<const uint32_t*>(&h[3]))
+                 : "memory");
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      r[2 * j] -= __low2float(h[j]);
+      r[2 * j + 1] -= __high2float(h[j]);
+    }
+  }
+}
+// Writes channels C0 .. C0+N-1 (C0, N multiples of 4) of one operand row in the
+// K-major layout: 16-byte stores where a core-matrix row (8 channels) is
+// covered, 8-byte stores for half rows.  `row` is the shared address of
+// channel 0 of the row.
+template <int NT, int C0, int N>
+struct RowWriter {
+  __device__ __forceinline__ static void run(uint32_t row, uint32_t copy_bytes, const float* x) {
+    if constexpr (N <= 0) {
+      return;
+    } else if constexpr (C0 % 8 == 0 && N >= 8) {
+      sts_op8<NT>(row + (C0 / 8) * 128, copy_bytes, x);
+      RowWriter<NT, C0 + 8, N - 8>::run(row, copy_bytes, x + 8);
+    } else {
+      sts_op4<NT>(row + (C0 / 8) * 128 + (C0 % 8) * 2, copy_bytes, x);
+      RowWriter<NT, C0 + 4, N - 4>::run(row, copy_bytes, x + 4);
+    }
+  }
+};
+// Shared address of row t's channel 0 in a K-major buffer with row stride sbo.
+__device__ __forceinline__ uint32_t row_addr(uint32_t buf, int t, int sbo) {
+  return buf + (uint32_t)(t >> 3) * sbo + (uint32_t)(t & 7) * 16u;
+}
+
 // Raw 4-element vectors as fetched from global memory (prefetched in registers).
 template <typename T>
 struct Raw4;

@@ -45,7 +45,7 @@ _sz = ctypes.c_size_t
 lib.dig_gla_supported.restype = _i
 lib.dig_gla_supported.argtypes = [_i, _i]
 lib.dig_gla_workspace_bytes.restype = _sz
-lib.dig_gla_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
+lib.dig_gla_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i]
 lib.dig_gla_fwd.restype = _i
 lib.dig_gla_fwd.argtypes = [_vp, _vp, _vp, _vp, _i, _f, _vp, _vp, _vp, _f, _vp,
                             _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]
@@ -107,13 +107,13 @@ def _check(st, where):
         raise DigError(st, where)
 
 
-def gla_workspace_bytes(B, H, L, d_k, d_v, backward=False) -> int:
-    return int(lib.dig_gla_workspace_bytes(B, H, L, d_k, d_v, 1 if backward else 0))
+def gla_workspace_bytes(B, H, L, d_k, d_v, backward=False, gate_heads=1) -> int:
+    return int(lib.dig_gla_workspace_bytes(B, H, gate_heads, L, d_k, d_v, 1 if backward else 0))
 
 
-def new_workspace(B, H, L, d_k, d_v, backward=False, device="cuda") -> torch.Tensor:
+def new_workspace(B, H, L, d_k, d_v, backward=False, device="cuda", gate_heads=1) -> torch.Tensor:
     """A zero-filled workspace (uint8) sized for dig_gla_fwd / dig_gla_bwd."""
-    n = gla_workspace_bytes(B, H, L, d_k, d_v, backward)
+    n = gla_workspace_bytes(B, H, L, d_k, d_v, backward, gate_heads)
     return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
 
 

@@ -74,12 +74,13 @@ enum { DIG_F32 = 0, DIG_BF16 = 1 };
 int dig_gla_supported(int d_k, int d_v);
 
 /* Bytes of device workspace dig_gla_fwd (pass = 0) or dig_gla_bwd (pass = 1)
- * needs for this shape on the current device.  The workspace must be
+ * needs for this shape (gate_heads: 1 or H, as passed to those calls) on the
+ * current device.  The workspace must be
  * zero-filled before its first use; every call that ends with status DIG_OK
  * leaves it ready for the next call (no re-zeroing needed).  After a device
  * status other than DIG_OK, zero it again.  Calls that may run concurrently
  * need separate workspaces.  Returns 0 for invalid shapes. */
-size_t dig_gla_workspace_bytes(int B, int H, int L, int d_k, int d_v, int pass);
+size_t dig_gla_workspace_bytes(int B, int H, int gate_heads, int L, int d_k, int d_v, int pass);
 
 /* GLA forward (slide eq. (5)-(8), chunkwise).
  *   q, k   [B, L, H, d_k]   dtype        queries / keys (no extra 1/sqrt(d) scale)
@@ -106,9 +107,10 @@ dig_status dig_gla_fwd(const void *q, const void *k, const void *v, const float 
  * forbids its extensions to allocate; host programs that link only this library
  * and have no device allocator).  The paper has no counterpart: this is an
  * interface convenience.  Same arguments and results as dig_gla_fwd, but the
- * workspace is a 4 MiB scratch array built into the library (one per GPU that
+ * workspace is a 16 MiB scratch array built into the library (one per GPU that
  * loads it, held until the process exits); nothing is allocated or freed.
- *   - Shapes whose dig_gla_workspace_bytes(B, H, L, d_k, d_v, 0) exceeds 4 MiB
+ *   - Shapes whose dig_gla_workspace_bytes(B, H, gate_heads, L, d_k, d_v, 0)
+ *     exceeds 16 MiB
  *     are rejected with DIG_ERR_WORKSPACE_TOO_SMALL (see dig_last_error).
  *   - The first call on a device looks up the scratch array's device address
  *     (with that device current); make that first call before any stream capture.

@@ -85,8 +85,10 @@ def test_bwd_and_conv_reject_bad_arguments_on_host():
 def test_workspace_bytes():
     assert dig.gla_workspace_bytes(4, 6, 4096, 32, 64) > 256
     assert dig.gla_workspace_bytes(4, 6, 4096, 32, 64, backward=True) > dig.gla_workspace_bytes(4, 6, 4096, 32, 64)
-    assert dig.lib.dig_gla_workspace_bytes(1, 0, 16, 32, 64, 0) == 0
-    assert dig.lib.dig_gla_workspace_bytes(1, 1, 16, 32, 64, 2) == 0
+    assert dig.lib.dig_gla_workspace_bytes(1, 0, 1, 16, 32, 64, 0) == 0
+    assert dig.lib.dig_gla_workspace_bytes(1, 1, 1, 16, 32, 64, 2) == 0
+    assert dig.lib.dig_gla_workspace_bytes(1, 4, 3, 16, 32, 64, 0) == 0      # gate_heads neither 1 nor H
+    assert dig.gla_workspace_bytes(2, 4, 256, 32, 64, gate_heads=4) > dig.gla_workspace_bytes(2, 4, 256, 32, 64)
 
 
 def test_status_strings():

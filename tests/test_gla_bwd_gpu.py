@@ -32,7 +32,7 @@ def run_bwd(w, x, mode, out_dtype="f32", gate=None, ws=None):
     dvv = torch.full((B, L, H, dv), float("nan"), dtype=odt, device="cuda")
     dla = torch.full(tuple(z.shape), float("nan"), dtype=torch.float32, device="cuda")
     if ws is None:
-        ws = dig.new_workspace(B, H, L, dk, dv, backward=True)
+        ws = dig.new_workspace(B, H, L, dk, dv, backward=True, gate_heads=z.shape[2])
     dig.dig_gla_bwd(q, k, v, z, w.inv_tau, dO, dq, dkk, dvv, dla, w.grid_h, w.grid_w, mode, ws)
     st = dig.dig_read_status(ws)
     return (dq, dkk, dvv, dla), st

@@ -34,7 +34,7 @@ def run_fwd(w, x, mode, out_dtype="f32", epilogue=False, gamma=None, ws=None, ga
         if gamma is not None:
             g = dev(gamma)
     if ws is None:
-        ws = dig.new_workspace(B, H, L, dk, dv)
+        ws = dig.new_workspace(B, H, L, dk, dv, gate_heads=z.shape[2])
     dig.dig_gla_fwd(q, k, v, z, w.inv_tau, o, w.grid_h, w.grid_w, mode, ws, r=r, gamma=g, eps=1e-5, y=y)
     st = dig.dig_read_status(ws)
     return o, y, st

@@ -47,8 +47,8 @@ def test_noalloc_forward_matches_the_workspace_forward_on_two_calls_in_a_row():
 
 def test_noalloc_rejects_a_shape_beyond_the_scratch():
     from gated_linear_attention_fwd_b200 import dig
-    B, H, Hg, Wg, dk, dv = 64, 64, 64, 64, 64, 64      # 4096 sequences: far more records than 4 MiB holds
-    assert dig.gla_workspace_bytes(B, H, Hg * Wg, dk, dv) > (4 << 20)
+    B, H, Hg, Wg, dk, dv = 64, 64, 64, 64, 64, 64      # 4096 sequences: far more than the 16 MiB scratch holds
+    assert dig.gla_workspace_bytes(B, H, Hg * Wg, dk, dv) > (16 << 20)
     buf = torch.zeros(64, dtype=torch.float32, device="cuda")   # never touched: rejected before any launch
     p = ctypes.c_void_p(buf.data_ptr())
     st = dig.lib.dig_gla_fwd_noalloc(p, p, p, p, 1, 0.0625, p, None, None, 1e-5, None, B, H, Hg * Wg, dk, dv, Hg, Wg,
