@@ -33,24 +33,24 @@ WsLayout ws_layout(int B, int H, int gate_heads, int L, int nseg, int nchunks, i
   const size_t nbz = (size_t)B * gate_heads;
   WsLayout w{};
   size_t off = sizeof(WsHeader);
-  w.flags = off;
-  off = align_up(off + nrec * 4, 256);
-  w.flags2 = off;
-  off = align_up(off + (backward ? nrec * 4 : 0), 256);
-  w.seg_gam = off;
-  off = align_up(off + nrec * dkp * 4, 256);
-  w.seg_S = off;
-  off = align_up(off + nrec * (size_t)dk * dv * 4, 256);
-  w.seg_H = off;
-  off = align_up(off + (backward ? nrec * (size_t)dk * dv * 4 : 0), 256);
-  w.chunk_S = off;
-  off = align_up(off + (backward ? nseq * nchunks * dk * dv * 4 : 0), 256);
-  w.chunk_B = off;
-  off = align_up(off + (backward ? nseq * nchunks * dkp * 4 : 0), 256);
-  w.gEQ = off;
-  off = align_up(off + nbz * (size_t)L * dk * 4, 256);
-  w.gCH = off;
-  off = align_up(off + nbz * (size_t)nchunks * 4 * dk * 4, 256);
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, 256);
+    return at;
+  };
+  if (!backward) {
+    w.gEQ = take(nbz * (size_t)L * dk * 4);
+    w.gCH = take(nbz * (size_t)nchunks * 4 * dk * 4);
+    w.dsn = take(nseq * (size_t)nchunks * dk * dv * 4);
+  } else {
+    w.flags = take(nrec * 4);
+    w.flags2 = take(nrec * 4);
+    w.seg_gam = take(nrec * dkp * 4);
+    w.seg_S = take(nrec * (size_t)dk * dv * 4);
+    w.seg_H = take(nrec * (size_t)dk * dv * 4);
+    w.chunk_S = take(nseq * nchunks * (size_t)dk * dv * 4);
+    w.chunk_B = take(nseq * nchunks * dkp * 4);
+  }
   w.total = off;
   return w;
 }
@@ -74,8 +74,8 @@ int device_sms() {
 // Tokens per chunk: forward 128 (bf16 inputs) / 64 (fp32); backward 64 / 32.
 int chunk_len(int dtype, bool backward) { return (dtype == DIG_BF16 ? 128 : 64) >> (backward ? 1 : 0); }
 
-// Segments per sequence: enough CTAs to cover the SMs once (one resident CTA
-// per SM), never more than the sequence has chunks.
+// Backward segments per sequence: enough CTAs to cover the SMs once (one
+// resident CTA per SM), never more than the sequence has chunks.
 int choose_nseg(int nseq, int nchunks) {
   const int slots = device_sms();  // kernels run one CTA per SM
   if (nseq >= slots || nchunks <= 1) return 1;
@@ -121,7 +121,7 @@ size_t dig_gla_workspace_bytes(int B, int H, int gate_heads, int L, int d_k, int
   const int nseq = B * H;
   // sized for the largest chunk count (fp32 inputs use shorter chunks)
   const int nchunks = pass == 1 ? (L + 31) / 32 : (L + 63) / 64;
-  const int nseg = choose_nseg(nseq > 0 ? nseq : 1, nchunks);
+  const int nseg = pass == 1 ? choose_nseg(nseq > 0 ? nseq : 1, nchunks) : 1;
   return ws_layout(B > 0 ? B : 1, H, gate_heads, L, nseg, nchunks, d_k, d_v, pass == 1).total;
 }
 
@@ -139,10 +139,8 @@ dig_status dig_gla_fwd(const void* q, const void* k, const void* v, const float*
       !aligned16(gamma) || !aligned16(y))
     return fail(DIG_ERR_MISALIGNED, "a tensor pointer is not 16-byte aligned");
   const int C = chunk_len(dtype, false);
-  const int nseq = B * H;
   const int nchunks = (L + C - 1) / C;
-  const int nseg = choose_nseg(nseq, nchunks);
-  const WsLayout lay = ws_layout(B, H, gate_heads, L, nseg, nchunks, d_k, d_v, false);
+  const WsLayout lay = ws_layout(B, H, gate_heads, L, 1, nchunks, d_k, d_v, false);
   if (workspace_bytes < lay.total)
     return fail(DIG_ERR_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, needs %zu", workspace_bytes, lay.total);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -150,19 +148,15 @@ dig_status dig_gla_fwd(const void* q, const void* k, const void* v, const float*
   a.q = q; a.k = k; a.v = v; a.z = z; a.r = r; a.gamma = gamma; a.o = o; a.y = y;
   a.B = B; a.H = H; a.L = L; a.Hg = grid_h; a.Wg = grid_w; a.mode = scan_mode; a.gate_heads = gate_heads;
   a.inv_tau = inv_tau; a.eps = eps;
-  a.nchunks = nchunks; a.nseg = nseg;
+  a.nchunks = nchunks; a.nseg = 1;
   a.status = reinterpret_cast<uint32_t*>(ws);
   a.done = reinterpret_cast<uint32_t*>(ws) + 1;
-  a.flags = reinterpret_cast<uint32_t*>(ws + lay.flags);
-  a.seg_gam = reinterpret_cast<float*>(ws + lay.seg_gam);
-  a.seg_S = reinterpret_cast<float*>(ws + lay.seg_S);
   a.gEQ = reinterpret_cast<float*>(ws + lay.gEQ);
   a.gCH = reinterpret_cast<float*>(ws + lay.gCH);
+  a.dsn = reinterpret_cast<float*>(ws + lay.dsn);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_gla_gate(a, C, d_k, nchunks, a.gEQ, a.gCH, s);
-  if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "gla_gate launch: %s", cudaGetErrorString(e));
   GlaVariant var{C, dtype == DIG_BF16 ? 1 : 2, d_k, d_v, dtype, out_dtype};
-  e = launch_gla_fwd(var, a, nseq * nseg, nseg > 1, s);
+  const cudaError_t e = launch_gla_fwd(var, a, s);
   if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "gla_fwd launch: %s", cudaGetErrorString(e));
   return DIG_OK;
 }
@@ -209,12 +203,8 @@ dig_status dig_gla_bwd(const void* q, const void* k, const void* v, const float*
   a.seg_H = reinterpret_cast<float*>(ws + lay.seg_H);
   a.chunk_S = reinterpret_cast<float*>(ws + lay.chunk_S);
   a.chunk_B = reinterpret_cast<float*>(ws + lay.chunk_B);
-  a.gEQ = reinterpret_cast<float*>(ws + lay.gEQ);
-  a.gCH = reinterpret_cast<float*>(ws + lay.gCH);
-  cudaError_t e = launch_gla_gate(a, C, d_k, nchunks, a.gEQ, a.gCH, s);
-  if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "gla_gate launch: %s", cudaGetErrorString(e));
   GlaVariant var{C, dtype == DIG_BF16 ? 1 : 2, d_k, d_v, dtype, out_dtype};
-  e = launch_gla_bwd(var, a, nseq * nseg, nseg > 1, s);
+  const cudaError_t e = launch_gla_bwd(var, a, nseq * nseg, nseg > 1, s);
   if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "gla_bwd launch: %s", cudaGetErrorString(e));
   return DIG_OK;
 }

@@ -15,7 +15,7 @@
 namespace {
 
 constexpr size_t kScratchBytes = 16u << 20;  // 16 MiB per device
-constexpr size_t kClearBytes = 256 + 16384;  // header + the flag words of up to 4096 segments
+constexpr size_t kClearBytes = 256;  // the header (status word)
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
@@ -60,7 +60,7 @@ extern "C" dig_status dig_gla_fwd_noalloc(const void* q, const void* k, const vo
     return DIG_ERR_WORKSPACE_TOO_SMALL;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the status word and the inter-CTA flags must start at zero on every call
+  // the status word must start at zero on every call
   if (cudaMemsetAsync(scratch, 0, kClearBytes, s) != cudaSuccess) return DIG_ERR_CUDA;
   const dig_status st = dig_gla_fwd(q, k, v, z, gate_heads, inv_tau, o, r, gamma, eps, y, B, H, L, d_k, d_v, grid_h,
                                     grid_w, scan_mode, dtype, out_dtype, scratch, kScratchBytes, stream);

@@ -40,9 +40,10 @@ struct GlaArgs {
   float* seg_H;      // [nseq * nseg][DV][DK] segment state gradient (backward scan record)
   float* chunk_S;    // [nseq * nchunks][DV][DK] in-segment state entering each chunk (backward)
   float* chunk_B;    // [nseq * nchunks][DKP] in-segment log decay before each chunk (backward)
-  // gate factors shared by the heads (written by the gate kernel)
+  // forward: gate factors shared by the heads, and the chunk states
   float* gEQ;        // [B * gate_heads][L (scan order)][DK]   2^(b - r)
   float* gCH;        // [B * gate_heads][nchunks][4][DK]       2^r, 2^(Gamma-r), 2^Gamma, Gamma
+  float* dsn;        // [nseq][nchunks][DV][DK]  chunk state contribution, then the state entering the chunk
 };
 
 // Kernel-variant selection: chunk length, split count, head dims, types.
@@ -55,20 +56,19 @@ struct GlaVariant {
 
 // Workspace layout for a given decomposition (bytes from the workspace start).
 struct WsLayout {
-  size_t flags, flags2, seg_gam, seg_S, seg_H, chunk_S, chunk_B, gEQ, gCH, total;
+  size_t flags, flags2, seg_gam, seg_S, seg_H, chunk_S, chunk_B, gEQ, gCH, dsn, total;
 };
+// Forward (backward = false): gate factors and chunk states.  Backward: the
+// segment records of its two sweeps.
 WsLayout ws_layout(int B, int H, int gate_heads, int L, int nseg, int nchunks, int dk, int dv, bool backward);
 
-// Gate factors of every chunk (see gla_gate.cu); launched before the GLA kernels.
-cudaError_t launch_gla_gate(const GlaArgs& a, int chunk, int dk, int nchunks, float* EQ, float* CH,
-                            cudaStream_t s);
-
-// Launch helpers; return cudaSuccess or the launch error.  `coop` requests a
-// cooperative launch (all CTAs co-resident; needed when nseg > 1).
-cudaError_t launch_gla_fwd(const GlaVariant& var, const GlaArgs& a, int grid, bool coop, cudaStream_t s);
+// Launch helpers; return cudaSuccess or the launch error.  The forward enqueues
+// its three kernels (chunk states, state scan, outputs).  For the backward,
+// `coop` requests a cooperative launch (all CTAs co-resident; needed when
+// nseg > 1).
+cudaError_t launch_gla_fwd(const GlaVariant& var, const GlaArgs& a, cudaStream_t s);
 cudaError_t launch_gla_bwd(const GlaVariant& var, const GlaArgs& a, int grid, bool coop, cudaStream_t s);
-// Resident CTAs per SM of the variant's kernel (0 if the variant is not built).
-int gla_fwd_blocks_per_sm(const GlaVariant& var);
+// Resident CTAs per SM of the backward kernel (0 if the variant is not built).
 int gla_bwd_blocks_per_sm(const GlaVariant& var);
 bool gla_variant_built(int dk, int dv);
 

@@ -109,6 +109,91 @@ __device__ __forceinline__ uint32_t row_addr(uint32_t buf, int t, int sbo) {
   return buf + (uint32_t)(t >> 3) * sbo + (uint32_t)(t & 7) * 16u;
 }
 
+__host__ __device__ constexpr int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// Coalesced work split of a [rows][NG] grid of row pieces over a CTA: piece i
+// is (row, group) with runs of 8 consecutive rows per group, so a warp touches
+// 8 rows x 4 groups (few cache lines per load) and every 8-lane phase of a
+// 16-byte shared-memory store covers 8 consecutive K-major rows (no bank
+// conflicts).
+template <int NG>
+__device__ __forceinline__ void piece_of(int i, int& row, int& g) {
+  const int rest = i >> 3;
+  g = rest % NG;
+  row = (rest / NG) * 8 + (i & 7);
+}
+
+// PS consecutive elements of one row as raw 32-bit words (vector loads).
+template <typename T, int PS>
+struct Piece {
+  static constexpr int NW = PS * (int)sizeof(T) / 4;
+  static_assert(NW == 2 || NW % 4 == 0, "8-byte or whole 16-byte pieces");
+  uint32_t w[NW];
+  __device__ __forceinline__ void load(const T* p, bool valid) {
+    if constexpr (NW == 2) {
+      const uint2 u = valid ? __ldg(reinterpret_cast<const uint2*>(p)) : make_uint2(0u, 0u);
+      w[0] = u.x;
+      w[1] = u.y;
+    } else {
+#pragma unroll
+      for (int i = 0; i < NW; i += 4) {
+        const uint4 u = valid ? __ldg(reinterpret_cast<const uint4*>(p) + i / 4) : make_uint4(0u, 0u, 0u, 0u);
+        w[i] = u.x;
+        w[i + 1] = u.y;
+        w[i + 2] = u.z;
+        w[i + 3] = u.w;
+      }
+    }
+  }
+  // L2-only load of data written earlier in the same stream by another kernel
+  __device__ __forceinline__ void load_cg(const T* p, bool valid) {
+#pragma unroll
+    for (int i = 0; i < NW; i += 4) {
+      const uint4 u = valid ? __ldcg(reinterpret_cast<const uint4*>(p) + i / 4) : make_uint4(0u, 0u, 0u, 0u);
+      w[i] = u.x;
+      w[i + 1] = u.y;
+      w[i + 2] = u.z;
+      w[i + 3] = u.w;
+    }
+  }
+  __device__ __forceinline__ void unpack(float* o) const {
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+      for (int i = 0; i < NW; ++i) {
+        o[2 * i] = __uint_as_float(w[i] << 16);
+        o[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < NW; ++i) o[i] = __uint_as_float(w[i]);
+    }
+  }
+};
+
+// Stores PS values (PS = 4 or 8) at channel c0 (c0 % PS == 0) of row `row` of a
+// K-major operand buffer, as NT bf16 terms.
+template <int NT, int PS>
+__device__ __forceinline__ void st_piece(uint32_t buf, int row, int sbo, int c0, uint32_t copy_bytes,
+                                         const float* x) {
+  const uint32_t a = row_addr(buf, row, sbo) + (uint32_t)(c0 >> 3) * 128u + (uint32_t)(c0 & 7) * 2u;
+  if constexpr (PS == 8) sts_op8<NT>(a, copy_bytes, x);
+  else sts_op4<NT>(a, copy_bytes, x);
+}
+
+// Stores 8 values to global memory as bf16 (one 16-byte store) or fp32 (two).
+__device__ __forceinline__ void st_global8(__nv_bfloat16* p, const float* v) {
+  uint4 u;
+  u.x = pack_bf16x2(v[0], v[1]);
+  u.y = pack_bf16x2(v[2], v[3]);
+  u.z = pack_bf16x2(v[4], v[5]);
+  u.w = pack_bf16x2(v[6], v[7]);
+  *reinterpret_cast<uint4*>(p) = u;
+}
+__device__ __forceinline__ void st_global8(float* p, const float* v) {
+  reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+  reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+
 // Raw 4-element vectors as fetched from global memory (prefetched in registers).
 template <typename T>
 struct Raw4;

@@ -114,8 +114,8 @@ dig_status dig_gla_fwd(const void *q, const void *k, const void *v, const float 
  *     are rejected with DIG_ERR_WORKSPACE_TOO_SMALL (see dig_last_error).
  *   - The first call on a device looks up the scratch array's device address
  *     (with that device current); make that first call before any stream capture.
- *   - Every call clears the scratch's status word and flags (a small memset on
- *     `stream`) and shares the one array: calls that overlap on the GPU (other
+ *   - Every call clears the scratch's status word (a small memset on `stream`)
+ *     and shares the one array: calls that overlap on the GPU (other
  *     streams, other threads) race on it and must not be issued.
  *   - device_status (optional, device pointer): receives the call's device
  *     status word (DIG_OK, DIG_ERR_DEVICE_TIMEOUT, DIG_ERR_GATE_RANGE) in

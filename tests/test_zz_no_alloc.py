@@ -21,8 +21,8 @@ pytestmark = pytest.mark.gpu
 
 def test_noalloc_forward_matches_the_workspace_forward_on_two_calls_in_a_row():
     from gated_linear_attention_fwd_b200 import dig
-    # 4 x 6 sequences split over several segments: the inter-CTA flags and segment
-    # records live in the built-in scratch
+    # 4 x 6 sequences of 32 chunks: the gate factors and the chunk states live in
+    # the built-in scratch
     w = inputs.WORKLOADS[2]
     x = inputs.make_inputs(w)
     q, k, v, z = dev(x["q"], w.dtype), dev(x["k"], w.dtype), dev(x["v"], w.dtype), dev(x["z"])
