@@ -26,10 +26,8 @@ static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Lets other entry points of the library report a message through dig_last_error.
 void set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
 
-WsLayout ws_layout(int B, int H, int gate_heads, int L, int nseg, int nchunks, int dk, int dv, bool backward) {
-  const size_t dkp = (size_t)((dk + 15) / 16 * 16);
+WsLayout ws_layout(int B, int H, int gate_heads, int L, int nchunks, int dk, int dv, bool backward) {
   const size_t nseq = (size_t)B * H;
-  const size_t nrec = nseq * nseg;
   const size_t nbz = (size_t)B * gate_heads;
   WsLayout w{};
   size_t off = sizeof(WsHeader);
@@ -38,50 +36,20 @@ WsLayout ws_layout(int B, int H, int gate_heads, int L, int nseg, int nchunks, i
     off = align_up(off + bytes, 256);
     return at;
   };
-  if (!backward) {
-    w.gEQ = take(nbz * (size_t)L * dk * 4);
-    w.gCH = take(nbz * (size_t)nchunks * 4 * dk * 4);
-    w.dsn = take(nseq * (size_t)nchunks * dk * dv * 4);
-  } else {
-    w.flags = take(nrec * 4);
-    w.flags2 = take(nrec * 4);
-    w.seg_gam = take(nrec * dkp * 4);
-    w.seg_S = take(nrec * (size_t)dk * dv * 4);
-    w.seg_H = take(nrec * (size_t)dk * dv * 4);
-    w.chunk_S = take(nseq * nchunks * (size_t)dk * dv * 4);
-    w.chunk_B = take(nseq * nchunks * dkp * 4);
-  }
+  w.gEQ = take(nbz * (size_t)L * dk * 4);
+  w.gCH = take(nbz * (size_t)nchunks * 4 * dk * 4);
+  w.dsn = take(nseq * (size_t)nchunks * dk * dv * 4);
+  w.dhn = take(backward ? nseq * (size_t)nchunks * dk * dv * 4 : 0);
   w.total = off;
   return w;
 }
 
 namespace {
 
-constexpr int kMaxDev = 64;
-int g_sms[kMaxDev];
-
-int device_sms() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return 148;
-  if (g_sms[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    g_sms[dev] = n;
-  }
-  return g_sms[dev];
-}
-
-// Tokens per chunk: forward 128 (bf16 inputs) / 64 (fp32); backward 64 / 32.
-int chunk_len(int dtype, bool backward) { return (dtype == DIG_BF16 ? 128 : 64) >> (backward ? 1 : 0); }
-
-// Backward segments per sequence: enough CTAs to cover the SMs once (one
-// resident CTA per SM), never more than the sequence has chunks.
-int choose_nseg(int nseq, int nchunks) {
-  const int slots = device_sms();  // kernels run one CTA per SM
-  if (nseq >= slots || nchunks <= 1) return 1;
-  int nseg = slots / nseq;
-  if (nseg > nchunks) nseg = nchunks;
-  return nseg < 1 ? 1 : nseg;
+// Tokens per chunk: forward 128 (bf16 inputs) / 64 (fp32); backward by head dims.
+int chunk_len(int dtype, bool backward, int dk, int dv) {
+  if (backward) return gla_bwd_chunk(dk, dv, dtype);
+  return dtype == DIG_BF16 ? 128 : 64;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -118,11 +86,11 @@ int dig_gla_supported(int d_k, int d_v) { return gla_variant_built(d_k, d_v) ? 1
 size_t dig_gla_workspace_bytes(int B, int H, int gate_heads, int L, int d_k, int d_v, int pass) {
   if (B < 0 || H <= 0 || L < 0 || d_k <= 0 || d_v <= 0 || (pass != 0 && pass != 1)) return 0;
   if (gate_heads != 1 && gate_heads != H) return 0;
-  const int nseq = B * H;
-  // sized for the largest chunk count (fp32 inputs use shorter chunks)
-  const int nchunks = pass == 1 ? (L + 31) / 32 : (L + 63) / 64;
-  const int nseg = pass == 1 ? choose_nseg(nseq > 0 ? nseq : 1, nchunks) : 1;
-  return ws_layout(B > 0 ? B : 1, H, gate_heads, L, nseg, nchunks, d_k, d_v, pass == 1).total;
+  if (!gla_variant_built(d_k, d_v)) return 0;
+  // sized for the largest chunk count of either input type
+  const int C = pass == 1 ? gla_bwd_chunk(d_k, d_v, DIG_F32) : 64;
+  const int nchunks = (L + C - 1) / C;
+  return ws_layout(B > 0 ? B : 1, H, gate_heads, L, nchunks, d_k, d_v, pass == 1).total;
 }
 
 dig_status dig_gla_fwd(const void* q, const void* k, const void* v, const float* z, int gate_heads, float inv_tau,
@@ -138,9 +106,9 @@ dig_status dig_gla_fwd(const void* q, const void* k, const void* v, const float*
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(z) || !aligned16(o) || !aligned16(r) ||
       !aligned16(gamma) || !aligned16(y))
     return fail(DIG_ERR_MISALIGNED, "a tensor pointer is not 16-byte aligned");
-  const int C = chunk_len(dtype, false);
+  const int C = chunk_len(dtype, false, d_k, d_v);
   const int nchunks = (L + C - 1) / C;
-  const WsLayout lay = ws_layout(B, H, gate_heads, L, 1, nchunks, d_k, d_v, false);
+  const WsLayout lay = ws_layout(B, H, gate_heads, L, nchunks, d_k, d_v, false);
   if (workspace_bytes < lay.total)
     return fail(DIG_ERR_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, needs %zu", workspace_bytes, lay.total);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -148,14 +116,13 @@ dig_status dig_gla_fwd(const void* q, const void* k, const void* v, const float*
   a.q = q; a.k = k; a.v = v; a.z = z; a.r = r; a.gamma = gamma; a.o = o; a.y = y;
   a.B = B; a.H = H; a.L = L; a.Hg = grid_h; a.Wg = grid_w; a.mode = scan_mode; a.gate_heads = gate_heads;
   a.inv_tau = inv_tau; a.eps = eps;
-  a.nchunks = nchunks; a.nseg = 1;
+  a.nchunks = nchunks;
   a.status = reinterpret_cast<uint32_t*>(ws);
-  a.done = reinterpret_cast<uint32_t*>(ws) + 1;
   a.gEQ = reinterpret_cast<float*>(ws + lay.gEQ);
   a.gCH = reinterpret_cast<float*>(ws + lay.gCH);
   a.dsn = reinterpret_cast<float*>(ws + lay.dsn);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  GlaVariant var{C, dtype == DIG_BF16 ? 1 : 2, d_k, d_v, dtype, out_dtype};
+  GlaVariant var{C, dtype == DIG_BF16 ? 2 : 3, d_k, d_v, dtype, out_dtype};
   const cudaError_t e = launch_gla_fwd(var, a, s);
   if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "gla_fwd launch: %s", cudaGetErrorString(e));
   return DIG_OK;
@@ -175,11 +142,9 @@ dig_status dig_gla_bwd(const void* q, const void* k, const void* v, const float*
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(z) || !aligned16(dO) || !aligned16(dq) ||
       !aligned16(dk) || !aligned16(dv) || !aligned16(dlog_alpha))
     return fail(DIG_ERR_MISALIGNED, "a tensor pointer is not 16-byte aligned");
-  const int C = chunk_len(dtype, true);
-  const int nseq = B * H;
+  const int C = chunk_len(dtype, true, d_k, d_v);
   const int nchunks = (L + C - 1) / C;
-  const int nseg = choose_nseg(nseq, nchunks);
-  const WsLayout lay = ws_layout(B, H, gate_heads, L, nseg, nchunks, d_k, d_v, true);
+  const WsLayout lay = ws_layout(B, H, gate_heads, L, nchunks, d_k, d_v, true);
   if (workspace_bytes < lay.total)
     return fail(DIG_ERR_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, needs %zu", workspace_bytes, lay.total);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -193,18 +158,14 @@ dig_status dig_gla_bwd(const void* q, const void* k, const void* v, const float*
   a.q = q; a.k = k; a.v = v; a.z = z; a.dO = dO; a.dq = dq; a.dk = dk; a.dv = dv; a.dla = dlog_alpha;
   a.B = B; a.H = H; a.L = L; a.Hg = grid_h; a.Wg = grid_w; a.mode = scan_mode; a.gate_heads = gate_heads;
   a.inv_tau = inv_tau;
-  a.nchunks = nchunks; a.nseg = nseg;
+  a.nchunks = nchunks;
   a.status = reinterpret_cast<uint32_t*>(ws);
-  a.done = reinterpret_cast<uint32_t*>(ws) + 1;
-  a.flags = reinterpret_cast<uint32_t*>(ws + lay.flags);
-  a.flags2 = reinterpret_cast<uint32_t*>(ws + lay.flags2);
-  a.seg_gam = reinterpret_cast<float*>(ws + lay.seg_gam);
-  a.seg_S = reinterpret_cast<float*>(ws + lay.seg_S);
-  a.seg_H = reinterpret_cast<float*>(ws + lay.seg_H);
-  a.chunk_S = reinterpret_cast<float*>(ws + lay.chunk_S);
-  a.chunk_B = reinterpret_cast<float*>(ws + lay.chunk_B);
-  GlaVariant var{C, dtype == DIG_BF16 ? 1 : 2, d_k, d_v, dtype, out_dtype};
-  const cudaError_t e = launch_gla_bwd(var, a, nseq * nseg, nseg > 1, s);
+  a.gEQ = reinterpret_cast<float*>(ws + lay.gEQ);
+  a.gCH = reinterpret_cast<float*>(ws + lay.gCH);
+  a.dsn = reinterpret_cast<float*>(ws + lay.dsn);
+  a.dhn = reinterpret_cast<float*>(ws + lay.dhn);
+  GlaVariant var{C, dtype == DIG_BF16 ? 2 : 3, d_k, d_v, dtype, out_dtype};
+  const cudaError_t e = launch_gla_bwd(var, a, s);
   if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "gla_bwd launch: %s", cudaGetErrorString(e));
   return DIG_OK;
 }

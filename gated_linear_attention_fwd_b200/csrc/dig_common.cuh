@@ -83,39 +83,17 @@ __device__ __forceinline__ void store_row(float* p, const float* v) {
 __device__ __forceinline__ float log_sigmoid(float x) { return fminf(x, 0.f) - log1pf(expf(-fabsf(x))); }
 
 // ------------------------------------------------------------------ workspace
-// Header (256 bytes) followed by per-(sequence, segment) records.
+// Header (256 bytes) followed by the gate factors and per-chunk records.
 struct WsHeader {
-  uint32_t status;  // first device-side error code (0 = none)
-  uint32_t done;    // CTAs finished in the current launch (last one resets the flags)
-  uint32_t pad[62];
+  uint32_t status;  // first device-side condition (0 = none)
+  uint32_t pad[63];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
 __device__ __forceinline__ void set_status(uint32_t* status, uint32_t code) { atomicCAS(status, 0u, code); }
 
-__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Spin (bounded by time) until *flag == want.  Returns false on timeout.
-__device__ __forceinline__ bool wait_flag(const uint32_t* flag, uint32_t want, uint64_t limit_ns) {
-  if (ld_acquire(flag) == want) return true;
-  uint64_t t0;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
-  while (true) {
-    __nanosleep(64);
-    if (ld_acquire(flag) == want) return true;
-    uint64_t t1;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t1));
-    if (t1 - t0 > limit_ns) return false;
-  }
-}
-
+// Bound of every wait on the tensor core's completion barriers: far beyond any
+// legitimate wait; on expiry the kernel records DIG_ERR_DEVICE_TIMEOUT.
 constexpr uint64_t kSpinLimitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
 
 }  // namespace dig

@@ -1,0 +1,444 @@
+// gla_chunk.cuh -- pieces shared by the chunk-parallel GLA kernels (forward
+// and backward): operand layouts, the unit decomposition, row loads, and the
+// chunk-state kernel (gate cumsum, per-chunk state contribution, and for the
+// backward the per-chunk state-gradient contribution).
+//
+// A unit is one chunk of C consecutive scan positions of one (batch, head)
+// sequence.  Units are independent: kernels loop over them persistently and
+// never wait on one another.
+#pragma once
+#include <type_traits>
+
+#include "gla.h"
+#include "gla_common.cuh"
+
+namespace dig {
+
+template <int C_, int DK_, int DV_, typename TIN>
+struct ChunkCfg {
+  static constexpr int C = C_, DK = DK_, DV = DV_;
+  static constexpr int NTG = std::is_same<TIN, float>::value ? 3 : 2;  // terms of gated operands
+  static constexpr int NTV = std::is_same<TIN, float>::value ? 3 : 1;  // terms of raw v / dO
+  static constexpr int DKP = cround(DK, 16), DVP = cround(DV, 16);
+  // per-thread channel halves for TMEM row reads (multiples of 4 so rows stay 16-byte aligned)
+  static constexpr int DK0 = cround((DK + 1) / 2, 4), DK1 = DK - DK0;
+  static constexpr int DV0 = cround((DV + 1) / 2, 8), DV1 = DV - DV0;
+  // Operands are token rows (bf16, K-major over channels: 8-row x 16-byte core
+  // matrices, LBO = 128 between 8-channel groups, SBO = row-group stride), read
+  // K-major or, for products that contract over tokens, MN-major.
+  static constexpr int SBO_K = DKP * 16;            // rows of DKP values (q, k, khat, S', dH')
+  static constexpr int SBO_V = DVP * 16;            // rows of DVP values (v, dO)
+  static constexpr int AQ_SZ = (C / 8) * SBO_K;     // one term, C rows
+  static constexpr int VR_SZ = (C / 8) * SBO_V;     // one term, C rows
+  static constexpr int SPT_SZ = (DVP / 8) * SBO_K;  // one term, DVP rows
+  // an M = 128 read of C-row operands covers 128 rows (K-major) or, read
+  // MN-major as v^T / dO^T, 16 channel groups of every token group
+  static constexpr int AQ_READ = (NTG - 1) * AQ_SZ + 16 * SBO_K;
+  static constexpr int VR_READ = cmax((NTV - 1) * VR_SZ + (C / 8 - 1) * SBO_V + 16 * 128,
+                                      (NTV - 1) * VR_SZ + 16 * SBO_V);
+  // ---- row pieces of the coalesced loads and stores (see piece_of)
+  static constexpr int PSK = DK % 8 == 0 ? 8 : 4;  // channels per piece of q / k rows
+  static constexpr int NGK = DK / PSK;
+  static constexpr int NPK = cdiv(C * NGK, 256);    // pieces per thread
+  static constexpr int NGZ = DK / 4;                // gate logits / factors: 4 fp32 channels per piece
+  static constexpr int NPZ = cdiv(C * NGZ, 256);
+  static constexpr int NGS = DK / 4;                // state rows (fp32)
+  static constexpr int NPS = cdiv(DV * NGS, 256);
+  static constexpr int NGV = DV / 8;                // v / dO / r / o / y / dv rows: 8 channels per piece
+  static constexpr int NPV = cdiv(C * NGV, 256);
+  static constexpr int NPAD = (DKP - DK) / 4;       // zero pieces of the key-channel padding, per row
+  static constexpr int NPADV = (DVP - DV) / 8;      // zero pieces of the value-channel padding, per row
+  static_assert(DK % 4 == 0 && DV % 8 == 0 && DK1 > 0 && DV1 > 0 && DK <= 64 && DV <= 128, "head dims");
+  static_assert(C == 32 || C == 64 || C == 128, "chunk");
+};
+
+// Layout of the chunk-state kernel (BWD adds q 2^b and dO operands).
+template <int C, int DK, int DV, typename TIN, bool BWD>
+struct StateCfg {
+  using K = ChunkCfg<C, DK, DV, TIN>;
+  static constexpr int OFF_KH = 0;
+  static constexpr int OFF_QB = OFF_KH + K::NTG * K::AQ_SZ;  // BWD: q 2^b
+  static constexpr int OFF_VR = OFF_QB + (BWD ? K::NTG * K::AQ_SZ : 0);
+  static constexpr int OFF_DO = OFF_VR + K::NTV * K::VR_SZ;  // BWD: dO
+  static constexpr int END_ROWS = OFF_DO + (BWD ? K::NTV * K::VR_SZ : 0);
+  static constexpr int GP = DK + 4;                 // row pitch (floats) of the cumsum buffer
+  static constexpr int OFF_G = cround(END_ROWS, 16);
+  static constexpr int SDP = DK + 4;                // row pitch of the dS / dH staging rows
+  static constexpr int OFF_SD = OFF_G + C * GP * 4;
+  // the M = 128 reads of v^T / dO^T may run past their rows into the next
+  // buffers (those lanes are unused); they only have to stay inside the allocation
+  static constexpr int SMEM = cmax(cmax(OFF_SD + (BWD ? 2 : 1) * DV * SDP * 4, OFF_VR + K::VR_READ),
+                                   BWD ? OFF_DO + K::VR_READ : 0);
+  static constexpr int NSG = 256 / DK;              // token segments of the cumsum
+  static constexpr int SEGL = cdiv(C, NSG);
+  static constexpr int TM_DH = K::DKP;              // BWD: dH columns after dS
+  static constexpr int TM_COLS = pow2ceil((BWD ? 2 : 1) * K::DKP);
+  static constexpr int PER_SM = SMEM <= 72 * 1024 ? 3 : SMEM <= 110 * 1024 ? 2 : 1;  // resident CTAs per SM
+  static_assert(SMEM <= 225 * 1024, "shared-memory budget");
+  static_assert(NSG <= 8, "cumsum segments");
+};
+
+struct StateSmem {
+  float segtot[8][64];  // cumsum totals of the token segments
+  float gam[64];        // chunk decay Gamma (log2)
+  uint64_t bar;
+  uint32_t tmem;
+};
+
+// Unit u -> (sequence bh, chunk n); units of one sequence are consecutive.
+struct Unit {
+  int bh, n, b, h, bz;
+  __device__ Unit(const GlaArgs& a, int u) {
+    bh = u / a.nchunks;
+    n = u - bh * a.nchunks;
+    b = bh / a.H;
+    h = bh - b * a.H;
+    bz = b * a.gate_heads + (a.gate_heads == 1 ? 0 : h);
+  }
+};
+
+// Rows of a [B, L, H, DV] tensor (v or dO) for the unit's chunk into a K-major
+// operand buffer at `vr` (token rows of DVP channels).  bf16 values are copied
+// unchanged (one exact term) by asynchronous 16-byte copies, zero-filled past
+// the sequence end (complete after cp_async_wait_all); fp32 values are split
+// into three bf16 terms.  Channels DV..DVP are zeroed (they are a contracted
+// dimension in some products).
+template <int C, int DK, int DV, typename TIN>
+__device__ __forceinline__ void load_v_rows(const GlaArgs& a, const Unit& U, const void* src, uint32_t vr) {
+  using Cfg = ChunkCfg<C, DK, DV, TIN>;
+  const int tid = threadIdx.x;
+  if constexpr (std::is_same<TIN, __nv_bfloat16>::value) {
+#pragma unroll
+    for (int j = 0; j < Cfg::NPV; ++j) {
+      const int i = tid + 256 * j;
+      int t, g;
+      piece_of<Cfg::NGV>(i, t, g);
+      if (i < C * Cfg::NGV) {
+        const int p = U.n * C + t;
+        const bool valid = p < a.L;
+        const long long grow = valid ? (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode) : 0;
+        cp_async16_zfill(row_addr(vr, t, Cfg::SBO_V) + 128u * g,
+                         reinterpret_cast<const TIN*>(src) + ((size_t)grow * a.H + U.h) * DV + 8 * g, valid);
+      }
+    }
+  } else {
+    Piece<TIN, 8> pv[Cfg::NPV];
+#pragma unroll
+    for (int j = 0; j < Cfg::NPV; ++j) {
+      const int i = tid + 256 * j;
+      int t, g;
+      piece_of<Cfg::NGV>(i, t, g);
+      const int p = U.n * C + t;
+      const bool valid = i < C * Cfg::NGV && p < a.L;
+      const long long grow = valid ? (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode) : 0;
+      pv[j].load(reinterpret_cast<const TIN*>(src) + ((size_t)grow * a.H + U.h) * DV + 8 * g, valid);
+    }
+#pragma unroll
+    for (int j = 0; j < Cfg::NPV; ++j) {
+      const int i = tid + 256 * j;
+      int t, g;
+      piece_of<Cfg::NGV>(i, t, g);
+      if (i < C * Cfg::NGV) {
+        float x[8];
+        pv[j].unpack(x);
+        st_piece<Cfg::NTV, 8>(vr, t, Cfg::SBO_V, 8 * g, Cfg::VR_SZ, x);
+      }
+    }
+  }
+  if constexpr (Cfg::NPADV > 0) {
+    const float zz[8] = {};
+    for (int i = tid; i < C * Cfg::NPADV; i += 256)
+      st_piece<Cfg::NTV, 8>(vr, i / Cfg::NPADV, Cfg::SBO_V, DV + 8 * (i % Cfg::NPADV), Cfg::VR_SZ, zz);
+  }
+}
+
+// ============================================================== chunk state
+// Rows of a dS / dH accumulator (TMEM lane j = value channel j, columns `col0`
+// + key channels) of this thread's channel half -> staging rows.
+template <int C, int DK, int DV, typename TIN, int H>
+__device__ __forceinline__ void stage_rows_dk(uint32_t tmem, int col0, float* sd, int pitch) {
+  using Cfg = ChunkCfg<C, DK, DV, TIN>;
+  constexpr int KO = H ? Cfg::DK0 : 0, KN = H ? Cfg::DK1 : Cfg::DK0;
+  const int t = threadIdx.x & 127, wq = t >> 5;
+  if (32 * wq >= DV) return;  // warp-uniform: these lanes hold no value channel
+  float ds[cround(KN, 8)];
+#pragma unroll
+  for (int c = 0; c < cround(KN, 8); c += 8)
+    tmem_ld8(tmem + (static_cast<uint32_t>(32 * wq) << 16) + col0 + KO + c, ds + c);
+  tmem_ld_wait();
+  if (t < DV) {
+#pragma unroll
+    for (int g = 0; g < KN / 4; ++g)
+      *reinterpret_cast<float4*>(sd + t * pitch + KO + 4 * g) =
+          make_float4(ds[4 * g], ds[4 * g + 1], ds[4 * g + 2], ds[4 * g + 3]);
+  }
+}
+
+// Per unit: the gate of the chunk (inclusive cumsum b of the base-2 log decays
+// over its tokens, per key channel), stored once per gate head as the factors
+// EQ = 2^(b - r) and the chunk constants {2^r, 2^(Gamma - r), 2^Gamma, Gamma};
+// and the chunk's state contribution dS = khat^T v with khat = k 2^(Gamma - b)
+// (value-major rows, to `dsn`).  With BWD it also forms the chunk's
+// state-gradient contribution dH = (q 2^b)^T dO (to `dhn`), which the reverse
+// scan turns into the gradient of every chunk's exit state.
+template <int C, int DK, int DV, typename TIN, bool BWD>
+__global__ void __launch_bounds__(256, BWD ? 2 : 3) gla_chunk_state_kernel(const GlaArgs a) {
+  using Cfg = ChunkCfg<C, DK, DV, TIN>;
+  using SC = StateCfg<C, DK, DV, TIN, BWD>;
+  constexpr int NTG = Cfg::NTG, NTV = Cfg::NTV, DKP = Cfg::DKP, PSK = Cfg::PSK;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  __shared__ StateSmem sh;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  if (warp == 0) {
+    tmem_alloc(&sh.tmem, SC::TM_COLS);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(&sh.bar, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem;
+  const uint32_t sbase = smem_u32(smem);
+  float* G = reinterpret_cast<float*>(smem + SC::OFF_G);    // [C][GP] cumsum of log2 decays
+  float* SD = reinterpret_cast<float*>(smem + SC::OFF_SD);  // [DV][SDP] dS staging, then dH
+  const uint64_t dVRm = sdesc(sbase + SC::OFF_VR, Cfg::SBO_V, 128);
+  const uint64_t dKHm = sdesc(sbase + SC::OFF_KH, Cfg::SBO_K, 128);
+  const uint64_t dDOm = sdesc(sbase + SC::OFF_DO, Cfg::SBO_V, 128);
+  const uint64_t dQBm = sdesc(sbase + SC::OFF_QB, Cfg::SBO_K, 128);
+  const int nunits = a.B * a.H * a.nchunks;
+  uint32_t ph = 0;
+  bool timed_out = false, bad = false;
+
+  for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+    const Unit U(a, u);
+    const bool writer = a.gate_heads != 1 || U.h == 0;  // one unit per gate head stores the factors
+    const int hz = U.bz - U.b * a.gate_heads;
+    // ---- loads: gate logits, k (and q) pieces; v (and dO) straight into operand rows
+    Piece<float, 4> pz[Cfg::NPZ];
+    Piece<TIN, PSK> pk[Cfg::NPK], pq[BWD ? Cfg::NPK : 1];
+#pragma unroll
+    for (int j = 0; j < Cfg::NPZ; ++j) {
+      const int i = tid + 256 * j;
+      int t, g;
+      piece_of<Cfg::NGZ>(i, t, g);
+      const int p = U.n * C + t;
+      const bool valid = i < C * Cfg::NGZ && p < a.L;
+      const long long grow = valid ? (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode) : 0;
+      pz[j].load(a.z + ((size_t)grow * a.gate_heads + hz) * DK + 4 * g, valid);
+    }
+#pragma unroll
+    for (int j = 0; j < Cfg::NPK; ++j) {
+      const int i = tid + 256 * j;
+      int t, g;
+      piece_of<Cfg::NGK>(i, t, g);
+      const int p = U.n * C + t;
+      const bool valid = i < C * Cfg::NGK && p < a.L;
+      const long long grow = valid ? (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode) : 0;
+      const size_t off = ((size_t)grow * a.H + U.h) * DK + g * PSK;
+      pk[j].load(reinterpret_cast<const TIN*>(a.k) + off, valid);
+      if constexpr (BWD) pq[j].load(reinterpret_cast<const TIN*>(a.q) + off, valid);
+    }
+    load_v_rows<C, DK, DV, TIN>(a, U, a.v, sbase + SC::OFF_VR);
+    if constexpr (BWD) load_v_rows<C, DK, DV, TIN>(a, U, a.dO, sbase + SC::OFF_DO);
+    // ---- inclusive cumsum over the chunk's tokens, per key channel (shared memory)
+#pragma unroll
+    for (int j = 0; j < Cfg::NPZ; ++j) {
+      const int i = tid + 256 * j;
+      int t, g;
+      piece_of<Cfg::NGZ>(i, t, g);
+      if (i < C * Cfg::NGZ) {
+        const int p = U.n * C + t;
+        float zz[4];
+        pz[j].unpack(zz);
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);  // padding tokens do not decay
+        if (p < a.L)
+          x = make_float4(log2_decay(zz[0], a.inv_tau), log2_decay(zz[1], a.inv_tau), log2_decay(zz[2], a.inv_tau),
+                          log2_decay(zz[3], a.inv_tau));
+        *reinterpret_cast<float4*>(G + t * SC::GP + 4 * g) = x;
+      }
+    }
+    __syncthreads();
+    const int sc = tid % DK, sg = tid / DK;
+    const int t0 = sg * SC::SEGL, t1 = min(C, t0 + SC::SEGL);
+    if (sg < SC::NSG) {
+      float acc = 0.f;
+      for (int t = t0; t < t1; ++t) {
+        acc += G[t * SC::GP + sc];
+        G[t * SC::GP + sc] = acc;
+      }
+      sh.segtot[sg][sc] = acc;
+    }
+    __syncthreads();
+    if (sg < SC::NSG) {
+      float pre = 0.f, tot = 0.f;
+      for (int s2 = 0; s2 < SC::NSG; ++s2) {
+        const float x = sh.segtot[s2][sc];
+        pre += s2 < sg ? x : 0.f;
+        tot += x;
+      }
+      if (sg > 0)
+        for (int t = t0; t < t1; ++t) G[t * SC::GP + sc] += pre;
+      if (sg == 0) sh.gam[sc] = tot;
+    }
+    __syncthreads();
+    const float* Gr = G + (C / 2 - 1) * SC::GP;  // b at the reference token
+    // ---- gate factors (one writer per gate head)
+#pragma unroll
+    for (int j = 0; j < Cfg::NPZ; ++j) {
+      const int i = tid + 256 * j;
+      int t, g;
+      piece_of<Cfg::NGZ>(i, t, g);
+      const int p = U.n * C + t;
+      if (i < C * Cfg::NGZ && p < a.L) {
+        const float4 bt = *reinterpret_cast<const float4*>(G + t * SC::GP + 4 * g);
+        const float4 rr = *reinterpret_cast<const float4*>(Gr + 4 * g);
+        const float d0 = bt.x - rr.x, d1 = bt.y - rr.y, d2 = bt.z - rr.z, d3 = bt.w - rr.w;
+        bad |= fmaxf(fmaxf(fabsf(d0), fabsf(d1)), fmaxf(fabsf(d2), fabsf(d3))) > 115.f;
+        if (writer)
+          *reinterpret_cast<float4*>(a.gEQ + ((size_t)U.bz * a.L + p) * DK + 4 * g) =
+              make_float4(exp2f(d0), exp2f(d1), exp2f(d2), exp2f(d3));
+      }
+    }
+    if (writer && tid < DK) {
+      float* ch = a.gCH + ((size_t)U.bz * a.nchunks + U.n) * 4 * DK + tid;
+      const float r = Gr[tid], gm = sh.gam[tid];
+      ch[0 * DK] = exp2f(r);
+      ch[1 * DK] = exp2f(gm - r);
+      ch[2 * DK] = exp2f(gm);
+      ch[3 * DK] = gm;
+    }
+    // ---- khat = k 2^(Gamma - b)   (BWD: and q 2^b)
+#pragma unroll
+    for (int j = 0; j < Cfg::NPK; ++j) {
+      const int i = tid + 256 * j;
+      int t, g;
+      piece_of<Cfg::NGK>(i, t, g);
+      if (i < C * Cfg::NGK) {
+        float kv[PSK];
+        pk[j].unpack(kv);
+#pragma unroll
+        for (int e = 0; e < PSK; ++e) kv[e] *= exp2f(sh.gam[g * PSK + e] - G[t * SC::GP + g * PSK + e]);
+        st_piece<NTG, PSK>(sbase + SC::OFF_KH, t, Cfg::SBO_K, g * PSK, Cfg::AQ_SZ, kv);
+        if constexpr (BWD) {
+          float qv[PSK];
+          pq[j].unpack(qv);
+#pragma unroll
+          for (int e = 0; e < PSK; ++e) qv[e] *= exp2f(G[t * SC::GP + g * PSK + e]);
+          st_piece<NTG, PSK>(sbase + SC::OFF_QB, t, Cfg::SBO_K, g * PSK, Cfg::AQ_SZ, qv);
+        }
+      }
+    }
+    if constexpr (Cfg::NPAD > 0) {
+      const float zz[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int i = tid; i < C * Cfg::NPAD; i += 256) {
+        st_piece<NTG, 4>(sbase + SC::OFF_KH, i / Cfg::NPAD, Cfg::SBO_K, DK + 4 * (i % Cfg::NPAD), Cfg::AQ_SZ, zz);
+        if constexpr (BWD)
+          st_piece<NTG, 4>(sbase + SC::OFF_QB, i / Cfg::NPAD, Cfg::SBO_K, DK + 4 * (i % Cfg::NPAD), Cfg::AQ_SZ, zz);
+      }
+    }
+    cp_async_wait_all();
+    // ---- dS = v^T khat, dH = dO^T (q 2^b)  (M = value channels, N = key channels, K = tokens)
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+      mma_issue<NTV, NTG, C / 16>(tmem, dVRm, Cfg::VR_SZ, 2 * Cfg::SBO_V, dKHm, Cfg::AQ_SZ, 2 * Cfg::SBO_K,
+                                  idesc_bf16(128, DKP, true, true), false);
+      if constexpr (BWD)
+        mma_issue<NTV, NTG, C / 16>(tmem + SC::TM_DH, dDOm, Cfg::VR_SZ, 2 * Cfg::SBO_V, dQBm, Cfg::AQ_SZ,
+                                    2 * Cfg::SBO_K, idesc_bf16(128, DKP, true, true), false);
+      mma_commit(&sh.bar);
+    }
+    if (!mbar_wait(&sh.bar, ph, kSpinLimitNs)) timed_out = true;
+    ph ^= 1u;
+    tc_fence_after();
+    if (tid < 128) stage_rows_dk<C, DK, DV, TIN, 0>(tmem, 0, SD, SC::SDP);
+    else stage_rows_dk<C, DK, DV, TIN, 1>(tmem, 0, SD, SC::SDP);
+    if constexpr (BWD) {
+      if (tid < 128) stage_rows_dk<C, DK, DV, TIN, 0>(tmem, SC::TM_DH, SD + DV * SC::SDP, SC::SDP);
+      else stage_rows_dk<C, DK, DV, TIN, 1>(tmem, SC::TM_DH, SD + DV * SC::SDP, SC::SDP);
+    }
+    tc_fence_before();
+    __syncthreads();
+    // ---- coalesced copies of dS (and dH): DV x DK, contiguous per unit
+    {
+      float4* dst = reinterpret_cast<float4*>(a.dsn + (size_t)u * DV * DK);
+      for (int i = tid; i < DV * DK / 4; i += 256) {
+        const int row = i / (DK / 4), c4 = i - row * (DK / 4);
+        __stcg(dst + i, *reinterpret_cast<const float4*>(SD + row * SC::SDP + 4 * c4));
+      }
+      if constexpr (BWD) {
+        float4* dh = reinterpret_cast<float4*>(a.dhn + (size_t)u * DV * DK);
+        for (int i = tid; i < DV * DK / 4; i += 256) {
+          const int row = i / (DK / 4), c4 = i - row * (DK / 4);
+          __stcg(dh + i, *reinterpret_cast<const float4*>(SD + (DV + row) * SC::SDP + 4 * c4));
+        }
+      }
+    }
+    __syncthreads();  // operands, staging and the cumsum buffer are reused by the next unit
+  }
+  if (bad) set_status(a.status, DIG_ERR_GATE_RANGE);
+  if (timed_out) set_status(a.status, DIG_ERR_DEVICE_TIMEOUT);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, SC::TM_COLS);
+}
+
+// Issues D (+)= A * B with A's NA terms in TMEM (term i of K-step s at column
+// a_tm + i * 8 + s * a_kstep) and B's NB terms in shared memory.
+template <int NA, int NB, int KSTEPS>
+__device__ __forceinline__ void mma_issue_ts(uint32_t dtm, uint32_t a_tm, uint32_t a_kstep, uint64_t b0,
+                                             uint32_t b_term, uint32_t b_kstep, uint32_t idesc, bool accumulate) {
+  constexpr int ORD = NA > NB ? NA : NB;
+  bool first = !accumulate;
+#pragma unroll
+  for (int i = 0; i < NA; ++i) {
+#pragma unroll
+    for (int j = 0; j < NB; ++j) {
+      if (i + j >= ORD) continue;
+#pragma unroll
+      for (int s = 0; s < KSTEPS; ++s) {
+        mma_bf16_ts(dtm, a_tm + i * 8 + s * a_kstep, b0 + (uint64_t)((j * b_term + s * b_kstep) >> 4), idesc,
+                    first ? 0u : 1u);
+        first = false;
+      }
+    }
+  }
+}
+
+// O rows (TMEM lane t = token t) of this thread's channel half -> staging and
+// the row's partial sum of squares.
+int num_sms();
+// Persistent grid: `per_sm` CTAs per SM (the residency each kernel is sized
+// for), never more than there are units.  Units are independent, so CTAs that
+// do not fit at once simply start later.
+inline int persistent_grid(int per_sm, long long units) {
+  const long long slots = (long long)per_sm * num_sms();
+  return (int)(units < slots ? units : slots);
+}
+
+// Chunk-state kernel launch (sets its shared-memory limit first).
+template <int C, int DK, int DV, typename TIN, bool BWD>
+cudaError_t launch_chunk_state(const GlaArgs& a, cudaStream_t s) {
+  using SC = StateCfg<C, DK, DV, TIN, BWD>;
+  const long long units = (long long)a.B * a.H * a.nchunks;
+  if (units <= 0) return cudaSuccess;
+  auto k1 = gla_chunk_state_kernel<C, DK, DV, TIN, BWD>;
+  cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, SC::SMEM);
+  if (e != cudaSuccess) return e;
+  k1<<<persistent_grid(SC::PER_SM, units), 256, SC::SMEM, s>>>(a);
+  return cudaGetLastError();
+}
+
+// Scan of per-chunk contributions X_n (DV x DK fp32 each, per sequence) into
+// the state entering every chunk: Y_0 = 0, Y_{n+1} = diag(2^Gamma_n) Y_n + X_n
+// (reverse = true: the same recurrence from the last chunk down, giving the
+// gradient leaving every chunk).  In place in `buf`.
+cudaError_t launch_state_scan(const GlaArgs& a, float* buf, bool reverse, int dk, int dv, cudaStream_t s);
+
+}  // namespace dig

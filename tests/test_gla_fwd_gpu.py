@@ -100,8 +100,9 @@ EDGE = [
     (1, 1, 3, 37, 64, 64, "f32", 1, 1 / 16, 0.0),       # fp32 ragged: 111 = 64 + 47
     (3, 4, 16, 40, 32, 64, "bf16", 4, 1 / 16, 0.0),     # one gate per head
     (2, 3, 20, 33, 36, 72, "bf16", 3, 1.0, 1.0),        # tau = 1 gates (alpha ~ sigmoid(N(1, 1.4)))
-    (64, 6, 16, 16, 32, 64, "bf16", 1, 1 / 16, 0.0),    # more sequences than SMs: one segment each
-    (1, 1, 64, 64, 32, 64, "bf16", 1, 1 / 16, 0.0),     # one sequence split over many segments
+    (64, 6, 16, 16, 32, 64, "bf16", 1, 1 / 16, 0.0),    # 384 two-chunk sequences: more units than CTAs
+    (1, 1, 64, 64, 32, 64, "bf16", 1, 1 / 16, 0.0),     # one sequence of 32 chunks over the 16 scan ranges
+    (1, 1, 128, 160, 32, 64, "bf16", 1, 1 / 16, 0.0),   # 160 chunks: two load windows per scan range
     (1, 1, 2, 2, 32, 64, "f32", 1, 1 / 16, 0.0),        # 4 tokens
 ]
 
