@@ -497,8 +497,7 @@ cudaError_t launch_typed(const GlaArgs& a, cudaStream_t s) {
   if (units <= 0) return cudaSuccess;
   cudaError_t e = launch_chunk_state<C, DK, DV, TIN, true>(a, s);
   if (e != cudaSuccess) return e;
-  if ((e = launch_state_scan(a, a.dsn, false, DK, DV, s)) != cudaSuccess) return e;
-  if ((e = launch_state_scan(a, a.dhn, true, DK, DV, s)) != cudaSuccess) return e;
+  if ((e = launch_state_scan(a, a.dsn, false, a.dhn, true, DK, DV, s)) != cudaSuccess) return e;
   auto k = gla_chunk_grad_kernel<C, DK, DV, TIN, TOUT>;
   if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, BC::SMEM)) != cudaSuccess) return e;
   k<<<persistent_grid(1, units), 256, BC::SMEM, s>>>(a);

@@ -437,8 +437,9 @@ cudaError_t launch_chunk_state(const GlaArgs& a, cudaStream_t s) {
 
 // Scan of per-chunk contributions X_n (DV x DK fp32 each, per sequence) into
 // the state entering every chunk: Y_0 = 0, Y_{n+1} = diag(2^Gamma_n) Y_n + X_n
-// (reverse = true: the same recurrence from the last chunk down, giving the
-// gradient leaving every chunk).  In place in `buf`.
-cudaError_t launch_state_scan(const GlaArgs& a, float* buf, bool reverse, int dk, int dv, cudaStream_t s);
+// (reverse: the same recurrence from the last chunk down, giving the gradient
+// leaving every chunk).  In place in buf0 and, when not null, buf1 (one launch).
+cudaError_t launch_state_scan(const GlaArgs& a, float* buf0, bool rev0, float* buf1, bool rev1, int dk, int dv,
+                              cudaStream_t s);
 
 }  // namespace dig

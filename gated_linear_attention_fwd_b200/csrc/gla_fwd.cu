@@ -80,15 +80,23 @@ struct OutSmem {
 
 // ============================================================== 2. state scan
 // One block covers 128 state elements (32 quads of 4) of one sequence; warp w
-// of 16 owns chunks [w*per, (w+1)*per) of them in scan direction, loaded
-// eight chunks at a time.  Pass 1 folds each range into (decay product A,
-// partial state s); the carry entering range w is the fold of ranges 0..w-1;
-// pass 2 rewrites X_n with the value entering chunk n.  `reverse` runs the
-// chunks from the last to the first.
-constexpr int kScanRanges = 16;
-__global__ void __launch_bounds__(32 * kScanRanges) gla_state_scan_kernel(const GlaArgs a, float* buf, int reverse,
-                                                                          int dk, int dv) {
+// of 16 owns chunks [w*per, (w+1)*per) of them in scan direction, loaded four
+// chunks at a time.  Pass 1 folds each range into (decay product A, partial
+// state s); the carry entering range w is the fold of ranges 0..w-1; pass 2
+// rewrites X_n with the value entering chunk n.  blockIdx.y selects one of two
+// buffers (the backward scans its states forward and its state gradients in
+// reverse in the same launch); `reverse` runs the chunks from the last to the
+// first.
+constexpr int kScanRanges = 16, kScanWindow = 4;
+struct ScanJob {
+  float* buf[2];
+  int reverse[2];
+};
+__global__ void __launch_bounds__(32 * kScanRanges, 2) gla_state_scan_kernel(const GlaArgs a, ScanJob job, int dk,
+                                                                             int dv) {
   __shared__ float4 sA[kScanRanges][32], sS[kScanRanges][32];
+  float* buf = blockIdx.y ? job.buf[1] : job.buf[0];
+  const int reverse = blockIdx.y ? job.reverse[1] : job.reverse[0];
   const int nq = dv * dk / 4;
   const int nblk = (nq + 31) / 32;
   const int bh = blockIdx.x / nblk, blk = blockIdx.x - bh * nblk;
@@ -104,23 +112,23 @@ __global__ void __launch_bounds__(32 * kScanRanges) gla_state_scan_kernel(const 
   float4* st = reinterpret_cast<float4*>(buf + (size_t)bh * nch * dv * dk) + quad;
   const size_t st_stride = (size_t)nq;
   const float* dec = a.gCH + ((size_t)bz * nch * 4 + 2) * dk + c0;  // 2^Gamma of chunk n at dec + n * 4 * dk
-  auto at = [&](int n) { return reverse ? nch - 1 - n : n; };  // physical chunk of scan step n
+  auto at = [&](int n) { return reverse ? nch - 1 - n : n; };         // physical chunk of scan step n
   auto fma4 = [](float4 g, float4 s, float4 d) {
     return make_float4(fmaf(g.x, s.x, d.x), fmaf(g.y, s.y, d.y), fmaf(g.z, s.z, d.z), fmaf(g.w, s.w, d.w));
   };
   float4 A = make_float4(1.f, 1.f, 1.f, 1.f), s = make_float4(0.f, 0.f, 0.f, 0.f);
   if (act) {
-    for (int w0 = n0; w0 < n1; w0 += 8) {
-      float4 g[8], d[8];
+    for (int w0 = n0; w0 < n1; w0 += kScanWindow) {
+      float4 g[kScanWindow], d[kScanWindow];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
+      for (int e = 0; e < kScanWindow; ++e) {
         if (w0 + e < n1) {
           g[e] = __ldg(reinterpret_cast<const float4*>(dec + (size_t)at(w0 + e) * 4 * dk));
           d[e] = __ldcg(st + at(w0 + e) * st_stride);
         }
       }
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
+      for (int e = 0; e < kScanWindow; ++e) {
         if (w0 + e < n1) {
           s = fma4(g[e], s, d[e]);
           A = make_float4(g[e].x * A.x, g[e].y * A.y, g[e].z * A.z, g[e].w * A.w);
@@ -134,17 +142,17 @@ __global__ void __launch_bounds__(32 * kScanRanges) gla_state_scan_kernel(const 
   if (!act) return;
   float4 S = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int m = 0; m < w; ++m) S = fma4(sA[m][lanei], S, sS[m][lanei]);
-  for (int w0 = n0; w0 < n1; w0 += 8) {
-    float4 g[8], d[8];
+  for (int w0 = n0; w0 < n1; w0 += kScanWindow) {
+    float4 g[kScanWindow], d[kScanWindow];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
+    for (int e = 0; e < kScanWindow; ++e) {
       if (w0 + e < n1) {
         g[e] = __ldg(reinterpret_cast<const float4*>(dec + (size_t)at(w0 + e) * 4 * dk));
         d[e] = __ldcg(st + at(w0 + e) * st_stride);
       }
     }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
+    for (int e = 0; e < kScanWindow; ++e) {
       if (w0 + e < n1) {
         __stcg(st + at(w0 + e) * st_stride, S);
         S = fma4(g[e], S, d[e]);
@@ -414,12 +422,14 @@ int num_sms() {
   return g_sms_cache[dev];
 }
 
-cudaError_t launch_state_scan(const GlaArgs& a, float* buf, bool reverse, int dk, int dv, cudaStream_t s) {
+cudaError_t launch_state_scan(const GlaArgs& a, float* buf0, bool rev0, float* buf1, bool rev1, int dk, int dv,
+                              cudaStream_t s) {
   const int nq = dv * dk / 4;
   const long long blocks = (long long)a.B * a.H * ((nq + 31) / 32);
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 2147483647LL) return cudaErrorInvalidValue;
-  gla_state_scan_kernel<<<(unsigned)blocks, 32 * kScanRanges, 0, s>>>(a, buf, reverse ? 1 : 0, dk, dv);
+  ScanJob job{{buf0, buf1}, {rev0 ? 1 : 0, rev1 ? 1 : 0}};
+  gla_state_scan_kernel<<<dim3((unsigned)blocks, buf1 ? 2u : 1u), 32 * kScanRanges, 0, s>>>(a, job, dk, dv);
   return cudaGetLastError();
 }
 
@@ -432,7 +442,7 @@ cudaError_t launch_typed(const GlaArgs& a, cudaStream_t s) {
   if (units <= 0) return cudaSuccess;
   cudaError_t e = launch_chunk_state<C, DK, DV, TIN, false>(a, s);
   if (e != cudaSuccess) return e;
-  if ((e = launch_state_scan(a, a.dsn, false, DK, DV, s)) != cudaSuccess) return e;
+  if ((e = launch_state_scan(a, a.dsn, false, nullptr, false, DK, DV, s)) != cudaSuccess) return e;
   auto k3 = gla_chunk_out_kernel<C, DK, DV, TIN, TOUT>;
   if ((e = cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, OC::SMEM)) != cudaSuccess) return e;
   k3<<<persistent_grid(2, units), 256, OC::SMEM, s>>>(a);
