@@ -18,19 +18,20 @@
 // Kernels: the forward's chunk-state kernel in backward mode (dS_n and dH_n per
 // chunk), the state scan forward over dS (entry states S_n) and in reverse over
 // dH (exit gradients G_n), then gla_chunk_grad_kernel over independent
-// (sequence, chunk) units.  dP, dP^T and P^T are formed by separate tensor-core
-// products so none needs a transpose; each is masked and converted to two bf16
-// terms in place in TMEM, where the second batch of products reads it as its A
-// operand.
+// (sequence, chunk) units.  P^T, dP^T and dP are formed by separate tensor-core
+// products so none needs a transpose.  They take turns in one TMEM region: each
+// is masked and converted to two bf16 terms in place, then read as the A operand
+// of its gradient product before the next one overwrites the region.  With the
+// three gradient accumulators this is 256 TMEM columns, so two CTAs share an SM.
 #include "gla_chunk.cuh"
 
 namespace dig {
 
-// Backward chunk length: 128 tokens when the three P-type matrices and the
-// three gradient accumulators fit the 512 TMEM columns (and, for fp32 inputs,
-// their three-term operands fit shared memory), else 64.
+// Backward chunk length: 128 tokens when one C x C region and the three
+// gradient accumulators fit 256 TMEM columns (two CTAs per SM) and the operands
+// fit shared memory (bf16 inputs), else 64.
 __host__ __device__ constexpr int bwd_chunk_len(int dk, int dv, bool f32) {
-  return !f32 && 3 * 128 + 2 * cround(dk, 16) + cround(dv, 16) <= 512 ? 128 : 64;
+  return !f32 && 128 + 2 * cround(dk, 16) + cround(dv, 16) <= 256 ? 128 : 64;
 }
 
 template <int C, int DK, int DV, typename TIN>
@@ -46,22 +47,24 @@ struct BwdCfg {
   static constexpr int OFF_SP = OFF_DO + NTV * K::VR_SZ;
   static constexpr int OFF_GT = OFF_SP + NTG * K::SPT_SZ;
   static constexpr int END_OPS = OFF_GT + NTG * K::SPT_SZ;
-  // staging of the gradient rows
+  // staging of the gradient rows, over the operands once every product is done
   static constexpr int VP = DV + 4, KP = DK + 4;
-  static constexpr int OFF_SV = cround(END_OPS, 16);
+  static constexpr int OFF_SV = 0;
   static constexpr int OFF_SQ = OFF_SV + C * VP * 4;
   static constexpr int OFF_SK = OFF_SQ + C * KP * 4;
-  static constexpr int OFF_SX = OFF_SK + C * KP * 4;
+  static constexpr int END_STAGE = OFF_SK + C * KP * 4;
+  // token terms of d log alpha (their own region: written while SQ / SK are read)
+  static constexpr int OFF_SX = cround(cmax(END_OPS, END_STAGE), 16);
   // M = 128 reads of C-row A operands (kbar, v, dO) may run past their rows
   // into the next buffers (those lanes are unused) but stay inside the allocation
   static constexpr int V_READ = (NTV - 1) * K::VR_SZ + 16 * K::SBO_V;
   static constexpr int SMEM = cmax(cmax(OFF_SX + C * KP * 4, OFF_K + K::AQ_READ), OFF_DO + V_READ);
-  // TMEM: P^T, dP^T, dP (fp32, then their bf16 terms in place: 8 columns per
-  // term and K-step), dqbar, dkbar, dv
+  static constexpr int PER_SM = SMEM <= 110 * 1024 ? 2 : 1;
+  // TMEM: one C x C region (P^T, then dP^T, then dP), dqbar, dkbar, dv
   static constexpr int PT_STRIDE = NTP * 8;
-  static constexpr int TM_PT = 0, TM_DPT = C, TM_DP = 2 * C;
-  static constexpr int TM_DQ = 3 * C, TM_DK = TM_DQ + K::DKP, TM_DV = TM_DK + K::DKP;
-  static constexpr int TM_COLS = 512;
+  static constexpr int TM_R = 0;
+  static constexpr int TM_DQ = C, TM_DK = TM_DQ + K::DKP, TM_DV = TM_DK + K::DKP;
+  static constexpr int TM_COLS = 256;
   static constexpr int NSG = 256 / DK;  // token segments of the d log alpha reverse cumsum
   static constexpr int SEGL = cdiv(C, NSG);
   static_assert(TM_DV + K::DVP <= TM_COLS, "TMEM budget");
@@ -72,7 +75,7 @@ struct BwdCfg {
 struct GradSmem {
   float segtot[8][64];  // reverse-cumsum totals of the token segments
   float bnd[2][64];     // rowsum(S_{n+1} o G_n), double-buffered by unit parity
-  uint64_t bar_a, bar_b;
+  uint64_t bar[6];      // completion of the six product groups of a unit
   uint32_t tmem;
 };
 
@@ -92,8 +95,12 @@ __device__ __forceinline__ void mask_to_terms(uint32_t tmem, uint32_t region, bo
     if (!zero_block) {
       tmem_ld16(tmem + lane_base + region + s0, pv);
       tmem_ld_wait();
+      // warp-uniform: only a block that crosses this warp's diagonal needs the mask
+      const bool full = upper ? (s0 >= 32 * wq + 31) : (s0 + 15 <= 32 * wq);
+      if (!full) {
 #pragma unroll
-      for (int e = 0; e < 16; ++e) pv[e] = (upper ? (s0 + e >= t) : (s0 + e <= t)) ? pv[e] : 0.f;
+        for (int e = 0; e < 16; ++e) pv[e] = (upper ? (s0 + e >= t) : (s0 + e <= t)) ? pv[e] : 0.f;
+      }
     } else {
 #pragma unroll
       for (int e = 0; e < 16; ++e) pv[e] = 0.f;
@@ -113,89 +120,34 @@ __device__ __forceinline__ void mask_to_terms(uint32_t tmem, uint32_t region, bo
   }
 }
 
-// Sum of the NT bf16 terms of N channels (from C0, multiples of 4) of one
-// K-major operand row.
-template <int NT, int C0, int N>
-struct RowReader {
-  __device__ __forceinline__ static void run(uint32_t row, uint32_t copy_bytes, float* x) {
-    if constexpr (N <= 0) {
-      return;
-    } else if constexpr (C0 % 8 == 0 && N >= 8) {
+// TMEM row of this thread (lane t, N columns from col0 + O) -> staging row.
+template <int O, int N>
+__device__ __forceinline__ void stage_row(uint32_t lane_tm, int col0, float* dst, bool store) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) x[e] = 0.f;
-#pragma unroll
-      for (int i = 0; i < NT; ++i) {
-        uint32_t w[4];
-        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
-                     : "r"(row + (C0 / 8) * 128 + i * copy_bytes));
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          x[2 * e] += __uint_as_float(w[e] << 16);
-          x[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
-        }
-      }
-      RowReader<NT, C0 + 8, N - 8>::run(row, copy_bytes, x + 8);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) x[e] = 0.f;
-#pragma unroll
-      for (int i = 0; i < NT; ++i) {
-        uint32_t w[2];
-        asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];"
-                     : "=r"(w[0]), "=r"(w[1])
-                     : "r"(row + (C0 / 8) * 128 + (C0 % 8) * 2 + i * copy_bytes));
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          x[2 * e] += __uint_as_float(w[e] << 16);
-          x[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
-        }
-      }
-      RowReader<NT, C0 + 4, N - 4>::run(row, copy_bytes, x + 4);
+  for (int c = 0; c < cround(N, 8); c += 8) {
+    float v[8];
+    tmem_ld8(lane_tm + col0 + O + c, v);
+    tmem_ld_wait();
+    if (store) {
+      if (c + 4 <= N) *reinterpret_cast<float4*>(dst + O + c) = make_float4(v[0], v[1], v[2], v[3]);
+      if (c + 8 <= N) *reinterpret_cast<float4*>(dst + O + c + 4) = make_float4(v[4], v[5], v[6], v[7]);
     }
   }
-};
+}
 
-// Gradient rows of this thread's token (TMEM lane t) and channel half ->
-// staging: dv, dqbar, dkbar, and x = qbar dqbar - kbar dkbar (the token's
-// d log alpha contribution).
+// Gradient rows of this thread's token (TMEM lane t) and channel half -> staging.
 template <int C, int DK, int DV, typename TIN, int H>
-__device__ __forceinline__ void stage_grads(uint32_t tmem, uint32_t sbase, uint8_t* smem) {
+__device__ __forceinline__ void stage_grads(uint32_t tmem, uint8_t* smem) {
   using K = ChunkCfg<C, DK, DV, TIN>;
   using BC = BwdCfg<C, DK, DV, TIN>;
   constexpr int KO = H ? K::DK0 : 0, KN = H ? K::DK1 : K::DK0;
   constexpr int VO = H ? K::DV0 : 0, VN = H ? K::DV1 : K::DV0;
   const int t = threadIdx.x & 127, wq = t >> 5;
-  const uint32_t lb = tmem + (static_cast<uint32_t>(32 * wq) << 16);
-  float dv[cround(VN, 8)], dq[cround(KN, 8)], dk[cround(KN, 8)];
-#pragma unroll
-  for (int c = 0; c < cround(VN, 8); c += 8) tmem_ld8(lb + BC::TM_DV + VO + c, dv + c);
-#pragma unroll
-  for (int c = 0; c < cround(KN, 8); c += 8) {
-    tmem_ld8(lb + BC::TM_DQ + KO + c, dq + c);
-    tmem_ld8(lb + BC::TM_DK + KO + c, dk + c);
-  }
-  tmem_ld_wait();
-  if (t >= C) return;
-  float* SV = reinterpret_cast<float*>(smem + BC::OFF_SV) + t * BC::VP;
-  float* SQ = reinterpret_cast<float*>(smem + BC::OFF_SQ) + t * BC::KP;
-  float* SK = reinterpret_cast<float*>(smem + BC::OFF_SK) + t * BC::KP;
-  float* SX = reinterpret_cast<float*>(smem + BC::OFF_SX) + t * BC::KP;
-#pragma unroll
-  for (int g = 0; g < VN / 4; ++g)
-    *reinterpret_cast<float4*>(SV + VO + 4 * g) = make_float4(dv[4 * g], dv[4 * g + 1], dv[4 * g + 2], dv[4 * g + 3]);
-  float qb[KN], kb[KN];
-  RowReader<BC::NTG, KO, KN>::run(row_addr(sbase + BC::OFF_Q, t, K::SBO_K), K::AQ_SZ, qb);
-  RowReader<BC::NTG, KO, KN>::run(row_addr(sbase + BC::OFF_K, t, K::SBO_K), K::AQ_SZ, kb);
-#pragma unroll
-  for (int g = 0; g < KN / 4; ++g) {
-    *reinterpret_cast<float4*>(SQ + KO + 4 * g) = make_float4(dq[4 * g], dq[4 * g + 1], dq[4 * g + 2], dq[4 * g + 3]);
-    *reinterpret_cast<float4*>(SK + KO + 4 * g) = make_float4(dk[4 * g], dk[4 * g + 1], dk[4 * g + 2], dk[4 * g + 3]);
-    float x[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) x[e] = qb[4 * g + e] * dq[4 * g + e] - kb[4 * g + e] * dk[4 * g + e];
-    *reinterpret_cast<float4*>(SX + KO + 4 * g) = make_float4(x[0], x[1], x[2], x[3]);
-  }
+  const uint32_t lt = tmem + (static_cast<uint32_t>(32 * wq) << 16);
+  const bool st = t < C;
+  stage_row<VO, VN>(lt, BC::TM_DV, reinterpret_cast<float*>(smem + BC::OFF_SV) + t * BC::VP, st);
+  stage_row<KO, KN>(lt, BC::TM_DQ, reinterpret_cast<float*>(smem + BC::OFF_SQ) + t * BC::KP, st);
+  stage_row<KO, KN>(lt, BC::TM_DK, reinterpret_cast<float*>(smem + BC::OFF_SK) + t * BC::KP, st);
 }
 
 __device__ __forceinline__ void st_global4(__nv_bfloat16* p, const float* v) {
@@ -214,7 +166,7 @@ __device__ __forceinline__ void st_global_piece(T* p, const float* v) {
 }
 
 template <int C, int DK, int DV, typename TIN, typename TOUT>
-__global__ void __launch_bounds__(256, 1) gla_chunk_grad_kernel(const GlaArgs a) {
+__global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a) {
   using K = ChunkCfg<C, DK, DV, TIN>;
   using BC = BwdCfg<C, DK, DV, TIN>;
   constexpr int NTG = BC::NTG, NTV = BC::NTV, NTP = BC::NTP, DKP = K::DKP, DVP = K::DVP, PSK = K::PSK;
@@ -226,8 +178,7 @@ __global__ void __launch_bounds__(256, 1) gla_chunk_grad_kernel(const GlaArgs a)
     tmem_relinquish();
   }
   if (tid == 0) {
-    mbar_init(&sh.bar_a, 1);
-    mbar_init(&sh.bar_b, 1);
+    for (int i = 0; i < 6; ++i) mbar_init(&sh.bar[i], 1);
     fence_mbar_init();
   }
   if (tid < 128) sh.bnd[tid >> 6][tid & 63] = 0.f;
@@ -250,100 +201,113 @@ __global__ void __launch_bounds__(256, 1) gla_chunk_grad_kernel(const GlaArgs a)
   uint32_t ph = 0;
   int it = 0;
   bool timed_out = false;
+  auto wait_all = [&](int i) {  // every thread: product group i of this unit is complete
+    if (!mbar_wait(&sh.bar[i], ph, kSpinLimitNs)) timed_out = true;
+    tc_fence_after();
+  };
+  auto publish = [&]() {  // this thread's TMEM / shared writes, then a CTA barrier
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  };
 
   for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
     const Unit U(a, u);
     const int hz = U.bz - U.b * a.gate_heads;
     float* bnd = sh.bnd[it & 1];
-    // ---- loads: q, k, gate-factor pieces; S_n, G_n (and S_{n+1}) rows; v and dO into operand rows
-    Piece<TIN, PSK> pq[K::NPK], pk[K::NPK];
-    Piece<float, PSK> pe[K::NPK];
-#pragma unroll
-    for (int j = 0; j < K::NPK; ++j) {
-      const int i = tid + 256 * j;
-      int tt, g;
-      piece_of<K::NGK>(i, tt, g);
-      const int p = U.n * C + tt;
-      const bool valid = i < C * K::NGK && p < a.L;
-      const long long grow = valid ? (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode) : 0;
-      const size_t off = ((size_t)grow * a.H + U.h) * DK + g * PSK;
-      pq[j].load(reinterpret_cast<const TIN*>(a.q) + off, valid);
-      pk[j].load(reinterpret_cast<const TIN*>(a.k) + off, valid);
-      pe[j].load(a.gEQ + ((size_t)U.bz * a.L + (valid ? p : 0)) * DK + g * PSK, valid);
-    }
-    const bool has_next = U.n + 1 < a.nchunks;  // G of the last chunk is zero
-    Piece<float, 4> ps[K::NPS], pg[K::NPS], pn[K::NPS], pc0[K::NPS], pc1[K::NPS];
-#pragma unroll
-    for (int j = 0; j < K::NPS; ++j) {
-      const int i = tid + 256 * j;
-      int jr, g;
-      piece_of<K::NGS>(i, jr, g);
-      const bool in = i < DV * K::NGS;
-      const size_t row = ((size_t)u * DV + (in ? jr : 0)) * DK + 4 * g;
-      ps[j].load_cg(a.dsn + row, in);
-      pg[j].load_cg(a.dhn + row, in);
-      pn[j].load_cg(a.dsn + row + (size_t)DV * DK, in && has_next);
-      const float* ch = a.gCH + ((size_t)U.bz * a.nchunks + U.n) * 4 * DK + 4 * g;
-      pc0[j].load(ch, in);
-      pc1[j].load(ch + DK, in);
-    }
+    // ---- operands: qbar, kbar rows; S' and Gt rows; v and dO rows; the boundary term of d log alpha
     load_v_rows<C, DK, DV, TIN>(a, U, a.v, sbase + BC::OFF_V);
     load_v_rows<C, DK, DV, TIN>(a, U, a.dO, sbase + BC::OFF_DO);
-    // ---- operands: qbar, kbar rows; S' and Gt rows; the boundary term of d log alpha
+    {
+      Piece<TIN, PSK> pq[K::NPK], pk[K::NPK];
+      Piece<float, PSK> pe[K::NPK];
 #pragma unroll
-    for (int j = 0; j < K::NPK; ++j) {
-      const int i = tid + 256 * j;
-      int tt, g;
-      piece_of<K::NGK>(i, tt, g);
-      if (i < C * K::NGK) {
-        const bool valid = U.n * C + tt < a.L;
-        float qv[PSK], kv[PSK], ev[PSK];
-        pq[j].unpack(qv);
-        pk[j].unpack(kv);
-        pe[j].unpack(ev);
+      for (int j = 0; j < K::NPK; ++j) {
+        const int i = tid + 256 * j;
+        int tt, g;
+        piece_of<K::NGK>(i, tt, g);
+        const int p = U.n * C + tt;
+        const bool valid = i < C * K::NGK && p < a.L;
+        const long long grow = valid ? (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode) : 0;
+        const size_t off = ((size_t)grow * a.H + U.h) * DK + g * PSK;
+        pq[j].load(reinterpret_cast<const TIN*>(a.q) + off, valid);
+        pk[j].load(reinterpret_cast<const TIN*>(a.k) + off, valid);
+        pe[j].load(a.gEQ + ((size_t)U.bz * a.L + (valid ? p : 0)) * DK + g * PSK, valid);
+      }
 #pragma unroll
-        for (int e = 0; e < PSK; ++e) {
-          const float f = valid ? ev[e] : 1.f;
-          qv[e] *= f;
-          kv[e] *= __fdividef(1.f, f);
+      for (int j = 0; j < K::NPK; ++j) {
+        const int i = tid + 256 * j;
+        int tt, g;
+        piece_of<K::NGK>(i, tt, g);
+        if (i < C * K::NGK) {
+          const bool valid = U.n * C + tt < a.L;
+          float qv[PSK], kv[PSK], ev[PSK];
+          pq[j].unpack(qv);
+          pk[j].unpack(kv);
+          pe[j].unpack(ev);
+#pragma unroll
+          for (int e = 0; e < PSK; ++e) {
+            const float f = valid ? ev[e] : 1.f;
+            qv[e] *= f;
+            kv[e] *= __fdividef(1.f, f);
+          }
+          st_piece<NTG, PSK>(sbase + BC::OFF_Q, tt, K::SBO_K, g * PSK, K::AQ_SZ, qv);
+          st_piece<NTG, PSK>(sbase + BC::OFF_K, tt, K::SBO_K, g * PSK, K::AQ_SZ, kv);
         }
-        st_piece<NTG, PSK>(sbase + BC::OFF_Q, tt, K::SBO_K, g * PSK, K::AQ_SZ, qv);
-        st_piece<NTG, PSK>(sbase + BC::OFF_K, tt, K::SBO_K, g * PSK, K::AQ_SZ, kv);
       }
     }
+    {
+      const bool has_next_chunk = U.n + 1 < a.nchunks;  // G of the last chunk is zero
+      Piece<float, 4> ps[K::NPS], pg[K::NPS], pn[K::NPS], pc0[K::NPS], pc1[K::NPS];
 #pragma unroll
-    for (int j = 0; j < K::NPS; ++j) {
-      const int i = tid + 256 * j;
-      int jr, g;
-      piece_of<K::NGS>(i, jr, g);
-      const bool in = i < DV * K::NGS;
-      float sv[4], gv[4], nv[4], c0[4], c1[4];
-      ps[j].unpack(sv);
-      pg[j].unpack(gv);
-      pn[j].unpack(nv);
-      pc0[j].unpack(c0);
-      pc1[j].unpack(c1);
-      float bp[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        bp[e] = nv[e] * gv[e];  // zero outside the rows and for the last chunk
-        sv[e] *= c0[e];         // S' = 2^r S_n
-        gv[e] *= c1[e];         // Gt = 2^(Gamma - r) G_n
+      for (int j = 0; j < K::NPS; ++j) {
+        const int i = tid + 256 * j;
+        int jr, g;
+        piece_of<K::NGS>(i, jr, g);
+        const bool in = i < DV * K::NGS;
+        const size_t row = ((size_t)u * DV + (in ? jr : 0)) * DK + 4 * g;
+        ps[j].load_cg(a.dsn + row, in);
+        pg[j].load_cg(a.dhn + row, in);
+        pn[j].load_cg(a.dsn + row + (size_t)DV * DK, in && has_next_chunk);
+        const float* ch = a.gCH + ((size_t)U.bz * a.nchunks + U.n) * 4 * DK + 4 * g;
+        pc0[j].load(ch, in);
+        pc1[j].load(ch + DK, in);
       }
-      if (in) {
-        st_piece<NTG, 4>(sbase + BC::OFF_SP, jr, K::SBO_K, 4 * g, K::SPT_SZ, sv);
-        st_piece<NTG, 4>(sbase + BC::OFF_GT, jr, K::SBO_K, 4 * g, K::SPT_SZ, gv);
-      }
-      // sum over the 8 rows of this lane group (lanes i..i+7 share the channel group)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        bp[e] += __shfl_xor_sync(0xffffffffu, bp[e], 1);
-        bp[e] += __shfl_xor_sync(0xffffffffu, bp[e], 2);
-        bp[e] += __shfl_xor_sync(0xffffffffu, bp[e], 4);
-      }
-      if (in && (i & 7) == 0) {
+      for (int j = 0; j < K::NPS; ++j) {
+        const int i = tid + 256 * j;
+        int jr, g;
+        piece_of<K::NGS>(i, jr, g);
+        const bool in = i < DV * K::NGS;
+        float sv[4], gv[4], nv[4], c0[4], c1[4];
+        ps[j].unpack(sv);
+        pg[j].unpack(gv);
+        pn[j].unpack(nv);
+        pc0[j].unpack(c0);
+        pc1[j].unpack(c1);
+        float bp[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) atomicAdd(&bnd[4 * g + e], bp[e]);
+        for (int e = 0; e < 4; ++e) {
+          bp[e] = nv[e] * gv[e];  // zero outside the rows and for the last chunk
+          sv[e] *= c0[e];         // S' = 2^r S_n
+          gv[e] *= c1[e];         // Gt = 2^(Gamma - r) G_n
+        }
+        if (in) {
+          st_piece<NTG, 4>(sbase + BC::OFF_SP, jr, K::SBO_K, 4 * g, K::SPT_SZ, sv);
+          st_piece<NTG, 4>(sbase + BC::OFF_GT, jr, K::SBO_K, 4 * g, K::SPT_SZ, gv);
+        }
+        // sum over the 8 rows of this lane group (lanes i..i+7 share the channel group)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          bp[e] += __shfl_xor_sync(0xffffffffu, bp[e], 1);
+          bp[e] += __shfl_xor_sync(0xffffffffu, bp[e], 2);
+          bp[e] += __shfl_xor_sync(0xffffffffu, bp[e], 4);
+        }
+        if (in && (i & 7) == 0) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) atomicAdd(&bnd[4 * g + e], bp[e]);
+        }
       }
     }
     {  // zero padding: key channels DK..DKP of every row; value rows DV..DVP of S' and Gt
@@ -369,53 +333,67 @@ __global__ void __launch_bounds__(256, 1) gla_chunk_grad_kernel(const GlaArgs a)
       }
     }
     cp_async_wait_all();
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    // ---- first products
+    publish();
+    // ---- P^T and the three inter-chunk terms
     if (tid == 0) {
-      mma_issue<NTG, NTG, DKP / 16>(tmem + BC::TM_PT, dKk, K::AQ_SZ, 256, dQk, K::AQ_SZ, 256, idesc_bf16(128, C),
+      mma_issue<NTG, NTG, DKP / 16>(tmem + BC::TM_R, dKk, K::AQ_SZ, 256, dQk, K::AQ_SZ, 256, idesc_bf16(128, C),
                                     false);  // P^T[s][t]
-      mma_issue<NTV, NTV, DVP / 16>(tmem + BC::TM_DPT, dVk, K::VR_SZ, 256, dDOk, K::VR_SZ, 256, idesc_bf16(128, C),
-                                    false);  // dP^T[s][t]
-      mma_issue<NTV, NTV, DVP / 16>(tmem + BC::TM_DP, dDOk, K::VR_SZ, 256, dVk, K::VR_SZ, 256, idesc_bf16(128, C),
-                                    false);  // dP[t][s]
       mma_issue<NTV, NTG, DVP / 16>(tmem + BC::TM_DQ, dDOk, K::VR_SZ, 256, dSPm, K::SPT_SZ, 2 * K::SBO_K,
                                     idesc_bf16(128, DKP, false, true), false);  // dO S'^T
       mma_issue<NTV, NTG, DVP / 16>(tmem + BC::TM_DK, dVk, K::VR_SZ, 256, dGTm, K::SPT_SZ, 2 * K::SBO_K,
                                     idesc_bf16(128, DKP, false, true), false);  // V Gt^T
       mma_issue<NTG, NTG, DKP / 16>(tmem + BC::TM_DV, dKk, K::AQ_SZ, 256, dGTk, K::SPT_SZ, 256, idesc_bf16(128, DVP),
                                     false);  // kbar Gt
-      mma_commit(&sh.bar_a);
+      mma_commit(&sh.bar[0]);
     }
-    if (!mbar_wait(&sh.bar_a, ph, kSpinLimitNs)) timed_out = true;
-    tc_fence_after();
-    mask_to_terms<C, BC::PT_STRIDE>(tmem, BC::TM_PT, true);
-    mask_to_terms<C, BC::PT_STRIDE>(tmem, BC::TM_DPT, true);
-    mask_to_terms<C, BC::PT_STRIDE>(tmem, BC::TM_DP, false);
+    wait_all(0);
+    mask_to_terms<C, BC::PT_STRIDE>(tmem, BC::TM_R, true);
     tmem_st_wait();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    // ---- second products (A operands from TMEM)
+    publish();
+    // ---- dv += P^T dO; then dP^T into the region once that product has read it
     if (tid == 0) {
-      mma_issue_ts<NTP, NTV, C / 16>(tmem + BC::TM_DV, tmem + BC::TM_PT, BC::PT_STRIDE, dDOm, K::VR_SZ, 2 * K::SBO_V,
-                                     idesc_bf16(128, DVP, false, true), true);  // dv += P^T dO
-      mma_issue_ts<NTP, NTG, C / 16>(tmem + BC::TM_DK, tmem + BC::TM_DPT, BC::PT_STRIDE, dQm, K::AQ_SZ, 2 * K::SBO_K,
-                                     idesc_bf16(128, DKP, false, true), true);  // dkbar += dP^T qbar
-      mma_issue_ts<NTP, NTG, C / 16>(tmem + BC::TM_DQ, tmem + BC::TM_DP, BC::PT_STRIDE, dKm, K::AQ_SZ, 2 * K::SBO_K,
-                                     idesc_bf16(128, DKP, false, true), true);  // dqbar += dP kbar
-      mma_commit(&sh.bar_b);
+      mma_issue_ts<NTP, NTV, C / 16>(tmem + BC::TM_DV, tmem + BC::TM_R, BC::PT_STRIDE, dDOm, K::VR_SZ, 2 * K::SBO_V,
+                                     idesc_bf16(128, DVP, false, true), true);
+      mma_commit(&sh.bar[1]);
+      if (!mbar_wait(&sh.bar[1], ph, kSpinLimitNs)) timed_out = true;
+      tc_fence_after();
+      mma_issue<NTV, NTV, DVP / 16>(tmem + BC::TM_R, dVk, K::VR_SZ, 256, dDOk, K::VR_SZ, 256, idesc_bf16(128, C),
+                                    false);  // dP^T[s][t]
+      mma_commit(&sh.bar[2]);
     }
-    if (!mbar_wait(&sh.bar_b, ph, kSpinLimitNs)) timed_out = true;
+    wait_all(2);
+    mask_to_terms<C, BC::PT_STRIDE>(tmem, BC::TM_R, true);
+    tmem_st_wait();
+    publish();
+    // ---- dkbar += dP^T qbar; then dP
+    if (tid == 0) {
+      mma_issue_ts<NTP, NTG, C / 16>(tmem + BC::TM_DK, tmem + BC::TM_R, BC::PT_STRIDE, dQm, K::AQ_SZ, 2 * K::SBO_K,
+                                     idesc_bf16(128, DKP, false, true), true);
+      mma_commit(&sh.bar[3]);
+      if (!mbar_wait(&sh.bar[3], ph, kSpinLimitNs)) timed_out = true;
+      tc_fence_after();
+      mma_issue<NTV, NTV, DVP / 16>(tmem + BC::TM_R, dDOk, K::VR_SZ, 256, dVk, K::VR_SZ, 256, idesc_bf16(128, C),
+                                    false);  // dP[t][s]
+      mma_commit(&sh.bar[4]);
+    }
+    wait_all(4);
+    mask_to_terms<C, BC::PT_STRIDE>(tmem, BC::TM_R, false);
+    tmem_st_wait();
+    publish();
+    // ---- dqbar += dP kbar
+    if (tid == 0) {
+      mma_issue_ts<NTP, NTG, C / 16>(tmem + BC::TM_DQ, tmem + BC::TM_R, BC::PT_STRIDE, dKm, K::AQ_SZ, 2 * K::SBO_K,
+                                     idesc_bf16(128, DKP, false, true), true);
+      mma_commit(&sh.bar[5]);
+    }
+    wait_all(5);
     ph ^= 1u;
-    tc_fence_after();
-    if (tid < 128) stage_grads<C, DK, DV, TIN, 0>(tmem, sbase, smem);
-    else stage_grads<C, DK, DV, TIN, 1>(tmem, sbase, smem);
+    // ---- gradient rows -> staging (the operands are no longer read)
+    if (tid < 128) stage_grads<C, DK, DV, TIN, 0>(tmem, smem);
+    else stage_grads<C, DK, DV, TIN, 1>(tmem, smem);
     tc_fence_before();
     __syncthreads();
-    // ---- dv, dq, dk rows (coalesced pieces)
+    // ---- dv, dq, dk rows (coalesced pieces); the tokens' d log alpha terms
 #pragma unroll
     for (int j = 0; j < K::NPV; ++j) {
       const int i = tid + 256 * j;
@@ -430,26 +408,55 @@ __global__ void __launch_bounds__(256, 1) gla_chunk_grad_kernel(const GlaArgs a)
         st_global8(reinterpret_cast<TOUT*>(a.dv) + ((size_t)grow * a.H + U.h) * DV + 8 * g, vv);
       }
     }
+    {
+      Piece<TIN, PSK> pq[K::NPK], pk[K::NPK];
+      Piece<float, PSK> pe[K::NPK];
 #pragma unroll
-    for (int j = 0; j < K::NPK; ++j) {
-      const int i = tid + 256 * j;
-      int tt, g;
-      piece_of<K::NGK>(i, tt, g);
-      const int p = U.n * C + tt;
-      if (i < C * K::NGK && p < a.L) {
-        const long long grow = (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode);
+      for (int j = 0; j < K::NPK; ++j) {  // q, k and the gate factors again (L2-resident)
+        const int i = tid + 256 * j;
+        int tt, g;
+        piece_of<K::NGK>(i, tt, g);
+        const int p = U.n * C + tt;
+        const bool valid = i < C * K::NGK && p < a.L;
+        const long long grow = valid ? (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode) : 0;
         const size_t off = ((size_t)grow * a.H + U.h) * DK + g * PSK;
-        float ev[PSK], dq[PSK], dk[PSK];
-        pe[j].unpack(ev);
+        pq[j].load(reinterpret_cast<const TIN*>(a.q) + off, valid);
+        pk[j].load(reinterpret_cast<const TIN*>(a.k) + off, valid);
+        pe[j].load(a.gEQ + ((size_t)U.bz * a.L + (valid ? p : 0)) * DK + g * PSK, valid);
+      }
 #pragma unroll
-        for (int e = 0; e < PSK; ++e) {
-          dq[e] = SQ[tt * BC::KP + g * PSK + e] * ev[e];
-          dk[e] = SK[tt * BC::KP + g * PSK + e] * __fdividef(1.f, ev[e]);
+      for (int j = 0; j < K::NPK; ++j) {
+        const int i = tid + 256 * j;
+        int tt, g;
+        piece_of<K::NGK>(i, tt, g);
+        const int p = U.n * C + tt;
+        if (i < C * K::NGK) {
+          const bool valid = p < a.L;
+          float qv[PSK], kv[PSK], ev[PSK], dq[PSK], dk[PSK], x[PSK];
+          pq[j].unpack(qv);
+          pk[j].unpack(kv);
+          pe[j].unpack(ev);
+#pragma unroll
+          for (int e = 0; e < PSK; ++e) {
+            const float f = valid ? ev[e] : 1.f, rf = __fdividef(1.f, f);
+            const float dqb = SQ[tt * BC::KP + g * PSK + e], dkb = SK[tt * BC::KP + g * PSK + e];
+            dq[e] = dqb * f;
+            dk[e] = dkb * rf;
+            x[e] = qv[e] * f * dqb - kv[e] * rf * dkb;  // qbar dqbar - kbar dkbar
+          }
+#pragma unroll
+          for (int e = 0; e < PSK; e += 4)
+            *reinterpret_cast<float4*>(SX + tt * BC::KP + g * PSK + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+          if (valid) {
+            const long long grow = (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode);
+            const size_t off = ((size_t)grow * a.H + U.h) * DK + g * PSK;
+            st_global_piece<PSK>(reinterpret_cast<TOUT*>(a.dq) + off, dq);
+            st_global_piece<PSK>(reinterpret_cast<TOUT*>(a.dk) + off, dk);
+          }
         }
-        st_global_piece<PSK>(reinterpret_cast<TOUT*>(a.dq) + off, dq);
-        st_global_piece<PSK>(reinterpret_cast<TOUT*>(a.dk) + off, dk);
       }
     }
+    __syncthreads();
     // ---- d log alpha: reverse cumsum over the chunk's tokens + the boundary term
     const int sc = tid % DK, sg = tid / DK;
     const int t0 = sg * BC::SEGL, t1 = min(C, t0 + BC::SEGL);
@@ -500,7 +507,7 @@ cudaError_t launch_typed(const GlaArgs& a, cudaStream_t s) {
   if ((e = launch_state_scan(a, a.dsn, false, a.dhn, true, DK, DV, s)) != cudaSuccess) return e;
   auto k = gla_chunk_grad_kernel<C, DK, DV, TIN, TOUT>;
   if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, BC::SMEM)) != cudaSuccess) return e;
-  k<<<persistent_grid(1, units), 256, BC::SMEM, s>>>(a);
+  k<<<persistent_grid(BC::PER_SM, units), 256, BC::SMEM, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -212,13 +212,14 @@ __global__ void __launch_bounds__(256, BWD ? 2 : 3) gla_chunk_state_kernel(const
   uint32_t ph = 0;
   bool timed_out = false, bad = false;
 
-  for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+  // Row pieces of a unit, loaded one unit ahead: gate logits, k (and q) are
+  // issued once the current unit's operands are written, v (and dO) once its
+  // products have completed.
+  Piece<float, 4> pz[Cfg::NPZ];
+  Piece<TIN, PSK> pk[Cfg::NPK], pq[BWD ? Cfg::NPK : 1];
+  auto issue_rows = [&](int u) {
     const Unit U(a, u);
-    const bool writer = a.gate_heads != 1 || U.h == 0;  // one unit per gate head stores the factors
     const int hz = U.bz - U.b * a.gate_heads;
-    // ---- loads: gate logits, k (and q) pieces; v (and dO) straight into operand rows
-    Piece<float, 4> pz[Cfg::NPZ];
-    Piece<TIN, PSK> pk[Cfg::NPK], pq[BWD ? Cfg::NPK : 1];
 #pragma unroll
     for (int j = 0; j < Cfg::NPZ; ++j) {
       const int i = tid + 256 * j;
@@ -241,8 +242,22 @@ __global__ void __launch_bounds__(256, BWD ? 2 : 3) gla_chunk_state_kernel(const
       pk[j].load(reinterpret_cast<const TIN*>(a.k) + off, valid);
       if constexpr (BWD) pq[j].load(reinterpret_cast<const TIN*>(a.q) + off, valid);
     }
+  };
+  auto issue_vd = [&](int u) {
+    const Unit U(a, u);
     load_v_rows<C, DK, DV, TIN>(a, U, a.v, sbase + SC::OFF_VR);
     if constexpr (BWD) load_v_rows<C, DK, DV, TIN>(a, U, a.dO, sbase + SC::OFF_DO);
+  };
+  if ((int)blockIdx.x < nunits) {
+    issue_rows(blockIdx.x);
+    issue_vd(blockIdx.x);
+  }
+
+  for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+    const Unit U(a, u);
+    const bool writer = a.gate_heads != 1 || U.h == 0;  // one unit per gate head stores the factors
+    const int un = u + gridDim.x;
+    const bool has_next = un < nunits;
     // ---- inclusive cumsum over the chunk's tokens, per key channel (shared memory)
 #pragma unroll
     for (int j = 0; j < Cfg::NPZ; ++j) {
@@ -339,6 +354,7 @@ __global__ void __launch_bounds__(256, BWD ? 2 : 3) gla_chunk_state_kernel(const
           st_piece<NTG, 4>(sbase + SC::OFF_QB, i / Cfg::NPAD, Cfg::SBO_K, DK + 4 * (i % Cfg::NPAD), Cfg::AQ_SZ, zz);
       }
     }
+    if (has_next) issue_rows(un);  // this unit's row pieces are consumed
     cp_async_wait_all();
     // ---- dS = v^T khat, dH = dO^T (q 2^b)  (M = value channels, N = key channels, K = tokens)
     fence_async_smem();
@@ -356,6 +372,7 @@ __global__ void __launch_bounds__(256, BWD ? 2 : 3) gla_chunk_state_kernel(const
     if (!mbar_wait(&sh.bar, ph, kSpinLimitNs)) timed_out = true;
     ph ^= 1u;
     tc_fence_after();
+    if (has_next) issue_vd(un);  // v (and dO) of this unit are consumed
     if (tid < 128) stage_rows_dk<C, DK, DV, TIN, 0>(tmem, 0, SD, SC::SDP);
     else stage_rows_dk<C, DK, DV, TIN, 1>(tmem, 0, SD, SC::SDP);
     if constexpr (BWD) {

@@ -69,6 +69,7 @@ struct OutCfg {
   static constexpr int TM_COLS = pow2ceil(TM_O + K::DVP);
   static_assert(TM_COLS <= 256, "two output CTAs per SM share the 512 TMEM columns");
   static_assert(SMEM <= 110 * 1024, "two output CTAs per SM share shared memory");
+  static_assert(C * OP * 4 <= OFF_VR, "the output staging leaves v's rows alone (v is prefetched during the epilogue)");
 };
 
 struct OutSmem {
@@ -219,11 +220,15 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
   uint32_t ph = 0;
   bool timed_out = false;
 
-  for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+  // Row pieces of a unit, loaded one unit ahead: q, k, gate factors, entry-state
+  // rows and 2^r are issued as soon as the current unit's operands are written,
+  // v once its P V has completed, r once its epilogue is done.
+  Piece<TIN, PSK> pq[Cfg::NPK], pk[Cfg::NPK];
+  Piece<float, PSK> pe[Cfg::NPK];
+  Piece<float, 4> ps[Cfg::NPS], pc[Cfg::NPS];
+  Piece<TIN, 8> pr[Cfg::NPV];
+  auto issue_rows = [&](int u) {
     const Unit U(a, u);
-    // ---- loads: q, k and gate-factor pieces, the entry-state rows; v straight into its operand rows
-    Piece<TIN, PSK> pq[Cfg::NPK], pk[Cfg::NPK];
-    Piece<float, PSK> pe[Cfg::NPK];
 #pragma unroll
     for (int j = 0; j < Cfg::NPK; ++j) {
       const int i = tid + 256 * j;
@@ -237,7 +242,6 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
       pk[j].load(reinterpret_cast<const TIN*>(a.k) + off, valid);
       pe[j].load(a.gEQ + ((size_t)U.bz * a.L + (valid ? p : 0)) * DK + g * PSK, valid);
     }
-    Piece<float, 4> ps[Cfg::NPS], pc[Cfg::NPS];
 #pragma unroll
     for (int j = 0; j < Cfg::NPS; ++j) {
       const int i = tid + 256 * j;
@@ -247,7 +251,31 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
       ps[j].load_cg(a.dsn + ((size_t)u * DV + (in ? jr : 0)) * DK + 4 * g, in);
       pc[j].load(a.gCH + ((size_t)U.bz * a.nchunks + U.n) * 4 * DK + 4 * g, in);
     }
-    load_v_rows<C, DK, DV, TIN>(a, U, a.v, sbase + OC::OFF_VR);
+  };
+  auto issue_r = [&](int u) {
+    if (!with_y) return;
+    const Unit U(a, u);
+#pragma unroll
+    for (int j = 0; j < Cfg::NPV; ++j) {
+      const int i = tid + 256 * j;
+      int tt, g;
+      piece_of<Cfg::NGV>(i, tt, g);
+      const int p = U.n * C + tt;
+      const bool valid = i < C * Cfg::NGV && p < a.L;
+      const long long grow = valid ? (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode) : 0;
+      pr[j].load(reinterpret_cast<const TIN*>(a.r) + ((size_t)grow * a.H + U.h) * DV + 8 * g, valid);
+    }
+  };
+  if ((int)blockIdx.x < nunits) {
+    issue_rows(blockIdx.x);
+    load_v_rows<C, DK, DV, TIN>(a, Unit(a, blockIdx.x), a.v, sbase + OC::OFF_VR);
+    issue_r(blockIdx.x);
+  }
+
+  for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+    const Unit U(a, u);
+    const int un = u + gridDim.x;
+    const bool has_next = un < nunits;
     // ---- operands: qbar = q 2^(b-r), kbar = k 2^(r-b); S'^T rows = (2^r S_n)[:, j]
 #pragma unroll
     for (int j = 0; j < Cfg::NPK; ++j) {
@@ -305,6 +333,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
                                     idesc_bf16(128, DVP), false);
       mma_commit(&sh.bar_a);
     }
+    if (has_next) issue_rows(un);  // this unit's row pieces are consumed
     if (!mbar_wait(&sh.bar_a, ph, kSpinLimitNs)) timed_out = true;
     tc_fence_after();
     // ---- mask P (s <= t) and store it as bf16 terms in TMEM, one K-step of 16 at a time
@@ -316,8 +345,10 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
         if (s0 <= 32 * wq + 31) {
           tmem_ld16(tmem + lane_base + OC::TM_P + s0, pv);
           tmem_ld_wait();
+          if (s0 + 15 > 32 * wq) {  // warp-uniform: the block crosses this warp's diagonal
 #pragma unroll
-          for (int e = 0; e < 16; ++e) pv[e] = (s0 + e <= t) ? pv[e] : 0.f;
+            for (int e = 0; e < 16; ++e) pv[e] = (s0 + e <= t) ? pv[e] : 0.f;
+          }
         } else {
 #pragma unroll
           for (int e = 0; e < 16; ++e) pv[e] = 0.f;  // the whole warp's rows precede this block
@@ -345,23 +376,10 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
                                      2 * Cfg::SBO_V, idesc_bf16(128, DVP, false, true), true);
       mma_commit(&sh.bar_b);
     }
-    // ---- epilogue inputs while P V runs
-    Piece<TIN, 8> pr[Cfg::NPV];
-    if (with_y) {
-#pragma unroll
-      for (int j = 0; j < Cfg::NPV; ++j) {
-        const int i = tid + 256 * j;
-        int tt, g;
-        piece_of<Cfg::NGV>(i, tt, g);
-        const int p = U.n * C + tt;
-        const bool valid = i < C * Cfg::NGV && p < a.L;
-        const long long grow = valid ? (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode) : 0;
-        pr[j].load(reinterpret_cast<const TIN*>(a.r) + ((size_t)grow * a.H + U.h) * DV + 8 * g, valid);
-      }
-    }
     if (!mbar_wait(&sh.bar_b, ph, kSpinLimitNs)) timed_out = true;
     ph ^= 1u;
     tc_fence_after();
+    if (has_next) load_v_rows<C, DK, DV, TIN>(a, Unit(a, un), a.v, sbase + OC::OFF_VR);  // v of this unit is consumed
     if (tid < 128) stage_o<C, DK, DV, TIN, 0>(tmem, stage, sh.red);
     else stage_o<C, DK, DV, TIN, 1>(tmem, stage, sh.red);
     tc_fence_before();
@@ -384,18 +402,27 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
         st_global8(reinterpret_cast<TOUT*>(a.o) + off, ov);
         if (with_y) {
           const float inv = rsqrtf((sh.red[tt] + sh.red[tt + 128]) / (float)DV + a.eps);
-          float rv[8], yv[8];
+          float rv[8], yv[8], gm[8];
           pr[j].unpack(rv);
+          if (a.gamma != nullptr) {
+            const float4 g0 = __ldg(reinterpret_cast<const float4*>(a.gamma + 8 * g));
+            const float4 g1 = __ldg(reinterpret_cast<const float4*>(a.gamma + 8 * g) + 1);
+            gm[0] = g0.x; gm[1] = g0.y; gm[2] = g0.z; gm[3] = g0.w;
+            gm[4] = g1.x; gm[5] = g1.y; gm[6] = g1.z; gm[7] = g1.w;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) gm[e] = 1.f;
+          }
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const float gmm = a.gamma != nullptr ? __ldg(a.gamma + 8 * g + e) : 1.f;
-            const float sw = rv[e] / (1.f + exp2f(-rv[e] * kLog2e));
-            yv[e] = sw * ov[e] * inv * gmm;
+            const float sw = __fdividef(rv[e], 1.f + exp2f(-rv[e] * kLog2e));  // Swish(r) = r sigmoid(r)
+            yv[e] = sw * ov[e] * inv * gm[e];
           }
           st_global8(reinterpret_cast<TOUT*>(a.y) + off, yv);
         }
       }
     }
+    if (has_next) issue_r(un);
     __syncthreads();  // staging and row sums are rewritten by the next unit
   }
   if (timed_out) set_status(a.status, DIG_ERR_DEVICE_TIMEOUT);
