@@ -49,24 +49,28 @@
 namespace dig {
 
 
-// Layout of the chunk-output kernel.
+// Layout of the chunk-output kernel.  P = qbar kbar^T and O = qbar S' share
+// their A operand, so kbar rows and S'^T rows are one B operand (N = C + DVP,
+// per term: C kbar rows then DVP S'^T rows) and one product fills the
+// adjacent P and O columns of TMEM.
 template <int C, int DK, int DV, typename TIN>
 struct OutCfg {
   using K = ChunkCfg<C, DK, DV, TIN>;
-  static constexpr int OFF_AQ = 0;                          // qbar
-  static constexpr int OFF_BK = K::NTG * K::AQ_SZ;          // kbar
-  static constexpr int OFF_SPT = 2 * K::NTG * K::AQ_SZ;     // S'^T rows
-  static constexpr int OFF_VR = OFF_SPT + K::NTG * K::SPT_SZ;
-  static constexpr int OP = DV + 4;                         // row pitch of the output staging (over the operands)
+  static constexpr int NB = C + K::DVP;                       // rows of the combined B operand
+  static constexpr int BS_SZ = (NB / 8) * K::SBO_K;           // one term of it
+  static constexpr int OFF_AQ = 0;                            // qbar
+  static constexpr int OFF_BS = K::NTG * K::AQ_SZ;            // kbar rows, then S'^T rows
+  static constexpr int OFF_VR = OFF_BS + K::NTG * BS_SZ;
+  static constexpr int OP = DV + 4;                           // row pitch of the output staging (over the operands)
   static constexpr int SMEM = cmax(cmax(OFF_VR + K::NTV * K::VR_SZ, OFF_AQ + K::AQ_READ), C * OP * 4);
-  // TMEM columns: P (fp32), P as bf16 terms (8 columns per term and K-step,
-  // the terms of K-step k at TM_PT + k * PT_STRIDE; in place over P when two
-  // terms fit), O
-  static constexpr int TM_P = 0;
-  static constexpr int TM_PT = K::NTG == 2 ? 0 : C;
+  // TMEM columns: P (fp32) and O side by side, P as bf16 terms (8 columns per
+  // term and K-step, the terms of K-step k at TM_PT + k * PT_STRIDE; in place
+  // over P when two terms fit)
+  static constexpr int TM_P = 0, TM_O = C;
+  static constexpr int TM_PT = K::NTG == 2 ? 0 : C + K::DVP;
   static constexpr int PT_STRIDE = K::NTG * 8;
-  static constexpr int TM_O = K::NTG == 2 ? C : C + K::NTG * C / 2;
-  static constexpr int TM_COLS = pow2ceil(TM_O + K::DVP);
+  static constexpr int TM_COLS = pow2ceil(K::NTG == 2 ? C + K::DVP : C + K::DVP + K::NTG * C / 2);
+  static_assert(NB <= 256 && NB % 16 == 0, "one M = 128 product");
   static_assert(TM_COLS <= 256, "two output CTAs per SM share the 512 TMEM columns");
   static_assert(SMEM <= 110 * 1024, "two output CTAs per SM share shared memory");
   static_assert(C * OP * 4 <= OFF_VR, "the output staging leaves v's rows alone (v is prefetched during the epilogue)");
@@ -80,36 +84,38 @@ struct OutSmem {
 };
 
 // ============================================================== 2. state scan
-// One block covers 128 state elements (32 quads of 4) of one sequence; warp w
-// of 16 owns chunks [w*per, (w+1)*per) of them in scan direction, loaded four
-// chunks at a time.  Pass 1 folds each range into (decay product A, partial
-// state s); the carry entering range w is the fold of ranges 0..w-1; pass 2
-// rewrites X_n with the value entering chunk n.  blockIdx.y selects one of two
-// buffers (the backward scans its states forward and its state gradients in
-// reverse in the same launch); `reverse` runs the chunks from the last to the
-// first.
-constexpr int kScanRanges = 16, kScanWindow = 4;
+// A block covers 64 state elements (16 quads of 4) of one sequence: lane l of
+// warp w owns quad l % 16 and chunk range 2w + l / 16 of 16, i.e. chunks
+// [range*per, (range+1)*per) in scan direction.  Pass 1 folds each range into
+// (decay product A, partial state s); the carry entering a range is the fold
+// of the ranges before it; pass 2 rewrites X_n with the value entering chunk n.
+// Ranges of up to kScanWindow chunks keep their chunks in registers between
+// the passes (two memory round trips in all); longer ones stream in windows.
+// blockIdx.y selects one of two buffers (the backward scans its states forward
+// and its state gradients in reverse in one launch); `reverse` runs the chunks
+// from the last to the first.
+constexpr int kScanRanges = 16, kScanQuads = 16, kScanWindow = 8;
 struct ScanJob {
   float* buf[2];
   int reverse[2];
 };
-__global__ void __launch_bounds__(32 * kScanRanges, 2) gla_state_scan_kernel(const GlaArgs a, ScanJob job, int dk,
-                                                                             int dv) {
-  __shared__ float4 sA[kScanRanges][32], sS[kScanRanges][32];
+__global__ void __launch_bounds__(kScanRanges * kScanQuads, 2) gla_state_scan_kernel(const GlaArgs a, ScanJob job,
+                                                                                     int dk, int dv) {
+  __shared__ float4 sA[kScanRanges][kScanQuads], sS[kScanRanges][kScanQuads];
   float* buf = blockIdx.y ? job.buf[1] : job.buf[0];
   const int reverse = blockIdx.y ? job.reverse[1] : job.reverse[0];
   const int nq = dv * dk / 4;
-  const int nblk = (nq + 31) / 32;
+  const int nblk = (nq + kScanQuads - 1) / kScanQuads;
   const int bh = blockIdx.x / nblk, blk = blockIdx.x - bh * nblk;
-  const int lanei = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int quad = blk * 32 + lanei;
+  const int lq = threadIdx.x & (kScanQuads - 1), rg = threadIdx.x / kScanQuads;
+  const int quad = blk * kScanQuads + lq;
   const bool act = quad < nq;
   const int c0 = (quad * 4) % dk;  // the quad's four key channels (dk % 4 == 0)
   const int b = bh / a.H, h = bh - b * a.H;
   const int bz = b * a.gate_heads + (a.gate_heads == 1 ? 0 : h);
   const int nch = a.nchunks;
   const int per = (nch + kScanRanges - 1) / kScanRanges;
-  const int n0 = min(nch, w * per), n1 = min(nch, n0 + per);
+  const int n0 = min(nch, rg * per), n1 = min(nch, n0 + per);
   float4* st = reinterpret_cast<float4*>(buf + (size_t)bh * nch * dv * dk) + quad;
   const size_t st_stride = (size_t)nq;
   const float* dec = a.gCH + ((size_t)bz * nch * 4 + 2) * dk + c0;  // 2^Gamma of chunk n at dec + n * 4 * dk
@@ -117,10 +123,13 @@ __global__ void __launch_bounds__(32 * kScanRanges, 2) gla_state_scan_kernel(con
   auto fma4 = [](float4 g, float4 s, float4 d) {
     return make_float4(fmaf(g.x, s.x, d.x), fmaf(g.y, s.y, d.y), fmaf(g.z, s.z, d.z), fmaf(g.w, s.w, d.w));
   };
+  auto mul4 = [](float4 g, float4 x) { return make_float4(g.x * x.x, g.y * x.y, g.z * x.z, g.w * x.w); };
   float4 A = make_float4(1.f, 1.f, 1.f, 1.f), s = make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 d[kScanWindow];
+  const bool resident = per <= kScanWindow;  // uniform: one window holds the whole range
   if (act) {
     for (int w0 = n0; w0 < n1; w0 += kScanWindow) {
-      float4 g[kScanWindow], d[kScanWindow];
+      float4 g[kScanWindow];
 #pragma unroll
       for (int e = 0; e < kScanWindow; ++e) {
         if (w0 + e < n1) {
@@ -132,19 +141,29 @@ __global__ void __launch_bounds__(32 * kScanRanges, 2) gla_state_scan_kernel(con
       for (int e = 0; e < kScanWindow; ++e) {
         if (w0 + e < n1) {
           s = fma4(g[e], s, d[e]);
-          A = make_float4(g[e].x * A.x, g[e].y * A.y, g[e].z * A.z, g[e].w * A.w);
+          A = mul4(g[e], A);
         }
       }
     }
   }
-  sA[w][lanei] = A;
-  sS[w][lanei] = s;
+  sA[rg][lq] = A;
+  sS[rg][lq] = s;
   __syncthreads();
   if (!act) return;
   float4 S = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int m = 0; m < w; ++m) S = fma4(sA[m][lanei], S, sS[m][lanei]);
+  for (int m = 0; m < rg; ++m) S = fma4(sA[m][lq], S, sS[m][lq]);
+  if (resident) {  // the range's contributions are still in registers; its decays are reread (L1)
+#pragma unroll
+    for (int e = 0; e < kScanWindow; ++e) {
+      if (n0 + e < n1) {
+        __stcg(st + at(n0 + e) * st_stride, S);
+        S = fma4(__ldg(reinterpret_cast<const float4*>(dec + (size_t)at(n0 + e) * 4 * dk)), S, d[e]);
+      }
+    }
+    return;
+  }
   for (int w0 = n0; w0 < n1; w0 += kScanWindow) {
-    float4 g[kScanWindow], d[kScanWindow];
+    float4 g[kScanWindow];
 #pragma unroll
     for (int e = 0; e < kScanWindow; ++e) {
       if (w0 + e < n1) {
@@ -212,8 +231,8 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
   const uint32_t sbase = smem_u32(smem);
   float* stage = reinterpret_cast<float*>(smem);  // [C][OP] output rows, over the operands
   const uint64_t dAQ = sdesc(sbase + OC::OFF_AQ, 128, Cfg::SBO_K);
-  const uint64_t dBK = sdesc(sbase + OC::OFF_BK, 128, Cfg::SBO_K);
-  const uint64_t dSPT = sdesc(sbase + OC::OFF_SPT, 128, Cfg::SBO_K);
+  const uint64_t dBS = sdesc(sbase + OC::OFF_BS, 128, Cfg::SBO_K);
+  const uint32_t sSPT = sbase + OC::OFF_BS + (C / 8) * Cfg::SBO_K;  // S'^T rows inside the combined operand
   const uint64_t dVRm = sdesc(sbase + OC::OFF_VR, Cfg::SBO_V, 128);
   const int nunits = a.B * a.H * a.nchunks;
   const bool with_y = a.y != nullptr && a.r != nullptr;
@@ -266,7 +285,10 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
       pr[j].load(reinterpret_cast<const TIN*>(a.r) + ((size_t)grow * a.H + U.h) * DV + 8 * g, valid);
     }
   };
-  if ((int)blockIdx.x < nunits) {
+  // Loading one unit ahead holds two units' pieces in registers; with 8-byte
+  // pieces (d_k not a multiple of 8) that spills, so those variants load per unit.
+  constexpr bool kAhead = PSK == 8;
+  if (kAhead && (int)blockIdx.x < nunits) {
     issue_rows(blockIdx.x);
     load_v_rows<C, DK, DV, TIN>(a, Unit(a, blockIdx.x), a.v, sbase + OC::OFF_VR);
     issue_r(blockIdx.x);
@@ -275,7 +297,11 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
   for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
     const Unit U(a, u);
     const int un = u + gridDim.x;
-    const bool has_next = un < nunits;
+    const bool has_next = kAhead && un < nunits;
+    if (!kAhead) {
+      issue_rows(u);
+      load_v_rows<C, DK, DV, TIN>(a, U, a.v, sbase + OC::OFF_VR);
+    }
     // ---- operands: qbar = q 2^(b-r), kbar = k 2^(r-b); S'^T rows = (2^r S_n)[:, j]
 #pragma unroll
     for (int j = 0; j < Cfg::NPK; ++j) {
@@ -295,7 +321,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
           kv[e] *= __fdividef(1.f, f);
         }
         st_piece<NTG, PSK>(sbase + OC::OFF_AQ, tt, Cfg::SBO_K, g * PSK, Cfg::AQ_SZ, qv);
-        st_piece<NTG, PSK>(sbase + OC::OFF_BK, tt, Cfg::SBO_K, g * PSK, Cfg::AQ_SZ, kv);
+        st_piece<NTG, PSK>(sbase + OC::OFF_BS, tt, Cfg::SBO_K, g * PSK, OC::BS_SZ, kv);
       }
     }
 #pragma unroll
@@ -309,7 +335,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
         pc[j].unpack(cv);
 #pragma unroll
         for (int e = 0; e < 4; ++e) sv[e] *= cv[e];
-        st_piece<NTG, 4>(sbase + OC::OFF_SPT, jr, Cfg::SBO_K, 4 * g, Cfg::SPT_SZ, sv);
+        st_piece<NTG, 4>(sSPT, jr, Cfg::SBO_K, 4 * g, OC::BS_SZ, sv);
       }
     }
     if constexpr (Cfg::NPAD > 0) {  // zero K padding (the output staging of the previous unit overwrote it)
@@ -317,8 +343,8 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
       for (int i = tid; i < C * Cfg::NPAD; i += 256) {
         const int row = i / Cfg::NPAD, c = DK + 4 * (i % Cfg::NPAD);
         st_piece<NTG, 4>(sbase + OC::OFF_AQ, row, Cfg::SBO_K, c, Cfg::AQ_SZ, zz);
-        st_piece<NTG, 4>(sbase + OC::OFF_BK, row, Cfg::SBO_K, c, Cfg::AQ_SZ, zz);
-        if (row < DV) st_piece<NTG, 4>(sbase + OC::OFF_SPT, row, Cfg::SBO_K, c, Cfg::SPT_SZ, zz);
+        st_piece<NTG, 4>(sbase + OC::OFF_BS, row, Cfg::SBO_K, c, OC::BS_SZ, zz);
+        if (row < DV) st_piece<NTG, 4>(sSPT, row, Cfg::SBO_K, c, OC::BS_SZ, zz);
       }
     }
     cp_async_wait_all();
@@ -327,10 +353,8 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
     __syncthreads();
     tc_fence_after();
     if (tid == 0) {
-      mma_issue<NTG, NTG, DKP / 16>(tmem + OC::TM_P, dAQ, Cfg::AQ_SZ, 256, dBK, Cfg::AQ_SZ, 256, idesc_bf16(128, C),
-                                    false);
-      mma_issue<NTG, NTG, DKP / 16>(tmem + OC::TM_O, dAQ, Cfg::AQ_SZ, 256, dSPT, Cfg::SPT_SZ, 256,
-                                    idesc_bf16(128, DVP), false);
+      mma_issue<NTG, NTG, DKP / 16>(tmem + OC::TM_P, dAQ, Cfg::AQ_SZ, 256, dBS, OC::BS_SZ, 256,
+                                    idesc_bf16(128, OC::NB), false);  // [P | O] = qbar [kbar | S'^T]^T
       mma_commit(&sh.bar_a);
     }
     if (has_next) issue_rows(un);  // this unit's row pieces are consumed
@@ -380,6 +404,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
     ph ^= 1u;
     tc_fence_after();
     if (has_next) load_v_rows<C, DK, DV, TIN>(a, Unit(a, un), a.v, sbase + OC::OFF_VR);  // v of this unit is consumed
+    if (!kAhead) issue_r(u);
     if (tid < 128) stage_o<C, DK, DV, TIN, 0>(tmem, stage, sh.red);
     else stage_o<C, DK, DV, TIN, 1>(tmem, stage, sh.red);
     tc_fence_before();
@@ -452,11 +477,11 @@ int num_sms() {
 cudaError_t launch_state_scan(const GlaArgs& a, float* buf0, bool rev0, float* buf1, bool rev1, int dk, int dv,
                               cudaStream_t s) {
   const int nq = dv * dk / 4;
-  const long long blocks = (long long)a.B * a.H * ((nq + 31) / 32);
+  const long long blocks = (long long)a.B * a.H * ((nq + kScanQuads - 1) / kScanQuads);
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 2147483647LL) return cudaErrorInvalidValue;
   ScanJob job{{buf0, buf1}, {rev0 ? 1 : 0, rev1 ? 1 : 0}};
-  gla_state_scan_kernel<<<dim3((unsigned)blocks, buf1 ? 2u : 1u), 32 * kScanRanges, 0, s>>>(a, job, dk, dv);
+  gla_state_scan_kernel<<<dim3((unsigned)blocks, buf1 ? 2u : 1u), kScanRanges * kScanQuads, 0, s>>>(a, job, dk, dv);
   return cudaGetLastError();
 }
 
