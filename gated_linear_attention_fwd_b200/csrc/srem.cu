@@ -9,28 +9,9 @@
 // comment for the traversal.
 #include "dig_common.cuh"
 #include "gla.h"
+#include "gla_common.cuh"
 
 namespace dig {
-
-// Raw 16-byte vector of VEC input channels, unpacked to fp32 on use.
-template <typename T>
-__device__ __forceinline__ void unpack_vec(const uint4& u, float* o);
-template <>
-__device__ __forceinline__ void unpack_vec<__nv_bfloat16>(const uint4& u, float* o) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    o[2 * i] = __uint_as_float(w[i] << 16);
-    o[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
-template <>
-__device__ __forceinline__ void unpack_vec<float>(const uint4& u, float* o) {
-  o[0] = __uint_as_float(u.x);
-  o[1] = __uint_as_float(u.y);
-  o[2] = __uint_as_float(u.z);
-  o[3] = __uint_as_float(u.w);
-}
 
 // Scan position of grid token (r, c): the inverse of the scan order.
 __device__ __forceinline__ int grid_to_scan(int r, int c, int Hg, int Wg, int mode) {
@@ -38,66 +19,120 @@ __device__ __forceinline__ int grid_to_scan(int r, int c, int Hg, int Wg, int mo
   return (mode & 1) ? Hg * Wg - 1 - t : t;
 }
 
-// Shared-memory tile: a block produces an 8 x 32 pixel tile of one image for
-// one 128-byte slice of channels.  It first loads the tile plus its one-pixel
-// halo (10 x 34 pixels x 128 bytes) with 16-byte loads issued together, then
-// each thread computes 8 outputs of one 16-byte channel vector from shared
-// memory (its 9 x VEC weights stay in registers) and stores them at their scan
-// positions.  HBM reads are the tile plus halo (~1.33x the output tile).
-constexpr int kTR = 8, kTC = 32, kSliceBytes = 128;
+// Row-streaming kernel.  A thread owns 2 consecutive channels of one grid
+// column and kRows consecutive output rows.  It issues the loads of all
+// kRows + 2 input rows x 3 columns it needs at once (consecutive lanes read
+// consecutive channel pairs of one pixel, so every warp load is contiguous),
+// then walks down the rows with a 3-row window unpacked once per row and the
+// 9 x 2 weights in registers (one contiguous 72-byte run of w per thread).
+// Consecutive grid rows of one column are a fixed step apart in every scan
+// order, so the output pointer advances by a constant.
+constexpr int kConvRows = 8;
+
+template <typename T>
+struct Pair;  // two consecutive channels as loaded
+template <>
+struct Pair<__nv_bfloat16> {
+  using type = uint32_t;
+  __device__ __forceinline__ static void unpack(uint32_t u, float* o) {
+    o[0] = __uint_as_float(u << 16);
+    o[1] = __uint_as_float(u & 0xFFFF0000u);
+  }
+  __device__ __forceinline__ static void store(__nv_bfloat16* p, float a, float b) {
+    *reinterpret_cast<uint32_t*>(p) = pack_bf16x2(a, b);
+  }
+};
+template <>
+struct Pair<float> {
+  using type = float2;
+  __device__ __forceinline__ static void unpack(float2 u, float* o) {
+    o[0] = u.x;
+    o[1] = u.y;
+  }
+  __device__ __forceinline__ static void store(float* p, float a, float b) {
+    *reinterpret_cast<float2*>(p) = make_float2(a, b);
+  }
+};
 
 template <typename TIN, typename TOUT>
-__global__ void __launch_bounds__(256) srem_dwconv_kernel(const TIN* __restrict__ x, const float* __restrict__ w,
+__global__ void __launch_bounds__(256, 3) srem_dwconv_kernel(const TIN* __restrict__ x, const float* __restrict__ w,
                                                           const float* __restrict__ bias, TOUT* __restrict__ y,
                                                           int B, int Hg, int Wg, int C, int mode) {
-  constexpr int VEC = 16 / sizeof(TIN);
-  constexpr int CS = kSliceBytes / sizeof(TIN);  // channels per slice
-  constexpr int NV = kSliceBytes / 16;            // 16-byte vectors per pixel-slice (8)
-  constexpr int TW = kTC + 2, TH = kTR + 2;
-  __shared__ uint4 tile[TH * TW * NV];
-  const int nslice = (C + CS - 1) / CS;
-  const int b = blockIdx.z / nslice, slice = blockIdx.z - b * nslice;
-  const int ch_base = slice * CS;
-  const int r0 = blockIdx.y * kTR, c0 = blockIdx.x * kTC;
-  const TIN* img = x + (size_t)b * Hg * Wg * C;
-  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-  for (int i = threadIdx.x; i < TH * TW * NV; i += blockDim.x) {
-    const int v = i % NV, pix = i / NV;
-    const int rr = r0 - 1 + pix / TW, cc = c0 - 1 + pix % TW, ch = ch_base + v * VEC;
-    uint4 u = zero;
-    if (rr >= 0 && rr < Hg && cc >= 0 && cc < Wg && ch < C)
-      u = __ldg(reinterpret_cast<const uint4*>(img + ((size_t)rr * Wg + cc) * C + ch));
-    tile[i] = u;
-  }
-  __syncthreads();
-  const int v = threadIdx.x % NV;
-  const int ch0 = ch_base + v * VEC;
-  if (ch0 >= C) return;
-  float wr[9][VEC], bv[VEC];
+  constexpr int R = kConvRows;
+  using PT = typename Pair<TIN>::type;
+  const int np = C / 2;
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  const int c = idx / np, ch = 2 * (idx - c * np);
+  if (c >= Wg) return;
+  const int b = blockIdx.z, r0 = blockIdx.y * R;
+  const size_t pix = (size_t)C / 2;  // one pixel in units of PT
+  // input rows r0-1 .. r0+R, columns c-1 .. c+1 (zero outside the grid)
+  PT win[R + 2][3];
+  {
+    const bool cl = c > 0, cr = c + 1 < Wg;
+    const PT* row = reinterpret_cast<const PT*>(x + (((size_t)b * Hg + r0 - 1) * Wg + c) * C + ch);
 #pragma unroll
-  for (int i = 0; i < VEC; ++i) {
-    bv[i] = bias ? __ldg(bias + ch0 + i) : 0.f;
-#pragma unroll
-    for (int tap = 0; tap < 9; ++tap) wr[tap][i] = __ldg(w + (ch0 + i) * 9 + tap);
-  }
-  for (int pix = threadIdx.x / NV; pix < kTR * kTC; pix += blockDim.x / NV) {
-    const int tr = pix / kTC, tc = pix % kTC;
-    const int r = r0 + tr, c = c0 + tc;
-    if (r >= Hg || c >= Wg) continue;
-    float acc[VEC];
-#pragma unroll
-    for (int i = 0; i < VEC; ++i) acc[i] = bv[i];
-#pragma unroll
-    for (int di = 0; di < 3; ++di) {
-#pragma unroll
-      for (int dj = 0; dj < 3; ++dj) {
-        float xv[VEC];
-        unpack_vec<TIN>(tile[((tr + di) * TW + (tc + dj)) * NV + v], xv);
-#pragma unroll
-        for (int i = 0; i < VEC; ++i) acc[i] = fmaf(wr[di * 3 + dj][i], xv[i], acc[i]);
-      }
+    for (int i = 0; i < R + 2; ++i, row += (size_t)Wg * pix) {
+      const int rr = r0 - 1 + i;
+      const bool rok = rr >= 0 && rr < Hg;
+      win[i][0] = (rok && cl) ? __ldg(row - pix) : PT{};
+      win[i][1] = rok ? __ldg(row) : PT{};
+      win[i][2] = (rok && cr) ? __ldg(row + pix) : PT{};
     }
-    store_row<VEC>(y + ((size_t)b * Hg * Wg + grid_to_scan(r, c, Hg, Wg, mode)) * C + ch0, acc);
+  }
+  // the 9 taps of the two channels: 18 consecutive floats, 8-byte aligned
+  float wr[9][2];
+  {
+    const float2* wp = reinterpret_cast<const float2*>(w + (size_t)ch * 9);
+    float f[18];
+#pragma unroll
+    for (int i = 0; i < 9; ++i) {
+      const float2 v = __ldg(wp + i);
+      f[2 * i] = v.x;
+      f[2 * i + 1] = v.y;
+    }
+#pragma unroll
+    for (int tap = 0; tap < 9; ++tap) {
+      wr[tap][0] = f[tap];
+      wr[tap][1] = f[9 + tap];
+    }
+  }
+  const float2 bv = bias ? __ldg(reinterpret_cast<const float2*>(bias + ch)) : make_float2(0.f, 0.f);
+  // scan position of (r0, c) and its step per grid row
+  const int L = Hg * Wg;
+  const int t0 = grid_to_scan(r0 < Hg ? r0 : 0, c, Hg, Wg, mode);
+  const int step = (mode & 2) ? 1 : Wg;
+  const int sstep = (mode & 1) ? -step : step;
+  TOUT* out = y + ((size_t)b * L + t0) * C + ch;
+  const ptrdiff_t ostep = (ptrdiff_t)sstep * C;
+  float u0[3][2], u1[3][2], u2[3][2];
+#pragma unroll
+  for (int j = 0; j < 3; ++j) {
+    Pair<TIN>::unpack(win[0][j], u0[j]);
+    Pair<TIN>::unpack(win[1][j], u1[j]);
+  }
+#pragma unroll
+  for (int i = 0; i < R; ++i, out += ostep) {
+#pragma unroll
+    for (int j = 0; j < 3; ++j) Pair<TIN>::unpack(win[i + 2][j], u2[j]);
+    if (r0 + i < Hg) {
+      float a0 = bv.x, a1 = bv.y;
+#pragma unroll
+      for (int j = 0; j < 3; ++j) {
+        a0 = fmaf(wr[j][0], u0[j][0], a0);
+        a1 = fmaf(wr[j][1], u0[j][1], a1);
+        a0 = fmaf(wr[3 + j][0], u1[j][0], a0);
+        a1 = fmaf(wr[3 + j][1], u1[j][1], a1);
+        a0 = fmaf(wr[6 + j][0], u2[j][0], a0);
+        a1 = fmaf(wr[6 + j][1], u2[j][1], a1);
+      }
+      Pair<TOUT>::store(out, a0, a1);
+    }
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      u0[j][0] = u1[j][0]; u0[j][1] = u1[j][1];
+      u1[j][0] = u2[j][0]; u1[j][1] = u2[j][1];
+    }
   }
 }
 
@@ -130,8 +165,7 @@ __global__ void __launch_bounds__(256) srem_dwconv_scalar_kernel(const TIN* __re
 template <typename TIN, typename TOUT>
 static cudaError_t launch_typed(const void* x, const float* w, const float* bias, void* y, int B, int Hg, int Wg,
                                 int C, int mode, cudaStream_t s) {
-  constexpr int VEC = 16 / sizeof(TIN);  // one 16-byte vector of input channels
-  if (C % VEC != 0) {
+  if (C % 2 != 0) {  // channels that do not pair up
     const long long total = (long long)B * Hg * Wg * C;
     const long long blocks = (total + 255) / 256;
     const int grid = (int)(blocks < 148LL * 32 ? blocks : 148LL * 32);
@@ -139,11 +173,13 @@ static cudaError_t launch_typed(const void* x, const float* w, const float* bias
                                                                reinterpret_cast<TOUT*>(y), B, Hg, Wg, C, mode);
     return cudaGetLastError();
   }
-  const long long nz = (long long)B * ((C + kSliceBytes / (int)sizeof(TIN) - 1) / (kSliceBytes / (int)sizeof(TIN)));
-  if (nz > 65535 || (Hg + kTR - 1) / kTR > 65535) return cudaErrorInvalidValue;
-  const dim3 grid((Wg + kTC - 1) / kTC, (Hg + kTR - 1) / kTR, (unsigned)nz);
+  constexpr int R = kConvRows;
+  const long long gx = ((long long)Wg * (C / 2) + 255) / 256;
+  const long long gy = (Hg + R - 1) / R;
+  if (gx > 2147483647LL || gy > 65535 || B > 65535) return cudaErrorInvalidValue;
+  const dim3 grid((unsigned)gx, (unsigned)gy, (unsigned)B);
   srem_dwconv_kernel<TIN, TOUT><<<grid, 256, 0, s>>>(reinterpret_cast<const TIN*>(x), w, bias,
-                                                      reinterpret_cast<TOUT*>(y), B, Hg, Wg, C, mode);
+                                                           reinterpret_cast<TOUT*>(y), B, Hg, Wg, C, mode);
   return cudaGetLastError();
 }
 
