@@ -73,6 +73,7 @@ struct BwdCfg {
 };
 
 struct GradSmem {
+  long long rows[2][128];  // grid tokens of the current and the next unit (by unit parity)
   float segtot[8][64];  // reverse-cumsum totals of the token segments
   float bnd[2][64];     // rowsum(S_{n+1} o G_n), double-buffered by unit parity
   uint64_t bar[6];      // completion of the six product groups of a unit
@@ -182,6 +183,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
     fence_mbar_init();
   }
   if (tid < 128) sh.bnd[tid >> 6][tid & 63] = 0.f;
+  if ((int)blockIdx.x < a.B * a.H * a.nchunks) fill_rows(a, blockIdx.x, C, sh.rows[0]);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -216,9 +218,10 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
     const Unit U(a, u);
     const int hz = U.bz - U.b * a.gate_heads;
     float* bnd = sh.bnd[it & 1];
+    const long long* rows = sh.rows[it & 1];  // this unit's grid tokens
     // ---- operands: qbar, kbar rows; S' and Gt rows; v and dO rows; the boundary term of d log alpha
-    load_v_rows<C, DK, DV, TIN>(a, U, a.v, sbase + BC::OFF_V);
-    load_v_rows<C, DK, DV, TIN>(a, U, a.dO, sbase + BC::OFF_DO);
+    load_v_rows_t<C, DK, DV, TIN>(a, U.h, rows, a.v, sbase + BC::OFF_V);
+    load_v_rows_t<C, DK, DV, TIN>(a, U.h, rows, a.dO, sbase + BC::OFF_DO);
     {
       Piece<TIN, PSK> pq[K::NPK], pk[K::NPK];
       Piece<float, PSK> pe[K::NPK];
@@ -227,13 +230,12 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
         const int i = tid + 256 * j;
         int tt, g;
         piece_of<K::NGK>(i, tt, g);
-        const int p = U.n * C + tt;
-        const bool valid = i < C * K::NGK && p < a.L;
-        const long long grow = valid ? (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode) : 0;
-        const size_t off = ((size_t)grow * a.H + U.h) * DK + g * PSK;
+        const long long gr = i < C * K::NGK ? rows[tt] : -1;
+        const bool valid = gr >= 0;
+        const size_t off = tok_row(gr, a, U.h) * DK + g * PSK;
         pq[j].load(reinterpret_cast<const TIN*>(a.q) + off, valid);
         pk[j].load(reinterpret_cast<const TIN*>(a.k) + off, valid);
-        pe[j].load(a.gEQ + ((size_t)U.bz * a.L + (valid ? p : 0)) * DK + g * PSK, valid);
+        pe[j].load(a.gEQ + ((size_t)U.bz * a.L + (valid ? U.n * C + tt : 0)) * DK + g * PSK, valid);
       }
 #pragma unroll
       for (int j = 0; j < K::NPK; ++j) {
@@ -399,13 +401,12 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
       const int i = tid + 256 * j;
       int tt, g;
       piece_of<K::NGV>(i, tt, g);
-      const int p = U.n * C + tt;
-      if (i < C * K::NGV && p < a.L) {
-        const long long grow = (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode);
+      const long long gr = i < C * K::NGV ? rows[tt] : -1;
+      if (gr >= 0) {
         const float4 v0 = *reinterpret_cast<const float4*>(SV + tt * BC::VP + 8 * g);
         const float4 v1 = *reinterpret_cast<const float4*>(SV + tt * BC::VP + 8 * g + 4);
         const float vv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        st_global8(reinterpret_cast<TOUT*>(a.dv) + ((size_t)grow * a.H + U.h) * DV + 8 * g, vv);
+        st_global8(reinterpret_cast<TOUT*>(a.dv) + tok_row(gr, a, U.h) * DV + 8 * g, vv);
       }
     }
     {
@@ -416,13 +417,12 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
         const int i = tid + 256 * j;
         int tt, g;
         piece_of<K::NGK>(i, tt, g);
-        const int p = U.n * C + tt;
-        const bool valid = i < C * K::NGK && p < a.L;
-        const long long grow = valid ? (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode) : 0;
-        const size_t off = ((size_t)grow * a.H + U.h) * DK + g * PSK;
+        const long long gr = i < C * K::NGK ? rows[tt] : -1;
+        const bool valid = gr >= 0;
+        const size_t off = tok_row(gr, a, U.h) * DK + g * PSK;
         pq[j].load(reinterpret_cast<const TIN*>(a.q) + off, valid);
         pk[j].load(reinterpret_cast<const TIN*>(a.k) + off, valid);
-        pe[j].load(a.gEQ + ((size_t)U.bz * a.L + (valid ? p : 0)) * DK + g * PSK, valid);
+        pe[j].load(a.gEQ + ((size_t)U.bz * a.L + (valid ? U.n * C + tt : 0)) * DK + g * PSK, valid);
       }
 #pragma unroll
       for (int j = 0; j < K::NPK; ++j) {
@@ -448,8 +448,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
           for (int e = 0; e < PSK; e += 4)
             *reinterpret_cast<float4*>(SX + tt * BC::KP + g * PSK + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
           if (valid) {
-            const long long grow = (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode);
-            const size_t off = ((size_t)grow * a.H + U.h) * DK + g * PSK;
+            const size_t off = tok_row(rows[tt], a, U.h) * DK + g * PSK;
             st_global_piece<PSK>(reinterpret_cast<TOUT*>(a.dq) + off, dq);
             st_global_piece<PSK>(reinterpret_cast<TOUT*>(a.dk) + off, dk);
           }
@@ -474,16 +473,16 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
       float post = bnd[sc];
       for (int s2 = sg + 1; s2 < BC::NSG; ++s2) post += sh.segtot[s2][sc];
       for (int t = t0; t < t1; ++t) {
-        const int p = U.n * C + t;
-        if (p < a.L) {
-          const long long grow = (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode);
-          float* dst = a.dla + ((size_t)grow * a.gate_heads + hz) * DK + sc;
+        const long long gr = rows[t];
+        if (gr >= 0) {
+          float* dst = a.dla + ((size_t)gr * a.gate_heads + hz) * DK + sc;
           const float val = SX[t * BC::KP + sc] + post;
           if (a.gate_heads == 1) atomicAdd(dst, val);
           else *dst = val;
         }
       }
     }
+    if (u + (int)gridDim.x < nunits) fill_rows(a, u + gridDim.x, C, sh.rows[(it + 1) & 1]);
     __syncthreads();  // staging, segment totals and the operands are reused by the next unit
   }
   if (timed_out) set_status(a.status, DIG_ERR_DEVICE_TIMEOUT);

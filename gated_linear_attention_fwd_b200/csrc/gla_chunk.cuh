@@ -79,6 +79,7 @@ struct StateCfg {
 };
 
 struct StateSmem {
+  long long rows[2][128];  // grid tokens of the units whose loads are in flight (by unit parity)
   float segtot[8][64];  // cumsum totals of the token segments
   float gam[64];        // chunk decay Gamma (log2)
   uint64_t bar;
@@ -97,14 +98,32 @@ struct Unit {
   }
 };
 
-// Rows of a [B, L, H, DV] tensor (v or dO) for the unit's chunk into a K-major
-// operand buffer at `vr` (token rows of DVP channels).  bf16 values are copied
-// unchanged (one exact term) by asynchronous 16-byte copies, zero-filled past
-// the sequence end (complete after cp_async_wait_all); fp32 values are split
-// into three bf16 terms.  Channels DV..DVP are zeroed (they are a contracted
-// dimension in some products).
+// Grid token of token t of a unit, b * L + pi(n C + t), or -1 past the chunk or
+// the sequence end; its row in the [B, L, H, *] tensors is that times H plus h.
+// Kernels fill a unit's 128 entries into shared memory once (one thread per
+// token) instead of mapping the scan position of every row piece.
+__device__ __forceinline__ long long unit_grow(const GlaArgs& a, const Unit& U, int C, int t) {
+  const int p = U.n * C + t;
+  if (t >= C || p >= a.L) return -1;
+  return (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode);
+}
+__device__ __forceinline__ void fill_rows(const GlaArgs& a, int u, int C, long long* grows) {
+  if ((int)threadIdx.x < 128) grows[threadIdx.x] = unit_grow(a, Unit(a, u), C, threadIdx.x);
+}
+// Row of the unit's token in a [B, L, H, *] tensor (0 for an invalid token, which is never dereferenced).
+__device__ __forceinline__ size_t tok_row(long long grow, const GlaArgs& a, int h) {
+  return grow >= 0 ? (size_t)grow * a.H + h : 0;
+}
+
+// Rows of a [B, L, H, DV] tensor (v or dO) for a unit's chunk, its grid tokens
+// from a table (see unit_grow), into a K-major operand buffer at `vr` (token
+// rows of DVP channels).  bf16 values are copied unchanged (one exact term) by
+// asynchronous 16-byte copies, zero-filled past the sequence end (complete after
+// cp_async_wait_all); fp32 values are split into three bf16 terms.  Channels
+// DV..DVP are zeroed (they are a contracted dimension in some products).
 template <int C, int DK, int DV, typename TIN>
-__device__ __forceinline__ void load_v_rows(const GlaArgs& a, const Unit& U, const void* src, uint32_t vr) {
+__device__ __forceinline__ void load_v_rows_t(const GlaArgs& a, int h, const long long* rows, const void* src,
+                                              uint32_t vr) {
   using Cfg = ChunkCfg<C, DK, DV, TIN>;
   const int tid = threadIdx.x;
   if constexpr (std::is_same<TIN, __nv_bfloat16>::value) {
@@ -114,11 +133,9 @@ __device__ __forceinline__ void load_v_rows(const GlaArgs& a, const Unit& U, con
       int t, g;
       piece_of<Cfg::NGV>(i, t, g);
       if (i < C * Cfg::NGV) {
-        const int p = U.n * C + t;
-        const bool valid = p < a.L;
-        const long long grow = valid ? (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode) : 0;
+        const long long gr = rows[t];
         cp_async16_zfill(row_addr(vr, t, Cfg::SBO_V) + 128u * g,
-                         reinterpret_cast<const TIN*>(src) + ((size_t)grow * a.H + U.h) * DV + 8 * g, valid);
+                         reinterpret_cast<const TIN*>(src) + tok_row(gr, a, h) * DV + 8 * g, gr >= 0);
       }
     }
   } else {
@@ -128,10 +145,8 @@ __device__ __forceinline__ void load_v_rows(const GlaArgs& a, const Unit& U, con
       const int i = tid + 256 * j;
       int t, g;
       piece_of<Cfg::NGV>(i, t, g);
-      const int p = U.n * C + t;
-      const bool valid = i < C * Cfg::NGV && p < a.L;
-      const long long grow = valid ? (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode) : 0;
-      pv[j].load(reinterpret_cast<const TIN*>(src) + ((size_t)grow * a.H + U.h) * DV + 8 * g, valid);
+      const long long gr = i < C * Cfg::NGV ? rows[t] : -1;
+      pv[j].load(reinterpret_cast<const TIN*>(src) + tok_row(gr, a, h) * DV + 8 * g, gr >= 0);
     }
 #pragma unroll
     for (int j = 0; j < Cfg::NPV; ++j) {
@@ -197,6 +212,7 @@ __global__ void __launch_bounds__(256, BWD ? 2 : 3) gla_chunk_state_kernel(const
     mbar_init(&sh.bar, 1);
     fence_mbar_init();
   }
+  if ((int)blockIdx.x < a.B * a.H * a.nchunks) fill_rows(a, blockIdx.x, C, sh.rows[0]);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -217,7 +233,7 @@ __global__ void __launch_bounds__(256, BWD ? 2 : 3) gla_chunk_state_kernel(const
   // products have completed.
   Piece<float, 4> pz[Cfg::NPZ];
   Piece<TIN, PSK> pk[Cfg::NPK], pq[BWD ? Cfg::NPK : 1];
-  auto issue_rows = [&](int u) {
+  auto issue_rows = [&](int u, const long long* rows) {
     const Unit U(a, u);
     const int hz = U.bz - U.b * a.gate_heads;
 #pragma unroll
@@ -225,39 +241,38 @@ __global__ void __launch_bounds__(256, BWD ? 2 : 3) gla_chunk_state_kernel(const
       const int i = tid + 256 * j;
       int t, g;
       piece_of<Cfg::NGZ>(i, t, g);
-      const int p = U.n * C + t;
-      const bool valid = i < C * Cfg::NGZ && p < a.L;
-      const long long grow = valid ? (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode) : 0;
-      pz[j].load(a.z + ((size_t)grow * a.gate_heads + hz) * DK + 4 * g, valid);
+      const long long gr = i < C * Cfg::NGZ ? rows[t] : -1;
+      pz[j].load(a.z + ((size_t)(gr >= 0 ? gr : 0) * a.gate_heads + hz) * DK + 4 * g, gr >= 0);
     }
 #pragma unroll
     for (int j = 0; j < Cfg::NPK; ++j) {
       const int i = tid + 256 * j;
       int t, g;
       piece_of<Cfg::NGK>(i, t, g);
-      const int p = U.n * C + t;
-      const bool valid = i < C * Cfg::NGK && p < a.L;
-      const long long grow = valid ? (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode) : 0;
-      const size_t off = ((size_t)grow * a.H + U.h) * DK + g * PSK;
-      pk[j].load(reinterpret_cast<const TIN*>(a.k) + off, valid);
-      if constexpr (BWD) pq[j].load(reinterpret_cast<const TIN*>(a.q) + off, valid);
+      const long long gr = i < C * Cfg::NGK ? rows[t] : -1;
+      const size_t off = tok_row(gr, a, U.h) * DK + g * PSK;
+      pk[j].load(reinterpret_cast<const TIN*>(a.k) + off, gr >= 0);
+      if constexpr (BWD) pq[j].load(reinterpret_cast<const TIN*>(a.q) + off, gr >= 0);
     }
   };
-  auto issue_vd = [&](int u) {
-    const Unit U(a, u);
-    load_v_rows<C, DK, DV, TIN>(a, U, a.v, sbase + SC::OFF_VR);
-    if constexpr (BWD) load_v_rows<C, DK, DV, TIN>(a, U, a.dO, sbase + SC::OFF_DO);
+  auto issue_vd = [&](int u, const long long* rows) {
+    const int h = Unit(a, u).h;
+    load_v_rows_t<C, DK, DV, TIN>(a, h, rows, a.v, sbase + SC::OFF_VR);
+    if constexpr (BWD) load_v_rows_t<C, DK, DV, TIN>(a, h, rows, a.dO, sbase + SC::OFF_DO);
   };
   if ((int)blockIdx.x < nunits) {
-    issue_rows(blockIdx.x);
-    issue_vd(blockIdx.x);
+    issue_rows(blockIdx.x, sh.rows[0]);
+    issue_vd(blockIdx.x, sh.rows[0]);
   }
 
-  for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+  int it = 0;
+  for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
     const Unit U(a, u);
     const bool writer = a.gate_heads != 1 || U.h == 0;  // one unit per gate head stores the factors
     const int un = u + gridDim.x;
     const bool has_next = un < nunits;
+    long long* rows_next = sh.rows[(it + 1) & 1];
+    if (has_next) fill_rows(a, un, C, rows_next);  // read after this unit's next barrier
     // ---- inclusive cumsum over the chunk's tokens, per key channel (shared memory)
 #pragma unroll
     for (int j = 0; j < Cfg::NPZ; ++j) {
@@ -354,7 +369,7 @@ __global__ void __launch_bounds__(256, BWD ? 2 : 3) gla_chunk_state_kernel(const
           st_piece<NTG, 4>(sbase + SC::OFF_QB, i / Cfg::NPAD, Cfg::SBO_K, DK + 4 * (i % Cfg::NPAD), Cfg::AQ_SZ, zz);
       }
     }
-    if (has_next) issue_rows(un);  // this unit's row pieces are consumed
+    if (has_next) issue_rows(un, rows_next);  // this unit's row pieces are consumed
     cp_async_wait_all();
     // ---- dS = v^T khat, dH = dO^T (q 2^b)  (M = value channels, N = key channels, K = tokens)
     fence_async_smem();
@@ -372,7 +387,7 @@ __global__ void __launch_bounds__(256, BWD ? 2 : 3) gla_chunk_state_kernel(const
     if (!mbar_wait(&sh.bar, ph, kSpinLimitNs)) timed_out = true;
     ph ^= 1u;
     tc_fence_after();
-    if (has_next) issue_vd(un);  // v (and dO) of this unit are consumed
+    if (has_next) issue_vd(un, rows_next);  // v (and dO) of this unit are consumed
     if (tid < 128) stage_rows_dk<C, DK, DV, TIN, 0>(tmem, 0, SD, SC::SDP);
     else stage_rows_dk<C, DK, DV, TIN, 1>(tmem, 0, SD, SC::SDP);
     if constexpr (BWD) {

@@ -77,6 +77,7 @@ struct OutCfg {
 };
 
 struct OutSmem {
+  long long rows[2][128];  // grid tokens of the current and the next unit (by unit parity)
   float red[256];  // epilogue row sums of squares
   uint64_t bar_a;  // P, qbar S'
   uint64_t bar_b;  // P V
@@ -222,6 +223,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
     mbar_init(&sh.bar_b, 1);
     fence_mbar_init();
   }
+  if ((int)blockIdx.x < a.B * a.H * a.nchunks) fill_rows(a, blockIdx.x, C, sh.rows[0]);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -246,20 +248,19 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
   Piece<float, PSK> pe[Cfg::NPK];
   Piece<float, 4> ps[Cfg::NPS], pc[Cfg::NPS];
   Piece<TIN, 8> pr[Cfg::NPV];
-  auto issue_rows = [&](int u) {
+  auto issue_rows = [&](int u, const long long* rows) {
     const Unit U(a, u);
 #pragma unroll
     for (int j = 0; j < Cfg::NPK; ++j) {
       const int i = tid + 256 * j;
       int tt, g;
       piece_of<Cfg::NGK>(i, tt, g);
-      const int p = U.n * C + tt;
-      const bool valid = i < C * Cfg::NGK && p < a.L;
-      const long long grow = valid ? (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode) : 0;
-      const size_t off = ((size_t)grow * a.H + U.h) * DK + g * PSK;
+      const long long gr = i < C * Cfg::NGK ? rows[tt] : -1;
+      const bool valid = gr >= 0;
+      const size_t off = tok_row(gr, a, U.h) * DK + g * PSK;
       pq[j].load(reinterpret_cast<const TIN*>(a.q) + off, valid);
       pk[j].load(reinterpret_cast<const TIN*>(a.k) + off, valid);
-      pe[j].load(a.gEQ + ((size_t)U.bz * a.L + (valid ? p : 0)) * DK + g * PSK, valid);
+      pe[j].load(a.gEQ + ((size_t)U.bz * a.L + (valid ? U.n * C + tt : 0)) * DK + g * PSK, valid);
     }
 #pragma unroll
     for (int j = 0; j < Cfg::NPS; ++j) {
@@ -271,37 +272,43 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
       pc[j].load(a.gCH + ((size_t)U.bz * a.nchunks + U.n) * 4 * DK + 4 * g, in);
     }
   };
-  auto issue_r = [&](int u) {
+  auto issue_r = [&](int h, const long long* rows) {
     if (!with_y) return;
-    const Unit U(a, u);
 #pragma unroll
     for (int j = 0; j < Cfg::NPV; ++j) {
       const int i = tid + 256 * j;
       int tt, g;
       piece_of<Cfg::NGV>(i, tt, g);
-      const int p = U.n * C + tt;
-      const bool valid = i < C * Cfg::NGV && p < a.L;
-      const long long grow = valid ? (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode) : 0;
-      pr[j].load(reinterpret_cast<const TIN*>(a.r) + ((size_t)grow * a.H + U.h) * DV + 8 * g, valid);
+      const long long gr = i < C * Cfg::NGV ? rows[tt] : -1;
+      pr[j].load(reinterpret_cast<const TIN*>(a.r) + tok_row(gr, a, h) * DV + 8 * g, gr >= 0);
     }
   };
   // Loading one unit ahead holds two units' pieces in registers; with 8-byte
   // pieces (d_k not a multiple of 8) that spills, so those variants load per unit.
   constexpr bool kAhead = PSK == 8;
   if (kAhead && (int)blockIdx.x < nunits) {
-    issue_rows(blockIdx.x);
-    load_v_rows<C, DK, DV, TIN>(a, Unit(a, blockIdx.x), a.v, sbase + OC::OFF_VR);
-    issue_r(blockIdx.x);
+    const int h0 = Unit(a, blockIdx.x).h;
+    issue_rows(blockIdx.x, sh.rows[0]);
+    load_v_rows_t<C, DK, DV, TIN>(a, h0, sh.rows[0], a.v, sbase + OC::OFF_VR);
+    issue_r(h0, sh.rows[0]);
   }
 
-  for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+  int it = 0;
+  for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
     const Unit U(a, u);
     const int un = u + gridDim.x;
     const bool has_next = kAhead && un < nunits;
+    const long long* rows = sh.rows[it & 1];
+    long long* rows_next = sh.rows[(it + 1) & 1];
     if (!kAhead) {
-      issue_rows(u);
-      load_v_rows<C, DK, DV, TIN>(a, U, a.v, sbase + OC::OFF_VR);
+      if (it > 0) {  // the first unit's rows were filled before the first barrier
+        fill_rows(a, u, C, sh.rows[it & 1]);
+        __syncthreads();
+      }
+      issue_rows(u, rows);
+      load_v_rows_t<C, DK, DV, TIN>(a, U.h, rows, a.v, sbase + OC::OFF_VR);
     }
+    if (has_next) fill_rows(a, un, C, rows_next);  // visible after the next barrier
     // ---- operands: qbar = q 2^(b-r), kbar = k 2^(r-b); S'^T rows = (2^r S_n)[:, j]
 #pragma unroll
     for (int j = 0; j < Cfg::NPK; ++j) {
@@ -357,7 +364,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
                                     idesc_bf16(128, OC::NB), false);  // [P | O] = qbar [kbar | S'^T]^T
       mma_commit(&sh.bar_a);
     }
-    if (has_next) issue_rows(un);  // this unit's row pieces are consumed
+    if (has_next) issue_rows(un, rows_next);  // this unit's row pieces are consumed
     if (!mbar_wait(&sh.bar_a, ph, kSpinLimitNs)) timed_out = true;
     tc_fence_after();
     // ---- mask P (s <= t) and store it as bf16 terms in TMEM, one K-step of 16 at a time
@@ -403,8 +410,9 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
     if (!mbar_wait(&sh.bar_b, ph, kSpinLimitNs)) timed_out = true;
     ph ^= 1u;
     tc_fence_after();
-    if (has_next) load_v_rows<C, DK, DV, TIN>(a, Unit(a, un), a.v, sbase + OC::OFF_VR);  // v of this unit is consumed
-    if (!kAhead) issue_r(u);
+    const int hn = has_next ? Unit(a, un).h : 0;
+    if (has_next) load_v_rows_t<C, DK, DV, TIN>(a, hn, rows_next, a.v, sbase + OC::OFF_VR);  // v of this unit is consumed
+    if (!kAhead) issue_r(U.h, rows);
     if (tid < 128) stage_o<C, DK, DV, TIN, 0>(tmem, stage, sh.red);
     else stage_o<C, DK, DV, TIN, 1>(tmem, stage, sh.red);
     tc_fence_before();
@@ -415,10 +423,9 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
       const int i = tid + 256 * j;
       int tt, g;
       piece_of<Cfg::NGV>(i, tt, g);
-      const int p = U.n * C + tt;
-      if (i < C * Cfg::NGV && p < a.L) {
-        const long long grow = (long long)U.b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode);
-        const size_t off = ((size_t)grow * a.H + U.h) * DV + 8 * g;
+      const long long gr = i < C * Cfg::NGV ? rows[tt] : -1;
+      if (gr >= 0) {
+        const size_t off = tok_row(gr, a, U.h) * DV + 8 * g;
         float ov[8];
         const float4 o0 = *reinterpret_cast<const float4*>(stage + tt * OC::OP + 8 * g);
         const float4 o1 = *reinterpret_cast<const float4*>(stage + tt * OC::OP + 8 * g + 4);
@@ -447,7 +454,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
         }
       }
     }
-    if (has_next) issue_r(un);
+    if (has_next) issue_r(hn, rows_next);
     __syncthreads();  // staging and row sums are rewritten by the next unit
   }
   if (timed_out) set_status(a.status, DIG_ERR_DEVICE_TIMEOUT);
