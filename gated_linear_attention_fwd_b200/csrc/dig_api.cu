@@ -128,14 +128,15 @@ dig_status dig_gla_fwd(const void* q, const void* k, const void* v, const float*
   return DIG_OK;
 }
 
-dig_status dig_gla_bwd(const void* q, const void* k, const void* v, const float* z, int gate_heads, float inv_tau,
-                       const void* dO, void* dq, void* dk, void* dv, float* dlog_alpha, int B, int H, int L, int d_k,
-                       int d_v, int grid_h, int grid_w, int scan_mode, int dtype, int out_dtype, void* workspace,
-                       size_t workspace_bytes, void* stream) {
+static dig_status gla_bwd_impl(const void* q, const void* k, const void* v, const float* z, int gate_heads,
+                               float inv_tau, const void* dO, void* dq, void* dk, void* dv, float* dlog_alpha, int B,
+                               int H, int L, int d_k, int d_v, int grid_h, int grid_w, int scan_mode, int dtype,
+                               int out_dtype, const void* fwd_workspace, size_t fwd_workspace_bytes, void* workspace,
+                               size_t workspace_bytes, void* stream) {
   dig_status st = check_common(B, H, L, d_k, d_v, grid_h, grid_w, scan_mode, dtype, out_dtype, gate_heads);
   if (st != DIG_OK) return st;
   if (!workspace) return fail(DIG_ERR_INVALID_ARGUMENT, "workspace is NULL");
-  if (!aligned16(workspace)) return fail(DIG_ERR_MISALIGNED, "workspace not 16-byte aligned");
+  if (!aligned16(workspace) || !aligned16(fwd_workspace)) return fail(DIG_ERR_MISALIGNED, "workspace not 16-byte aligned");
   if (B == 0 || L == 0) return DIG_OK;
   if (!q || !k || !v || !z || !dO || !dq || !dk || !dv || !dlog_alpha)
     return fail(DIG_ERR_INVALID_ARGUMENT, "all tensor pointers of the backward must be non-NULL");
@@ -147,7 +148,14 @@ dig_status dig_gla_bwd(const void* q, const void* k, const void* v, const float*
   const WsLayout lay = ws_layout(B, H, gate_heads, L, nchunks, d_k, d_v, true);
   if (workspace_bytes < lay.total)
     return fail(DIG_ERR_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, needs %zu", workspace_bytes, lay.total);
+  // The forward's records are usable when both passes cut the sequence into the same chunks.
+  const bool saved = fwd_workspace != nullptr && chunk_len(dtype, false, d_k, d_v) == C;
+  const WsLayout flay = ws_layout(B, H, gate_heads, L, nchunks, d_k, d_v, false);
+  if (saved && fwd_workspace_bytes < flay.total)
+    return fail(DIG_ERR_WORKSPACE_TOO_SMALL, "forward workspace has %zu bytes, needs %zu", fwd_workspace_bytes,
+                flay.total);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* fws = static_cast<uint8_t*>(const_cast<void*>(fwd_workspace));  // only read
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (gate_heads == 1) {
     // heads add their contributions into dlog_alpha
@@ -160,14 +168,33 @@ dig_status dig_gla_bwd(const void* q, const void* k, const void* v, const float*
   a.inv_tau = inv_tau;
   a.nchunks = nchunks;
   a.status = reinterpret_cast<uint32_t*>(ws);
-  a.gEQ = reinterpret_cast<float*>(ws + lay.gEQ);
-  a.gCH = reinterpret_cast<float*>(ws + lay.gCH);
-  a.dsn = reinterpret_cast<float*>(ws + lay.dsn);
+  a.gEQ = reinterpret_cast<float*>((saved ? fws + flay.gEQ : ws + lay.gEQ));
+  a.gCH = reinterpret_cast<float*>((saved ? fws + flay.gCH : ws + lay.gCH));
+  a.dsn = reinterpret_cast<float*>((saved ? fws + flay.dsn : ws + lay.dsn));
   a.dhn = reinterpret_cast<float*>(ws + lay.dhn);
   GlaVariant var{C, dtype == DIG_BF16 ? 2 : 3, d_k, d_v, dtype, out_dtype};
-  const cudaError_t e = launch_gla_bwd(var, a, s);
+  const cudaError_t e = launch_gla_bwd(var, a, saved, s);
   if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "gla_bwd launch: %s", cudaGetErrorString(e));
   return DIG_OK;
+}
+
+dig_status dig_gla_bwd(const void* q, const void* k, const void* v, const float* z, int gate_heads, float inv_tau,
+                       const void* dO, void* dq, void* dk, void* dv, float* dlog_alpha, int B, int H, int L, int d_k,
+                       int d_v, int grid_h, int grid_w, int scan_mode, int dtype, int out_dtype, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  return gla_bwd_impl(q, k, v, z, gate_heads, inv_tau, dO, dq, dk, dv, dlog_alpha, B, H, L, d_k, d_v, grid_h, grid_w,
+                      scan_mode, dtype, out_dtype, nullptr, 0, workspace, workspace_bytes, stream);
+}
+
+dig_status dig_gla_bwd_saved(const void* q, const void* k, const void* v, const float* z, int gate_heads,
+                             float inv_tau, const void* dO, void* dq, void* dk, void* dv, float* dlog_alpha, int B,
+                             int H, int L, int d_k, int d_v, int grid_h, int grid_w, int scan_mode, int dtype,
+                             int out_dtype, const void* fwd_workspace, size_t fwd_workspace_bytes, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  if (!fwd_workspace) return fail(DIG_ERR_INVALID_ARGUMENT, "fwd_workspace is NULL");
+  return gla_bwd_impl(q, k, v, z, gate_heads, inv_tau, dO, dq, dk, dv, dlog_alpha, B, H, L, d_k, d_v, grid_h, grid_w,
+                      scan_mode, dtype, out_dtype, fwd_workspace, fwd_workspace_bytes, workspace, workspace_bytes,
+                      stream);
 }
 
 dig_status dig_srem_reorient_dwconv(const void* x, const float* w, const float* bias, void* y, int B, int grid_h,

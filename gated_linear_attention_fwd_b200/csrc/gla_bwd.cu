@@ -492,18 +492,157 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
   if (warp == 0) tmem_dealloc(tmem, BC::TM_COLS);
 }
 
+// ============================================================== dH from saved records
+// Per unit, when the forward's gate factors and states are reused: the chunk's
+// state-gradient contribution dH = (q 2^b)^T dO with q 2^b = q * EQ * 2^r (no
+// gate cumsum, no dS), rows stored value-major to `dhn`.
+template <int C, int DK, int DV, typename TIN>
+struct DhCfg {
+  using K = ChunkCfg<C, DK, DV, TIN>;
+  static constexpr int OFF_QB = 0;
+  static constexpr int OFF_DO = K::NTG * K::AQ_SZ;
+  static constexpr int SDP = DK + 4;
+  static constexpr int OFF_SD = cround(OFF_DO + K::NTV * K::VR_SZ, 16);
+  static constexpr int SMEM = cmax(OFF_SD + DV * SDP * 4, OFF_DO + K::VR_READ);
+  static constexpr int TM_COLS = pow2ceil(K::DKP);
+  static constexpr int PER_SM = SMEM <= 72 * 1024 ? 3 : SMEM <= 110 * 1024 ? 2 : 1;
+  static_assert(SMEM <= 225 * 1024, "shared-memory budget");
+};
+
+template <int C, int DK, int DV, typename TIN>
+__global__ void __launch_bounds__(256, 3) gla_chunk_dh_kernel(const GlaArgs a) {
+  using K = ChunkCfg<C, DK, DV, TIN>;
+  using DC = DhCfg<C, DK, DV, TIN>;
+  constexpr int NTG = K::NTG, NTV = K::NTV, DKP = K::DKP, PSK = K::PSK;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  __shared__ StateSmem sh;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  if (warp == 0) {
+    tmem_alloc(&sh.tmem, DC::TM_COLS);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(&sh.bar, 1);
+    fence_mbar_init();
+  }
+  const int nunits = a.B * a.H * a.nchunks;
+  if ((int)blockIdx.x < nunits) fill_rows(a, blockIdx.x, C, sh.rows[0]);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem;
+  const uint32_t sbase = smem_u32(smem);
+  float* SD = reinterpret_cast<float*>(smem + DC::OFF_SD);
+  const uint64_t dDOm = sdesc(sbase + DC::OFF_DO, K::SBO_V, 128);
+  const uint64_t dQBm = sdesc(sbase + DC::OFF_QB, K::SBO_K, 128);
+  uint32_t ph = 0;
+  bool timed_out = false;
+  Piece<TIN, PSK> pq[K::NPK];
+  Piece<float, PSK> pe[K::NPK];
+  Piece<float, 4> pc[K::NPK * PSK / 4];  // 2^r of the piece's channels
+  auto issue_rows = [&](int u, const long long* rows) {
+    const Unit U(a, u);
+#pragma unroll
+    for (int j = 0; j < K::NPK; ++j) {
+      const int i = tid + 256 * j;
+      int tt, g;
+      piece_of<K::NGK>(i, tt, g);
+      const long long gr = i < C * K::NGK ? rows[tt] : -1;
+      const bool valid = gr >= 0;
+      pq[j].load(reinterpret_cast<const TIN*>(a.q) + tok_row(gr, a, U.h) * DK + g * PSK, valid);
+      pe[j].load(a.gEQ + ((size_t)U.bz * a.L + (valid ? U.n * C + tt : 0)) * DK + g * PSK, valid);
+      const float* ch = a.gCH + ((size_t)U.bz * a.nchunks + U.n) * 4 * DK + g * PSK;
+#pragma unroll
+      for (int e = 0; e < PSK / 4; ++e) pc[j * (PSK / 4) + e].load(ch + 4 * e, i < C * K::NGK);
+    }
+  };
+  if ((int)blockIdx.x < nunits) {
+    issue_rows(blockIdx.x, sh.rows[0]);
+    load_v_rows_t<C, DK, DV, TIN>(a, Unit(a, blockIdx.x).h, sh.rows[0], a.dO, sbase + DC::OFF_DO);
+  }
+  int it = 0;
+  for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
+    const int un = u + gridDim.x;
+    const bool has_next = un < nunits;
+    long long* rows_next = sh.rows[(it + 1) & 1];
+    if (has_next) fill_rows(a, un, C, rows_next);  // read after the next barrier
+    // ---- q 2^b = q * EQ * 2^r as operand rows
+#pragma unroll
+    for (int j = 0; j < K::NPK; ++j) {
+      const int i = tid + 256 * j;
+      int tt, g;
+      piece_of<K::NGK>(i, tt, g);
+      if (i < C * K::NGK) {
+        float qv[PSK], ev[PSK], cv[PSK];
+        pq[j].unpack(qv);
+        pe[j].unpack(ev);
+#pragma unroll
+        for (int e = 0; e < PSK / 4; ++e) pc[j * (PSK / 4) + e].unpack(cv + 4 * e);
+#pragma unroll
+        for (int e = 0; e < PSK; ++e) qv[e] *= ev[e] * cv[e];
+        st_piece<NTG, PSK>(sbase + DC::OFF_QB, tt, K::SBO_K, g * PSK, K::AQ_SZ, qv);
+      }
+    }
+    if constexpr (K::NPAD > 0) {
+      const float zz[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int i = tid; i < C * K::NPAD; i += 256)
+        st_piece<NTG, 4>(sbase + DC::OFF_QB, i / K::NPAD, K::SBO_K, DK + 4 * (i % K::NPAD), K::AQ_SZ, zz);
+    }
+    cp_async_wait_all();
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (has_next) issue_rows(un, rows_next);  // this unit's row pieces are consumed
+    if (tid == 0) {
+      mma_issue<NTV, NTG, C / 16>(tmem, dDOm, K::VR_SZ, 2 * K::SBO_V, dQBm, K::AQ_SZ, 2 * K::SBO_K,
+                                  idesc_bf16(128, DKP, true, true), false);
+      mma_commit(&sh.bar);
+    }
+    if (!mbar_wait(&sh.bar, ph, kSpinLimitNs)) timed_out = true;
+    ph ^= 1u;
+    tc_fence_after();
+    if (has_next) load_v_rows_t<C, DK, DV, TIN>(a, Unit(a, un).h, rows_next, a.dO, sbase + DC::OFF_DO);
+    if (tid < 128) stage_rows_dk<C, DK, DV, TIN, 0>(tmem, 0, SD, DC::SDP);
+    else stage_rows_dk<C, DK, DV, TIN, 1>(tmem, 0, SD, DC::SDP);
+    tc_fence_before();
+    __syncthreads();
+    float4* dst = reinterpret_cast<float4*>(a.dhn + (size_t)u * DV * DK);
+    for (int i = tid; i < DV * DK / 4; i += 256) {
+      const int row = i / (DK / 4), c4 = i - row * (DK / 4);
+      __stcg(dst + i, *reinterpret_cast<const float4*>(SD + row * DC::SDP + 4 * c4));
+    }
+    __syncthreads();  // staging and operands are reused by the next unit
+  }
+  if (timed_out) set_status(a.status, DIG_ERR_DEVICE_TIMEOUT);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, DC::TM_COLS);
+}
+
 // ------------------------------------------------------------------ launch
 namespace {
 
 template <int DK, int DV, typename TIN, typename TOUT>
-cudaError_t launch_typed(const GlaArgs& a, cudaStream_t s) {
+cudaError_t launch_typed(const GlaArgs& a, bool saved, cudaStream_t s) {
   constexpr int C = bwd_chunk_len(DK, DV, std::is_same<TIN, float>::value);
   using BC = BwdCfg<C, DK, DV, TIN>;
   const long long units = (long long)a.B * a.H * a.nchunks;
   if (units <= 0) return cudaSuccess;
-  cudaError_t e = launch_chunk_state<C, DK, DV, TIN, true>(a, s);
-  if (e != cudaSuccess) return e;
-  if ((e = launch_state_scan(a, a.dsn, false, a.dhn, true, DK, DV, s)) != cudaSuccess) return e;
+  cudaError_t e;
+  if (saved) {  // gate factors and entry states come from the forward: only dH and its reverse scan
+    using DC = DhCfg<C, DK, DV, TIN>;
+    auto kd = gla_chunk_dh_kernel<C, DK, DV, TIN>;
+    if ((e = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, DC::SMEM)) != cudaSuccess)
+      return e;
+    kd<<<persistent_grid(DC::PER_SM, units), 256, DC::SMEM, s>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_state_scan(a, a.dhn, true, nullptr, false, DK, DV, s)) != cudaSuccess) return e;
+  } else {
+    if ((e = launch_chunk_state<C, DK, DV, TIN, true>(a, s)) != cudaSuccess) return e;
+    if ((e = launch_state_scan(a, a.dsn, false, a.dhn, true, DK, DV, s)) != cudaSuccess) return e;
+  }
   auto k = gla_chunk_grad_kernel<C, DK, DV, TIN, TOUT>;
   if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, BC::SMEM)) != cudaSuccess) return e;
   k<<<persistent_grid(BC::PER_SM, units), 256, BC::SMEM, s>>>(a);
@@ -511,24 +650,24 @@ cudaError_t launch_typed(const GlaArgs& a, cudaStream_t s) {
 }
 
 template <int DK, int DV>
-cudaError_t dispatch_types(const GlaVariant& v, const GlaArgs& a, cudaStream_t s) {
+cudaError_t dispatch_types(const GlaVariant& v, const GlaArgs& a, bool saved, cudaStream_t s) {
   using bf = __nv_bfloat16;
   if (v.tin == DIG_BF16) {
-    if (v.tout == DIG_BF16) return launch_typed<DK, DV, bf, bf>(a, s);
-    return launch_typed<DK, DV, bf, float>(a, s);
+    if (v.tout == DIG_BF16) return launch_typed<DK, DV, bf, bf>(a, saved, s);
+    return launch_typed<DK, DV, bf, float>(a, saved, s);
   }
-  if (v.tout == DIG_BF16) return launch_typed<DK, DV, float, bf>(a, s);
-  return launch_typed<DK, DV, float, float>(a, s);
+  if (v.tout == DIG_BF16) return launch_typed<DK, DV, float, bf>(a, saved, s);
+  return launch_typed<DK, DV, float, float>(a, saved, s);
 }
 
 }  // namespace
 
 int gla_bwd_chunk(int dk, int dv, int dtype) { return bwd_chunk_len(dk, dv, dtype != DIG_BF16); }
 
-cudaError_t launch_gla_bwd(const GlaVariant& v, const GlaArgs& a, cudaStream_t s) {
-  if (v.dk == 32 && v.dv == 64) return dispatch_types<32, 64>(v, a, s);
-  if (v.dk == 36 && v.dv == 72) return dispatch_types<36, 72>(v, a, s);
-  if (v.dk == 64 && v.dv == 64) return dispatch_types<64, 64>(v, a, s);
+cudaError_t launch_gla_bwd(const GlaVariant& v, const GlaArgs& a, bool saved, cudaStream_t s) {
+  if (v.dk == 32 && v.dv == 64) return dispatch_types<32, 64>(v, a, saved, s);
+  if (v.dk == 36 && v.dv == 72) return dispatch_types<36, 72>(v, a, saved, s);
+  if (v.dk == 64 && v.dv == 64) return dispatch_types<64, 64>(v, a, saved, s);
   return cudaErrorInvalidValue;
 }
 

@@ -55,6 +55,9 @@ lib.dig_gla_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i, _f, _vp, _vp, _vp, _
 lib.dig_gla_bwd.restype = _i
 lib.dig_gla_bwd.argtypes = [_vp, _vp, _vp, _vp, _i, _f, _vp, _vp, _vp, _vp, _vp,
                             _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]
+lib.dig_gla_bwd_saved.restype = _i
+lib.dig_gla_bwd_saved.argtypes = [_vp, _vp, _vp, _vp, _i, _f, _vp, _vp, _vp, _vp, _vp,
+                                  _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp, _sz, _vp]
 lib.dig_srem_reorient_dwconv.restype = _i
 lib.dig_srem_reorient_dwconv.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
 lib.dig_read_status.restype = _i
@@ -152,6 +155,19 @@ def dig_gla_bwd(q, k, v, z, inv_tau, dO, dq, dk, dv, dlog_alpha, grid_h, grid_w,
                          B, H, L, d_k, d_v, grid_h, grid_w, scan_mode, _code(q.dtype), _code(dq.dtype),
                          _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "dig_gla_bwd")
+
+
+def dig_gla_bwd_saved(q, k, v, z, inv_tau, dO, dq, dk, dv, dlog_alpha, grid_h, grid_w, scan_mode, fwd_workspace,
+                      workspace, stream=None):
+    """dig_gla_bwd reusing the records dig_gla_fwd left in fwd_workspace (same inputs, see include/dig.h)."""
+    B, L, H, d_k = q.shape
+    d_v = v.shape[3]
+    st = lib.dig_gla_bwd_saved(_ptr(q), _ptr(k), _ptr(v), _ptr(z), z.shape[2], float(inv_tau), _ptr(dO),
+                               _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlog_alpha),
+                               B, H, L, d_k, d_v, grid_h, grid_w, scan_mode, _code(q.dtype), _code(dq.dtype),
+                               _ptr(fwd_workspace), fwd_workspace.numel() * fwd_workspace.element_size(),
+                               _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "dig_gla_bwd_saved")
 
 
 def dig_srem_reorient_dwconv(x, w, bias, y, scan_mode, stream=None):

