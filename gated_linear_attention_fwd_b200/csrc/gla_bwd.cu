@@ -34,31 +34,38 @@ __host__ __device__ constexpr int bwd_chunk_len(int dk, int dv, bool f32) {
   return !f32 && 128 + 2 * cround(dk, 16) + cround(dv, 16) <= 256 ? 128 : 64;
 }
 
-template <int C, int DK, int DV, typename TIN>
+template <int C, int DK, int DV, typename TIN, typename TOUT>
 struct BwdCfg {
   using K = ChunkCfg<C, DK, DV, TIN>;
   static constexpr int NTG = K::NTG, NTV = K::NTV;
   static constexpr int NTP = 2;  // terms of the masked P-type matrices
-  // shared memory: operand rows (qbar, kbar, v, dO: token rows; S', Gt: value-channel rows)
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + NTG * K::AQ_SZ;
-  static constexpr int OFF_V = OFF_K + NTG * K::AQ_SZ;
+  // shared memory: v and dO rows first (the next unit's copies land there while
+  // this unit finishes), then qbar, kbar (token rows), S', Gt (value-channel rows)
+  static constexpr int OFF_V = 0;
   static constexpr int OFF_DO = OFF_V + NTV * K::VR_SZ;
-  static constexpr int OFF_SP = OFF_DO + NTV * K::VR_SZ;
+  static constexpr int OFF_Q = OFF_DO + NTV * K::VR_SZ;
+  static constexpr int OFF_K = OFF_Q + NTG * K::AQ_SZ;
+  static constexpr int OFF_SP = OFF_K + NTG * K::AQ_SZ;
   static constexpr int OFF_GT = OFF_SP + NTG * K::SPT_SZ;
   static constexpr int END_OPS = OFF_GT + NTG * K::SPT_SZ;
-  // staging of the gradient rows, over the operands once every product is done
-  static constexpr int VP = DV + 4, KP = DK + 4;
-  static constexpr int OFF_SV = 0;
-  static constexpr int OFF_SQ = OFF_SV + C * VP * 4;
-  static constexpr int OFF_SK = OFF_SQ + C * KP * 4;
-  static constexpr int END_STAGE = OFF_SK + C * KP * 4;
-  // token terms of d log alpha (their own region: written while SQ / SK are read)
-  static constexpr int OFF_SX = cround(cmax(END_OPS, END_STAGE), 16);
-  // M = 128 reads of C-row A operands (kbar, v, dO) may run past their rows
+  // gate factors EQ of the chunk's tokens (fp32 rows), overwritten in place by
+  // the tokens' d log alpha terms
+  static constexpr int EP = DK + 4;
+  static constexpr int OFF_EQ = cround(END_OPS, 16);
+  static constexpr int END_EQ = OFF_EQ + C * EP * 4;
+  // staging of the gradient rows in the output type, over qbar .. Gt once the
+  // last product is done; rows an odd number of 16-byte units apart (no bank
+  // conflicts between 8 consecutive rows)
+  static constexpr int KSB = 16 * (cdiv(DK * (int)sizeof(TOUT), 16) | 1);
+  static constexpr int VSB = 16 * (cdiv(DV * (int)sizeof(TOUT), 16) | 1);
+  static constexpr int OFF_SQ = OFF_Q, OFF_SK = OFF_SQ + C * KSB;
+  // dv beside dq and dk when all three fit, else alone in a second pass
+  static constexpr bool ONE_PASS = OFF_SK + C * KSB + C * VSB <= END_OPS;
+  static constexpr int OFF_SV = ONE_PASS ? OFF_SK + C * KSB : OFF_Q;
+  // M = 128 reads of C-row A operands (v, dO, kbar) may run past their rows
   // into the next buffers (those lanes are unused) but stay inside the allocation
   static constexpr int V_READ = (NTV - 1) * K::VR_SZ + 16 * K::SBO_V;
-  static constexpr int SMEM = cmax(cmax(OFF_SX + C * KP * 4, OFF_K + K::AQ_READ), OFF_DO + V_READ);
+  static constexpr int SMEM = cmax(cmax(END_EQ, OFF_K + K::AQ_READ), OFF_DO + V_READ);
   static constexpr int PER_SM = SMEM <= 110 * 1024 ? 2 : 1;
   // TMEM: one C x C region (P^T, then dP^T, then dP), dqbar, dkbar, dv
   static constexpr int PT_STRIDE = NTP * 8;
@@ -67,6 +74,7 @@ struct BwdCfg {
   static constexpr int TM_COLS = 256;
   static constexpr int NSG = 256 / DK;  // token segments of the d log alpha reverse cumsum
   static constexpr int SEGL = cdiv(C, NSG);
+  static_assert(OFF_SK + C * KSB <= END_OPS && OFF_SV + C * VSB <= END_OPS, "staging");
   static_assert(TM_DV + K::DVP <= TM_COLS, "TMEM budget");
   static_assert(SMEM <= 225 * 1024, "shared-memory budget");
   static_assert(C == bwd_chunk_len(DK, DV, std::is_same<TIN, float>::value), "chunk length");
@@ -81,8 +89,9 @@ struct GradSmem {
 };
 
 // Masks one C x C product in TMEM (lane = row r; keep column c >= r when
-// `upper`, else c <= r) and rewrites it as two bf16 terms in place, one K-step
-// of 16 columns at a time.  This thread covers the columns of its half.
+// `upper`, else c <= r) and rewrites it as two bf16 terms in place, 16 columns
+// (one K-step) at a time.  This thread covers the columns of its half; all of
+// its loads are issued before the one wait.
 template <int C, int PT_STRIDE>
 __device__ __forceinline__ void mask_to_terms(uint32_t tmem, uint32_t region, bool upper) {
   const int tid = threadIdx.x, t = tid & 127, wq = t >> 5, half = tid >> 7;
@@ -121,59 +130,122 @@ __device__ __forceinline__ void mask_to_terms(uint32_t tmem, uint32_t region, bo
   }
 }
 
-// TMEM row of this thread (lane t, N columns from col0 + O) -> staging row.
-template <int O, int N>
-__device__ __forceinline__ void stage_row(uint32_t lane_tm, int col0, float* dst, bool store) {
+// Sum of the NT bf16 terms of four consecutive K values of one operand row.
+template <int NT>
+__device__ __forceinline__ void ld_terms4(uint32_t saddr, uint32_t copy_bytes, float* x) {
+  x[0] = x[1] = x[2] = x[3] = 0.f;
 #pragma unroll
-  for (int c = 0; c < cround(N, 8); c += 8) {
-    float v[8];
-    tmem_ld8(lane_tm + col0 + O + c, v);
+  for (int i = 0; i < NT; ++i) {
+    uint32_t w0, w1;
+    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(saddr + i * copy_bytes));
+    x[0] += __uint_as_float(w0 << 16);
+    x[1] += __uint_as_float(w0 & 0xFFFF0000u);
+    x[2] += __uint_as_float(w1 << 16);
+    x[3] += __uint_as_float(w1 & 0xFFFF0000u);
+  }
+}
+
+// Four values in the output type to shared memory (8 bytes bf16, 16 bytes fp32).
+__device__ __forceinline__ void st_out4(__nv_bfloat16* p, const float* v) {
+  *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+}
+__device__ __forceinline__ void st_out4(float* p, const float* v) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+// BYTES (8, 16 or 32) from shared staging to global memory.
+template <int BYTES>
+__device__ __forceinline__ void copy_piece(void* dst, const void* src) {
+  if constexpr (BYTES == 8) {
+    *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(src);
+  } else {
+#pragma unroll
+    for (int i = 0; i < BYTES / 16; ++i) reinterpret_cast<uint4*>(dst)[i] = reinterpret_cast<const uint4*>(src)[i];
+  }
+}
+
+// Key gradients of this thread's token (TMEM lane t) and channel half:
+// dq = dqbar EQ and dk = dkbar / EQ into registers, and the token's d log alpha
+// terms x = qbar dqbar - kbar dkbar (qbar, kbar from their operand terms)
+// written over its EQ values.
+template <int C, int DK, int DV, typename TIN, typename TOUT, int H>
+__device__ __forceinline__ void key_grads(uint32_t tmem, uint32_t sbase, float* eqx, float* dq, float* dk) {
+  using K = ChunkCfg<C, DK, DV, TIN>;
+  using BC = BwdCfg<C, DK, DV, TIN, TOUT>;
+  constexpr int KO = H ? K::DK0 : 0, KN = H ? K::DK1 : K::DK0, NL = cround(KN, 8);
+  const int t = threadIdx.x & 127, wq = t >> 5;
+  if (32 * wq >= C) return;  // warp-uniform: lanes past the chunk
+  const uint32_t lt = tmem + (static_cast<uint32_t>(32 * wq) << 16);
+  float* row = eqx + t * BC::EP + KO;
+#pragma unroll
+  for (int c8 = 0; c8 < NL; c8 += 8) {
+    float dqb[8], dkb[8];
+    tmem_ld8(lt + BC::TM_DQ + KO + c8, dqb);
+    tmem_ld8(lt + BC::TM_DK + KO + c8, dkb);
     tmem_ld_wait();
-    if (store) {
-      if (c + 4 <= N) *reinterpret_cast<float4*>(dst + O + c) = make_float4(v[0], v[1], v[2], v[3]);
-      if (c + 8 <= N) *reinterpret_cast<float4*>(dst + O + c + 4) = make_float4(v[4], v[5], v[6], v[7]);
+#pragma unroll
+    for (int c4 = 0; c4 < 8 && c8 + c4 < KN; c4 += 4) {
+      const int c = c8 + c4;
+      const float4 f4 = *reinterpret_cast<const float4*>(row + c);
+      const float f[4] = {f4.x, f4.y, f4.z, f4.w};
+      float qb[4], kb[4], x[4];
+      ld_terms4<BC::NTG>(sbase + BC::OFF_Q + kmaj16(t, KO + c, 128, K::SBO_K), K::AQ_SZ, qb);
+      ld_terms4<BC::NTG>(sbase + BC::OFF_K + kmaj16(t, KO + c, 128, K::SBO_K), K::AQ_SZ, kb);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        dq[c + e] = dqb[c4 + e] * f[e];
+        dk[c + e] = dkb[c4 + e] * __fdividef(1.f, f[e]);
+        x[e] = qb[e] * dqb[c4 + e] - kb[e] * dkb[c4 + e];
+      }
+      *reinterpret_cast<float4*>(row + c) = make_float4(x[0], x[1], x[2], x[3]);
     }
   }
 }
 
-// Gradient rows of this thread's token (TMEM lane t) and channel half -> staging.
-template <int C, int DK, int DV, typename TIN, int H>
-__device__ __forceinline__ void stage_grads(uint32_t tmem, uint8_t* smem) {
+// dq and dk of this thread's token and channel half -> staging rows.
+template <int C, int DK, int DV, typename TIN, typename TOUT, int H>
+__device__ __forceinline__ void stage_key_grads(uint8_t* smem, const float* dq, const float* dk) {
   using K = ChunkCfg<C, DK, DV, TIN>;
-  using BC = BwdCfg<C, DK, DV, TIN>;
+  using BC = BwdCfg<C, DK, DV, TIN, TOUT>;
   constexpr int KO = H ? K::DK0 : 0, KN = H ? K::DK1 : K::DK0;
-  constexpr int VO = H ? K::DV0 : 0, VN = H ? K::DV1 : K::DV0;
-  const int t = threadIdx.x & 127, wq = t >> 5;
-  const uint32_t lt = tmem + (static_cast<uint32_t>(32 * wq) << 16);
-  const bool st = t < C;
-  stage_row<VO, VN>(lt, BC::TM_DV, reinterpret_cast<float*>(smem + BC::OFF_SV) + t * BC::VP, st);
-  stage_row<KO, KN>(lt, BC::TM_DQ, reinterpret_cast<float*>(smem + BC::OFF_SQ) + t * BC::KP, st);
-  stage_row<KO, KN>(lt, BC::TM_DK, reinterpret_cast<float*>(smem + BC::OFF_SK) + t * BC::KP, st);
+  const int t = threadIdx.x & 127;
+  if (t >= C) return;
+  TOUT* sq = reinterpret_cast<TOUT*>(smem + BC::OFF_SQ + t * BC::KSB) + KO;
+  TOUT* sk = reinterpret_cast<TOUT*>(smem + BC::OFF_SK + t * BC::KSB) + KO;
+#pragma unroll
+  for (int c = 0; c < KN; c += 4) {
+    st_out4(sq + c, dq + c);
+    st_out4(sk + c, dk + c);
+  }
 }
 
-__device__ __forceinline__ void st_global4(__nv_bfloat16* p, const float* v) {
-  uint2 u;
-  u.x = pack_bf16x2(v[0], v[1]);
-  u.y = pack_bf16x2(v[2], v[3]);
-  *reinterpret_cast<uint2*>(p) = u;
-}
-__device__ __forceinline__ void st_global4(float* p, const float* v) {
-  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
-}
-template <int PS, typename T>
-__device__ __forceinline__ void st_global_piece(T* p, const float* v) {
-  if constexpr (PS == 8) st_global8(p, v);
-  else st_global4(p, v);
+// dv of this thread's token (TMEM lane t) and channel half -> staging row.
+template <int C, int DK, int DV, typename TIN, typename TOUT, int H>
+__device__ __forceinline__ void stage_dv(uint32_t tmem, uint8_t* smem) {
+  using K = ChunkCfg<C, DK, DV, TIN>;
+  using BC = BwdCfg<C, DK, DV, TIN, TOUT>;
+  constexpr int VO = H ? K::DV0 : 0, VN = H ? K::DV1 : K::DV0;
+  const int t = threadIdx.x & 127, wq = t >> 5;
+  if (32 * wq >= C) return;  // warp-uniform
+  const uint32_t lt = tmem + (static_cast<uint32_t>(32 * wq) << 16) + BC::TM_DV + VO;
+  float v[VN];
+#pragma unroll
+  for (int c = 0; c < VN; c += 8) tmem_ld8(lt + c, v + c);
+  tmem_ld_wait();
+  TOUT* sv = reinterpret_cast<TOUT*>(smem + BC::OFF_SV + t * BC::VSB) + VO;
+#pragma unroll
+  for (int c = 0; c < VN; c += 4) st_out4(sv + c, v + c);
 }
 
 template <int C, int DK, int DV, typename TIN, typename TOUT>
 __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a) {
   using K = ChunkCfg<C, DK, DV, TIN>;
-  using BC = BwdCfg<C, DK, DV, TIN>;
+  using BC = BwdCfg<C, DK, DV, TIN, TOUT>;
   constexpr int NTG = BC::NTG, NTV = BC::NTV, NTP = BC::NTP, DKP = K::DKP, DVP = K::DVP, PSK = K::PSK;
+  constexpr int KL = cround(K::DK0, 8);  // key-gradient registers of a channel half
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ GradSmem sh;
   const int tid = threadIdx.x, warp = tid >> 5;
+  const int nunits = a.B * a.H * a.nchunks;
   if (warp == 0) {
     tmem_alloc(&sh.tmem, BC::TM_COLS);
     tmem_relinquish();
@@ -183,7 +255,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
     fence_mbar_init();
   }
   if (tid < 128) sh.bnd[tid >> 6][tid & 63] = 0.f;
-  if ((int)blockIdx.x < a.B * a.H * a.nchunks) fill_rows(a, blockIdx.x, C, sh.rows[0]);
+  if ((int)blockIdx.x < nunits) fill_rows(a, blockIdx.x, C, sh.rows[0]);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -195,11 +267,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
   const uint64_t dDOk = sdesc(sbase + BC::OFF_DO, 128, K::SBO_V), dDOm = sdesc(sbase + BC::OFF_DO, K::SBO_V, 128);
   const uint64_t dSPm = sdesc(sbase + BC::OFF_SP, K::SBO_K, 128);
   const uint64_t dGTm = sdesc(sbase + BC::OFF_GT, K::SBO_K, 128), dGTk = sdesc(sbase + BC::OFF_GT, 128, K::SBO_K);
-  const float* SQ = reinterpret_cast<const float*>(smem + BC::OFF_SQ);
-  const float* SK = reinterpret_cast<const float*>(smem + BC::OFF_SK);
-  const float* SV = reinterpret_cast<const float*>(smem + BC::OFF_SV);
-  float* SX = reinterpret_cast<float*>(smem + BC::OFF_SX);
-  const int nunits = a.B * a.H * a.nchunks;
+  float* EQ = reinterpret_cast<float*>(smem + BC::OFF_EQ);  // EQ rows, then the d log alpha terms
   uint32_t ph = 0;
   int it = 0;
   bool timed_out = false;
@@ -214,102 +282,129 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
     tc_fence_after();
   };
 
+  // Row pieces of a unit (q, k, EQ; S_n, G_n, S_{n+1} and chunk constants).
+  // With 128-token chunks (where they fit 72 registers) they are loaded one unit
+  // ahead: issued while the previous unit's d log alpha is formed, consumed as
+  // the unit's operands.  Otherwise (64-token chunks, whose wider rows leave no
+  // room) each group is loaded when the unit starts, just before its use.
+  constexpr int RQ = K::NPK * (2 * PSK * (int)sizeof(TIN) / 4 + PSK), RS = K::NPS * 20;
+  constexpr bool PRE = C == 128 && RQ + RS <= 72;
+  Piece<TIN, PSK> pq[K::NPK], pk[K::NPK];
+  Piece<float, PSK> pe[K::NPK];
+  Piece<float, 4> ps[K::NPS], pg[K::NPS], pn[K::NPS], pc0[K::NPS], pc1[K::NPS];
+  auto issue_qk = [&](int u, const long long* rows) {
+    const Unit U(a, u);
+#pragma unroll
+    for (int j = 0; j < K::NPK; ++j) {
+      const int i = tid + 256 * j;
+      int tt, g;
+      piece_of<K::NGK>(i, tt, g);
+      const long long gr = i < C * K::NGK ? rows[tt] : -1;
+      const bool valid = gr >= 0;
+      const size_t off = tok_row(gr, a, U.h) * DK + g * PSK;
+      pq[j].load(reinterpret_cast<const TIN*>(a.q) + off, valid);
+      pk[j].load(reinterpret_cast<const TIN*>(a.k) + off, valid);
+      pe[j].load(a.gEQ + ((size_t)U.bz * a.L + (valid ? U.n * C + tt : 0)) * DK + g * PSK, valid);
+    }
+  };
+  auto issue_s = [&](int u) {
+    const Unit U(a, u);
+    const bool has_next_chunk = U.n + 1 < a.nchunks;  // G of the last chunk is zero
+#pragma unroll
+    for (int j = 0; j < K::NPS; ++j) {
+      const int i = tid + 256 * j;
+      int jr, g;
+      piece_of<K::NGS>(i, jr, g);
+      const bool in = i < DV * K::NGS;
+      const size_t row = ((size_t)u * DV + (in ? jr : 0)) * DK + 4 * g;
+      ps[j].load_cg(a.dsn + row, in);
+      pg[j].load_cg(a.dhn + row, in);
+      pn[j].load_cg(a.dsn + row + (size_t)DV * DK, in && has_next_chunk);
+      const float* ch = a.gCH + ((size_t)U.bz * a.nchunks + U.n) * 4 * DK + 4 * g;
+      pc0[j].load(ch, in);
+      pc1[j].load(ch + DK, in);
+    }
+  };
+  if ((int)blockIdx.x < nunits) {
+    const int h0 = Unit(a, blockIdx.x).h;
+    if constexpr (PRE) {
+      issue_qk(blockIdx.x, sh.rows[0]);
+      issue_s(blockIdx.x);
+    }
+    load_v_rows_t<C, DK, DV, TIN>(a, h0, sh.rows[0], a.v, sbase + BC::OFF_V);
+    load_v_rows_t<C, DK, DV, TIN>(a, h0, sh.rows[0], a.dO, sbase + BC::OFF_DO);
+  }
+
   for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
     const Unit U(a, u);
     const int hz = U.bz - U.b * a.gate_heads;
+    const int un = u + gridDim.x;
+    const bool has_next = un < nunits;
     float* bnd = sh.bnd[it & 1];
     const long long* rows = sh.rows[it & 1];  // this unit's grid tokens
-    // ---- operands: qbar, kbar rows; S' and Gt rows; v and dO rows; the boundary term of d log alpha
-    load_v_rows_t<C, DK, DV, TIN>(a, U.h, rows, a.v, sbase + BC::OFF_V);
-    load_v_rows_t<C, DK, DV, TIN>(a, U.h, rows, a.dO, sbase + BC::OFF_DO);
-    {
-      Piece<TIN, PSK> pq[K::NPK], pk[K::NPK];
-      Piece<float, PSK> pe[K::NPK];
+    long long* rows_next = sh.rows[(it + 1) & 1];
+    if (has_next) fill_rows(a, un, C, rows_next);  // read after the operand barrier
+    if constexpr (!PRE) issue_qk(u, rows);
+    // ---- operands from the prefetched pieces: qbar, kbar rows and EQ; S' and Gt rows; the boundary term
 #pragma unroll
-      for (int j = 0; j < K::NPK; ++j) {
-        const int i = tid + 256 * j;
-        int tt, g;
-        piece_of<K::NGK>(i, tt, g);
-        const long long gr = i < C * K::NGK ? rows[tt] : -1;
-        const bool valid = gr >= 0;
-        const size_t off = tok_row(gr, a, U.h) * DK + g * PSK;
-        pq[j].load(reinterpret_cast<const TIN*>(a.q) + off, valid);
-        pk[j].load(reinterpret_cast<const TIN*>(a.k) + off, valid);
-        pe[j].load(a.gEQ + ((size_t)U.bz * a.L + (valid ? U.n * C + tt : 0)) * DK + g * PSK, valid);
-      }
+    for (int j = 0; j < K::NPK; ++j) {
+      const int i = tid + 256 * j;
+      int tt, g;
+      piece_of<K::NGK>(i, tt, g);
+      if (i < C * K::NGK) {
+        const bool valid = U.n * C + tt < a.L;
+        float qv[PSK], kv[PSK], ev[PSK];
+        pq[j].unpack(qv);
+        pk[j].unpack(kv);
+        pe[j].unpack(ev);
 #pragma unroll
-      for (int j = 0; j < K::NPK; ++j) {
-        const int i = tid + 256 * j;
-        int tt, g;
-        piece_of<K::NGK>(i, tt, g);
-        if (i < C * K::NGK) {
-          const bool valid = U.n * C + tt < a.L;
-          float qv[PSK], kv[PSK], ev[PSK];
-          pq[j].unpack(qv);
-          pk[j].unpack(kv);
-          pe[j].unpack(ev);
-#pragma unroll
-          for (int e = 0; e < PSK; ++e) {
-            const float f = valid ? ev[e] : 1.f;
-            qv[e] *= f;
-            kv[e] *= __fdividef(1.f, f);
-          }
-          st_piece<NTG, PSK>(sbase + BC::OFF_Q, tt, K::SBO_K, g * PSK, K::AQ_SZ, qv);
-          st_piece<NTG, PSK>(sbase + BC::OFF_K, tt, K::SBO_K, g * PSK, K::AQ_SZ, kv);
+        for (int e = 0; e < PSK; ++e) {
+          ev[e] = valid ? ev[e] : 1.f;
+          qv[e] *= ev[e];
+          kv[e] *= __fdividef(1.f, ev[e]);
         }
+        st_piece<NTG, PSK>(sbase + BC::OFF_Q, tt, K::SBO_K, g * PSK, K::AQ_SZ, qv);
+        st_piece<NTG, PSK>(sbase + BC::OFF_K, tt, K::SBO_K, g * PSK, K::AQ_SZ, kv);
+#pragma unroll
+        for (int e = 0; e < PSK; e += 4)
+          *reinterpret_cast<float4*>(EQ + tt * BC::EP + g * PSK + e) =
+              make_float4(ev[e], ev[e + 1], ev[e + 2], ev[e + 3]);
       }
     }
-    {
-      const bool has_next_chunk = U.n + 1 < a.nchunks;  // G of the last chunk is zero
-      Piece<float, 4> ps[K::NPS], pg[K::NPS], pn[K::NPS], pc0[K::NPS], pc1[K::NPS];
+    if constexpr (!PRE) issue_s(u);  // after the q / k pieces are consumed (register budget)
 #pragma unroll
-      for (int j = 0; j < K::NPS; ++j) {
-        const int i = tid + 256 * j;
-        int jr, g;
-        piece_of<K::NGS>(i, jr, g);
-        const bool in = i < DV * K::NGS;
-        const size_t row = ((size_t)u * DV + (in ? jr : 0)) * DK + 4 * g;
-        ps[j].load_cg(a.dsn + row, in);
-        pg[j].load_cg(a.dhn + row, in);
-        pn[j].load_cg(a.dsn + row + (size_t)DV * DK, in && has_next_chunk);
-        const float* ch = a.gCH + ((size_t)U.bz * a.nchunks + U.n) * 4 * DK + 4 * g;
-        pc0[j].load(ch, in);
-        pc1[j].load(ch + DK, in);
+    for (int j = 0; j < K::NPS; ++j) {
+      const int i = tid + 256 * j;
+      int jr, g;
+      piece_of<K::NGS>(i, jr, g);
+      const bool in = i < DV * K::NGS;
+      float sv[4], gv[4], nv[4], c0[4], c1[4];
+      ps[j].unpack(sv);
+      pg[j].unpack(gv);
+      pn[j].unpack(nv);
+      pc0[j].unpack(c0);
+      pc1[j].unpack(c1);
+      float bp[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        bp[e] = nv[e] * gv[e];  // zero outside the rows and for the last chunk
+        sv[e] *= c0[e];         // S' = 2^r S_n
+        gv[e] *= c1[e];         // Gt = 2^(Gamma - r) G_n
       }
+      if (in) {
+        st_piece<NTG, 4>(sbase + BC::OFF_SP, jr, K::SBO_K, 4 * g, K::SPT_SZ, sv);
+        st_piece<NTG, 4>(sbase + BC::OFF_GT, jr, K::SBO_K, 4 * g, K::SPT_SZ, gv);
+      }
+      // sum over the 8 rows of this lane group (lanes i..i+7 share the channel group)
 #pragma unroll
-      for (int j = 0; j < K::NPS; ++j) {
-        const int i = tid + 256 * j;
-        int jr, g;
-        piece_of<K::NGS>(i, jr, g);
-        const bool in = i < DV * K::NGS;
-        float sv[4], gv[4], nv[4], c0[4], c1[4];
-        ps[j].unpack(sv);
-        pg[j].unpack(gv);
-        pn[j].unpack(nv);
-        pc0[j].unpack(c0);
-        pc1[j].unpack(c1);
-        float bp[4];
+      for (int e = 0; e < 4; ++e) {
+        bp[e] += __shfl_xor_sync(0xffffffffu, bp[e], 1);
+        bp[e] += __shfl_xor_sync(0xffffffffu, bp[e], 2);
+        bp[e] += __shfl_xor_sync(0xffffffffu, bp[e], 4);
+      }
+      if (in && (i & 7) == 0) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          bp[e] = nv[e] * gv[e];  // zero outside the rows and for the last chunk
-          sv[e] *= c0[e];         // S' = 2^r S_n
-          gv[e] *= c1[e];         // Gt = 2^(Gamma - r) G_n
-        }
-        if (in) {
-          st_piece<NTG, 4>(sbase + BC::OFF_SP, jr, K::SBO_K, 4 * g, K::SPT_SZ, sv);
-          st_piece<NTG, 4>(sbase + BC::OFF_GT, jr, K::SBO_K, 4 * g, K::SPT_SZ, gv);
-        }
-        // sum over the 8 rows of this lane group (lanes i..i+7 share the channel group)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          bp[e] += __shfl_xor_sync(0xffffffffu, bp[e], 1);
-          bp[e] += __shfl_xor_sync(0xffffffffu, bp[e], 2);
-          bp[e] += __shfl_xor_sync(0xffffffffu, bp[e], 4);
-        }
-        if (in && (i & 7) == 0) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) atomicAdd(&bnd[4 * g + e], bp[e]);
-        }
+        for (int e = 0; e < 4; ++e) atomicAdd(&bnd[4 * g + e], bp[e]);
       }
     }
     {  // zero padding: key channels DK..DKP of every row; value rows DV..DVP of S' and Gt
@@ -379,6 +474,12 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
       mma_commit(&sh.bar[4]);
     }
     wait_all(4);
+    // v and dO are no longer read: the next unit's rows start to arrive now
+    if (has_next) {
+      const int hn = Unit(a, un).h;
+      load_v_rows_t<C, DK, DV, TIN>(a, hn, rows_next, a.v, sbase + BC::OFF_V);
+      load_v_rows_t<C, DK, DV, TIN>(a, hn, rows_next, a.dO, sbase + BC::OFF_DO);
+    }
     mask_to_terms<C, BC::PT_STRIDE>(tmem, BC::TM_R, false);
     tmem_st_wait();
     publish();
@@ -390,80 +491,67 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
     }
     wait_all(5);
     ph ^= 1u;
-    // ---- gradient rows -> staging (the operands are no longer read)
-    if (tid < 128) stage_grads<C, DK, DV, TIN, 0>(tmem, smem);
-    else stage_grads<C, DK, DV, TIN, 1>(tmem, smem);
+    // ---- dq, dk and the tokens' d log alpha terms from TMEM, the operands and EQ
+    float dq[KL], dk[KL];
+    if (tid < 128) key_grads<C, DK, DV, TIN, TOUT, 0>(tmem, sbase, EQ, dq, dk);
+    else key_grads<C, DK, DV, TIN, TOUT, 1>(tmem, sbase, EQ, dq, dk);
+    tc_fence_before();
+    __syncthreads();  // qbar, kbar read: their rows become staging
+    if (tid < 128) stage_key_grads<C, DK, DV, TIN, TOUT, 0>(smem, dq, dk);
+    else stage_key_grads<C, DK, DV, TIN, TOUT, 1>(smem, dq, dk);
+    if constexpr (BC::ONE_PASS) {
+      if (tid < 128) stage_dv<C, DK, DV, TIN, TOUT, 0>(tmem, smem);
+      else stage_dv<C, DK, DV, TIN, TOUT, 1>(tmem, smem);
+    }
     tc_fence_before();
     __syncthreads();
-    // ---- dv, dq, dk rows (coalesced pieces); the tokens' d log alpha terms
+    // ---- the next unit's row pieces start to arrive; dq, dk (and dv) rows as coalesced pieces
+    if (PRE && has_next) {
+      issue_qk(un, rows_next);
+      issue_s(un);
+    }
+    constexpr int KPB = PSK * (int)sizeof(TOUT), VPB = 8 * (int)sizeof(TOUT);
 #pragma unroll
-    for (int j = 0; j < K::NPV; ++j) {
+    for (int j = 0; j < K::NPK; ++j) {
       const int i = tid + 256 * j;
       int tt, g;
-      piece_of<K::NGV>(i, tt, g);
-      const long long gr = i < C * K::NGV ? rows[tt] : -1;
+      piece_of<K::NGK>(i, tt, g);
+      const long long gr = i < C * K::NGK ? rows[tt] : -1;
       if (gr >= 0) {
-        const float4 v0 = *reinterpret_cast<const float4*>(SV + tt * BC::VP + 8 * g);
-        const float4 v1 = *reinterpret_cast<const float4*>(SV + tt * BC::VP + 8 * g + 4);
-        const float vv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        st_global8(reinterpret_cast<TOUT*>(a.dv) + tok_row(gr, a, U.h) * DV + 8 * g, vv);
-      }
-    }
-    {
-      Piece<TIN, PSK> pq[K::NPK], pk[K::NPK];
-      Piece<float, PSK> pe[K::NPK];
-#pragma unroll
-      for (int j = 0; j < K::NPK; ++j) {  // q, k and the gate factors again (L2-resident)
-        const int i = tid + 256 * j;
-        int tt, g;
-        piece_of<K::NGK>(i, tt, g);
-        const long long gr = i < C * K::NGK ? rows[tt] : -1;
-        const bool valid = gr >= 0;
         const size_t off = tok_row(gr, a, U.h) * DK + g * PSK;
-        pq[j].load(reinterpret_cast<const TIN*>(a.q) + off, valid);
-        pk[j].load(reinterpret_cast<const TIN*>(a.k) + off, valid);
-        pe[j].load(a.gEQ + ((size_t)U.bz * a.L + (valid ? U.n * C + tt : 0)) * DK + g * PSK, valid);
-      }
-#pragma unroll
-      for (int j = 0; j < K::NPK; ++j) {
-        const int i = tid + 256 * j;
-        int tt, g;
-        piece_of<K::NGK>(i, tt, g);
-        const int p = U.n * C + tt;
-        if (i < C * K::NGK) {
-          const bool valid = p < a.L;
-          float qv[PSK], kv[PSK], ev[PSK], dq[PSK], dk[PSK], x[PSK];
-          pq[j].unpack(qv);
-          pk[j].unpack(kv);
-          pe[j].unpack(ev);
-#pragma unroll
-          for (int e = 0; e < PSK; ++e) {
-            const float f = valid ? ev[e] : 1.f, rf = __fdividef(1.f, f);
-            const float dqb = SQ[tt * BC::KP + g * PSK + e], dkb = SK[tt * BC::KP + g * PSK + e];
-            dq[e] = dqb * f;
-            dk[e] = dkb * rf;
-            x[e] = qv[e] * f * dqb - kv[e] * rf * dkb;  // qbar dqbar - kbar dkbar
-          }
-#pragma unroll
-          for (int e = 0; e < PSK; e += 4)
-            *reinterpret_cast<float4*>(SX + tt * BC::KP + g * PSK + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
-          if (valid) {
-            const size_t off = tok_row(rows[tt], a, U.h) * DK + g * PSK;
-            st_global_piece<PSK>(reinterpret_cast<TOUT*>(a.dq) + off, dq);
-            st_global_piece<PSK>(reinterpret_cast<TOUT*>(a.dk) + off, dk);
-          }
-        }
+        copy_piece<KPB>(reinterpret_cast<TOUT*>(a.dq) + off, smem + BC::OFF_SQ + tt * BC::KSB + g * KPB);
+        copy_piece<KPB>(reinterpret_cast<TOUT*>(a.dk) + off, smem + BC::OFF_SK + tt * BC::KSB + g * KPB);
       }
     }
-    __syncthreads();
+    auto store_dv = [&]() {
+#pragma unroll
+      for (int j = 0; j < K::NPV; ++j) {
+        const int i = tid + 256 * j;
+        int tt, g;
+        piece_of<K::NGV>(i, tt, g);
+        const long long gr = i < C * K::NGV ? rows[tt] : -1;
+        if (gr >= 0)
+          copy_piece<VPB>(reinterpret_cast<TOUT*>(a.dv) + tok_row(gr, a, U.h) * DV + 8 * g,
+                          smem + BC::OFF_SV + tt * BC::VSB + g * VPB);
+      }
+    };
+    if constexpr (BC::ONE_PASS) {
+      store_dv();
+    } else {
+      __syncthreads();  // dq / dk staging read: dv takes its place
+      if (tid < 128) stage_dv<C, DK, DV, TIN, TOUT, 0>(tmem, smem);
+      else stage_dv<C, DK, DV, TIN, TOUT, 1>(tmem, smem);
+      __syncthreads();
+      store_dv();
+    }
     // ---- d log alpha: reverse cumsum over the chunk's tokens + the boundary term
     const int sc = tid % DK, sg = tid / DK;
     const int t0 = sg * BC::SEGL, t1 = min(C, t0 + BC::SEGL);
     if (sg < BC::NSG) {
       float acc = 0.f;
       for (int t = t1 - 1; t >= t0; --t) {
-        acc += SX[t * BC::KP + sc];
-        SX[t * BC::KP + sc] = acc;
+        acc += EQ[t * BC::EP + sc];
+        EQ[t * BC::EP + sc] = acc;
       }
       sh.segtot[sg][sc] = acc;
     }
@@ -476,14 +564,13 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
         const long long gr = rows[t];
         if (gr >= 0) {
           float* dst = a.dla + ((size_t)gr * a.gate_heads + hz) * DK + sc;
-          const float val = SX[t * BC::KP + sc] + post;
+          const float val = EQ[t * BC::EP + sc] + post;
           if (a.gate_heads == 1) atomicAdd(dst, val);
           else *dst = val;
         }
       }
     }
-    if (u + (int)gridDim.x < nunits) fill_rows(a, u + gridDim.x, C, sh.rows[(it + 1) & 1]);
-    __syncthreads();  // staging, segment totals and the operands are reused by the next unit
+    __syncthreads();  // staging, EQ rows and segment totals are reused by the next unit
   }
   if (timed_out) set_status(a.status, DIG_ERR_DEVICE_TIMEOUT);
   tc_fence_before();
@@ -627,7 +714,7 @@ namespace {
 template <int DK, int DV, typename TIN, typename TOUT>
 cudaError_t launch_typed(const GlaArgs& a, bool saved, cudaStream_t s) {
   constexpr int C = bwd_chunk_len(DK, DV, std::is_same<TIN, float>::value);
-  using BC = BwdCfg<C, DK, DV, TIN>;
+  using BC = BwdCfg<C, DK, DV, TIN, TOUT>;
   const long long units = (long long)a.B * a.H * a.nchunks;
   if (units <= 0) return cudaSuccess;
   cudaError_t e;

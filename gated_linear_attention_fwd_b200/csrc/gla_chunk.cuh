@@ -121,15 +121,17 @@ __device__ __forceinline__ size_t tok_row(long long grow, const GlaArgs& a, int 
 // asynchronous 16-byte copies, zero-filled past the sequence end (complete after
 // cp_async_wait_all); fp32 values are split into three bf16 terms.  Channels
 // DV..DVP are zeroed (they are a contracted dimension in some products).
-template <int C, int DK, int DV, typename TIN>
+// NTH threads of the CTA share the pieces.
+template <int C, int DK, int DV, typename TIN, int NTH = 256>
 __device__ __forceinline__ void load_v_rows_t(const GlaArgs& a, int h, const long long* rows, const void* src,
                                               uint32_t vr) {
   using Cfg = ChunkCfg<C, DK, DV, TIN>;
+  constexpr int NPV = cdiv(C * Cfg::NGV, NTH);
   const int tid = threadIdx.x;
   if constexpr (std::is_same<TIN, __nv_bfloat16>::value) {
 #pragma unroll
-    for (int j = 0; j < Cfg::NPV; ++j) {
-      const int i = tid + 256 * j;
+    for (int j = 0; j < NPV; ++j) {
+      const int i = tid + NTH * j;
       int t, g;
       piece_of<Cfg::NGV>(i, t, g);
       if (i < C * Cfg::NGV) {
@@ -139,18 +141,18 @@ __device__ __forceinline__ void load_v_rows_t(const GlaArgs& a, int h, const lon
       }
     }
   } else {
-    Piece<TIN, 8> pv[Cfg::NPV];
+    Piece<TIN, 8> pv[NPV];
 #pragma unroll
-    for (int j = 0; j < Cfg::NPV; ++j) {
-      const int i = tid + 256 * j;
+    for (int j = 0; j < NPV; ++j) {
+      const int i = tid + NTH * j;
       int t, g;
       piece_of<Cfg::NGV>(i, t, g);
       const long long gr = i < C * Cfg::NGV ? rows[t] : -1;
       pv[j].load(reinterpret_cast<const TIN*>(src) + tok_row(gr, a, h) * DV + 8 * g, gr >= 0);
     }
 #pragma unroll
-    for (int j = 0; j < Cfg::NPV; ++j) {
-      const int i = tid + 256 * j;
+    for (int j = 0; j < NPV; ++j) {
+      const int i = tid + NTH * j;
       int t, g;
       piece_of<Cfg::NGV>(i, t, g);
       if (i < C * Cfg::NGV) {
@@ -162,7 +164,7 @@ __device__ __forceinline__ void load_v_rows_t(const GlaArgs& a, int h, const lon
   }
   if constexpr (Cfg::NPADV > 0) {
     const float zz[8] = {};
-    for (int i = tid; i < C * Cfg::NPADV; i += 256)
+    for (int i = tid; i < C * Cfg::NPADV; i += NTH)
       st_piece<Cfg::NTV, 8>(vr, i / Cfg::NPADV, Cfg::SBO_V, DV + 8 * (i % Cfg::NPADV), Cfg::VR_SZ, zz);
   }
 }
