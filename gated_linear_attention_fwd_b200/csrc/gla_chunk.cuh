@@ -331,7 +331,7 @@ __global__ void __launch_bounds__(256, BWD ? 2 : 3) gla_chunk_state_kernel(const
         bad |= fmaxf(fmaxf(fabsf(d0), fabsf(d1)), fmaxf(fabsf(d2), fabsf(d3))) > 115.f;
         if (writer)
           *reinterpret_cast<float4*>(a.gEQ + ((size_t)U.bz * a.L + p) * DK + 4 * g) =
-              make_float4(exp2f(d0), exp2f(d1), exp2f(d2), exp2f(d3));
+              make_float4(ex2(d0), ex2(d1), ex2(d2), ex2(d3));
       }
     }
     if (writer && tid < DK) {
@@ -352,13 +352,13 @@ __global__ void __launch_bounds__(256, BWD ? 2 : 3) gla_chunk_state_kernel(const
         float kv[PSK];
         pk[j].unpack(kv);
 #pragma unroll
-        for (int e = 0; e < PSK; ++e) kv[e] *= exp2f(sh.gam[g * PSK + e] - G[t * SC::GP + g * PSK + e]);
+        for (int e = 0; e < PSK; ++e) kv[e] *= ex2(sh.gam[g * PSK + e] - G[t * SC::GP + g * PSK + e]);
         st_piece<NTG, PSK>(sbase + SC::OFF_KH, t, Cfg::SBO_K, g * PSK, Cfg::AQ_SZ, kv);
         if constexpr (BWD) {
           float qv[PSK];
           pq[j].unpack(qv);
 #pragma unroll
-          for (int e = 0; e < PSK; ++e) qv[e] *= exp2f(G[t * SC::GP + g * PSK + e]);
+          for (int e = 0; e < PSK; ++e) qv[e] *= ex2(G[t * SC::GP + g * PSK + e]);
           st_piece<NTG, PSK>(sbase + SC::OFF_QB, t, Cfg::SBO_K, g * PSK, Cfg::AQ_SZ, qv);
         }
       }

@@ -225,10 +225,20 @@ __device__ __forceinline__ R zero4() {
 }
 
 constexpr float kLog2e = 1.4426950408889634f;
+// 2^x by the hardware's approximate base-2 exponential (PTX ex2.approx.ftz.f32:
+// a few ulp; results below 2^-126 flush to 0).  The gate factors stay within
+// 2^+-115 (checked), so only the contributions of tokens decayed by more than
+// 2^-126 are affected, and those are negligible.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 // Base-2 log decay of one gate logit: inv_tau * log2(sigmoid(z)), evaluated as
-// inv_tau * (min(z, 0) * log2(e) - log2(1 + 2^(-|z| log2(e)))).
+// inv_tau * (min(z, 0) * log2(e) - log2(1 + 2^(-|z| log2(e)))).  The logarithm's
+// argument lies in (1, 2], where the fast __log2f is accurate to about 2^-22.
 __device__ __forceinline__ float log2_decay(float z, float inv_tau) {
-  return inv_tau * (fminf(z, 0.f) * kLog2e - log2f(1.f + exp2f(-fabsf(z) * kLog2e)));
+  return inv_tau * (fminf(z, 0.f) * kLog2e - __log2f(1.f + ex2(-fabsf(z) * kLog2e)));
 }
 
 // Issues D (+)= A * B for operands stored as NA / NB bf16 terms: every term

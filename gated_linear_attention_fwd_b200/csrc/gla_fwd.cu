@@ -447,7 +447,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
           }
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const float sw = __fdividef(rv[e], 1.f + exp2f(-rv[e] * kLog2e));  // Swish(r) = r sigmoid(r)
+            const float sw = __fdividef(rv[e], 1.f + ex2(-rv[e] * kLog2e));  // Swish(r) = r sigmoid(r)
             yv[e] = sw * ov[e] * inv * gm[e];
           }
           st_global8(reinterpret_cast<TOUT*>(a.y) + off, yv);
