@@ -2,11 +2,31 @@
 // loads/stores, workspace layout, device status word.
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_runtime.h>
 #include <cstdint>
 
 #include "../../include/dig.h"
 
 namespace dig {
+
+// Launches a kernel with programmatic stream serialization: it may be scheduled
+// while the previous kernel of the stream is still running, and every kernel of
+// this library waits (griddepcontrol.wait) before its first global memory access.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
 // Scan position t -> grid token index (DiG scanning directions).  Reversed
 // modes visit the forward order backwards; column modes walk down each column.

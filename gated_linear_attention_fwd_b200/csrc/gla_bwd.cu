@@ -259,6 +259,8 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_wait();  // the kernels before this one have completed
+  griddep_launch_dependents();
   const uint32_t tmem = sh.tmem;
   const uint32_t sbase = smem_u32(smem);
   const uint64_t dQk = sdesc(sbase + BC::OFF_Q, 128, K::SBO_K), dQm = sdesc(sbase + BC::OFF_Q, K::SBO_K, 128);
@@ -617,6 +619,8 @@ __global__ void __launch_bounds__(256, 3) gla_chunk_dh_kernel(const GlaArgs a) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_wait();  // the kernels before this one have completed
+  griddep_launch_dependents();
   const uint32_t tmem = sh.tmem;
   const uint32_t sbase = smem_u32(smem);
   float* SD = reinterpret_cast<float*>(smem + DC::OFF_SD);
@@ -723,8 +727,7 @@ cudaError_t launch_typed(const GlaArgs& a, bool saved, cudaStream_t s) {
     auto kd = gla_chunk_dh_kernel<C, DK, DV, TIN>;
     if ((e = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, DC::SMEM)) != cudaSuccess)
       return e;
-    kd<<<persistent_grid(DC::PER_SM, units), 256, DC::SMEM, s>>>(a);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(kd, persistent_grid(DC::PER_SM, units), 256, DC::SMEM, s, a)) != cudaSuccess) return e;
     if ((e = launch_state_scan(a, a.dhn, true, nullptr, false, DK, DV, s)) != cudaSuccess) return e;
   } else {
     if ((e = launch_chunk_state<C, DK, DV, TIN, true>(a, s)) != cudaSuccess) return e;
@@ -732,8 +735,7 @@ cudaError_t launch_typed(const GlaArgs& a, bool saved, cudaStream_t s) {
   }
   auto k = gla_chunk_grad_kernel<C, DK, DV, TIN, TOUT>;
   if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, BC::SMEM)) != cudaSuccess) return e;
-  k<<<persistent_grid(BC::PER_SM, units), 256, BC::SMEM, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(k, persistent_grid(BC::PER_SM, units), 256, BC::SMEM, s, a);
 }
 
 template <int DK, int DV>

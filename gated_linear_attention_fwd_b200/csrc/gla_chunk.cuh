@@ -218,6 +218,8 @@ __global__ void __launch_bounds__(256, BWD ? 2 : 3) gla_chunk_state_kernel(const
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_wait();  // the kernels before this one have completed
+  griddep_launch_dependents();
   const uint32_t tmem = sh.tmem;
   const uint32_t sbase = smem_u32(smem);
   float* G = reinterpret_cast<float*>(smem + SC::OFF_G);    // [C][GP] cumsum of log2 decays
@@ -465,8 +467,7 @@ cudaError_t launch_chunk_state(const GlaArgs& a, cudaStream_t s) {
   auto k1 = gla_chunk_state_kernel<C, DK, DV, TIN, BWD>;
   cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, SC::SMEM);
   if (e != cudaSuccess) return e;
-  k1<<<persistent_grid(SC::PER_SM, units), 256, SC::SMEM, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(k1, persistent_grid(SC::PER_SM, units), 256, SC::SMEM, s, a);
 }
 
 // Scan of per-chunk contributions X_n (DV x DK fp32 each, per sequence) into

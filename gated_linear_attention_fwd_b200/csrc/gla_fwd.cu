@@ -103,6 +103,8 @@ struct ScanJob {
 __global__ void __launch_bounds__(kScanRanges * kScanQuads, 2) gla_state_scan_kernel(const GlaArgs a, ScanJob job,
                                                                                      int dk, int dv) {
   __shared__ float4 sA[kScanRanges][kScanQuads], sS[kScanRanges][kScanQuads];
+  griddep_wait();  // the kernels before this one have completed
+  griddep_launch_dependents();
   float* buf = blockIdx.y ? job.buf[1] : job.buf[0];
   const int reverse = blockIdx.y ? job.reverse[1] : job.reverse[0];
   const int nq = dv * dk / 4;
@@ -227,6 +229,8 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_wait();  // the kernels before this one have completed
+  griddep_launch_dependents();
   const int t = tid & 127, wq = (tid >> 5) & 3, half = tid >> 7;
   const uint32_t lane_base = static_cast<uint32_t>(32 * wq) << 16;
   const uint32_t tmem = sh.tmem;
@@ -488,8 +492,8 @@ cudaError_t launch_state_scan(const GlaArgs& a, float* buf0, bool rev0, float* b
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 2147483647LL) return cudaErrorInvalidValue;
   ScanJob job{{buf0, buf1}, {rev0 ? 1 : 0, rev1 ? 1 : 0}};
-  gla_state_scan_kernel<<<dim3((unsigned)blocks, buf1 ? 2u : 1u), kScanRanges * kScanQuads, 0, s>>>(a, job, dk, dv);
-  return cudaGetLastError();
+  return launch_pdl(gla_state_scan_kernel, dim3((unsigned)blocks, buf1 ? 2u : 1u), kScanRanges * kScanQuads, 0, s, a,
+                    job, dk, dv);
 }
 
 namespace {
@@ -504,7 +508,7 @@ cudaError_t launch_typed(const GlaArgs& a, cudaStream_t s) {
   if ((e = launch_state_scan(a, a.dsn, false, nullptr, false, DK, DV, s)) != cudaSuccess) return e;
   auto k3 = gla_chunk_out_kernel<C, DK, DV, TIN, TOUT>;
   if ((e = cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, OC::SMEM)) != cudaSuccess) return e;
-  k3<<<persistent_grid(2, units), 256, OC::SMEM, s>>>(a);
+  if ((e = launch_pdl(k3, persistent_grid(2, units), 256, OC::SMEM, s, a)) != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

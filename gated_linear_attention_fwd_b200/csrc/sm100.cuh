@@ -63,6 +63,20 @@ __device__ __forceinline__ void named_bar(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// ------------------------------------------------------------------ dependent launch
+// Kernels of one stream are launched with programmatic stream serialization: a
+// kernel may be scheduled while the kernel before it is still running, runs its
+// prologue (TMEM allocation, barrier setup, tables computed from its arguments;
+// no global memory), and then waits here until every kernel it depends on has
+// completed and its memory is visible.  A no-op for a plain launch.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel of the stream be scheduled.  Called only after this
+// kernel's own griddep_wait, so a kernel starts at the earliest once the one two
+// places before it has completed, and never overlaps a kernel whose buffers it writes.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ fences
 __device__ __forceinline__ void fence_async_smem() {
   // make generic-proxy shared-memory writes visible to the tensor core (async proxy)

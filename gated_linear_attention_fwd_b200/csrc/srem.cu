@@ -84,6 +84,8 @@ template <typename TIN, typename TOUT, int CP, int TW, int R, int MINB>
 __global__ void __launch_bounds__(256, MINB) srem_dwconv_kernel(const TIN* __restrict__ x, const float* __restrict__ w,
                                                              const float* __restrict__ bias, TOUT* __restrict__ y,
                                                              int B, int Hg, int Wg, int C, int mode) {
+  griddep_wait();  // the kernels before this one have completed
+  griddep_launch_dependents();
   using VT = typename Vec<TIN, CP>::type;
   const int nv = C / CP;  // channel vectors per pixel
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
@@ -178,6 +180,8 @@ __global__ void __launch_bounds__(256) srem_dwconv_scalar_kernel(const TIN* __re
                                                                  const float* __restrict__ w,
                                                                  const float* __restrict__ bias, TOUT* __restrict__ y,
                                                                  int B, int Hg, int Wg, int C, int mode) {
+  griddep_wait();  // the kernels before this one have completed
+  griddep_launch_dependents();
   const long long total = (long long)B * Hg * Wg * C;
   for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
@@ -210,18 +214,16 @@ static cudaError_t launch_typed(const void* x, const float* w, const float* bias
     const long long total = (long long)B * Hg * Wg * C;
     const long long blocks = (total + 255) / 256;
     const int grid = (int)(blocks < 148LL * 32 ? blocks : 148LL * 32);
-    srem_dwconv_scalar_kernel<TIN, TOUT><<<grid, 256, 0, s>>>(reinterpret_cast<const TIN*>(x), w, bias,
-                                                               reinterpret_cast<TOUT*>(y), B, Hg, Wg, C, mode);
-    return cudaGetLastError();
+    return launch_pdl(srem_dwconv_scalar_kernel<TIN, TOUT>, dim3(grid), dim3(256), 0, s,
+                      reinterpret_cast<const TIN*>(x), w, bias, reinterpret_cast<TOUT*>(y), B, Hg, Wg, C, mode);
   }
   constexpr int CP = kConvCh, TW = kConvCols, R = kConvRows;
   const long long gx = ((long long)((Wg + TW - 1) / TW) * (C / CP) + 255) / 256;
   const long long gy = (Hg + R - 1) / R;
   if (gx > 2147483647LL || gy > 65535 || B > 65535) return cudaErrorInvalidValue;
   const dim3 grid((unsigned)gx, (unsigned)gy, (unsigned)B);
-  srem_dwconv_kernel<TIN, TOUT, CP, TW, R, kConvMinBlocks><<<grid, 256, 0, s>>>(
-      reinterpret_cast<const TIN*>(x), w, bias, reinterpret_cast<TOUT*>(y), B, Hg, Wg, C, mode);
-  return cudaGetLastError();
+  return launch_pdl(srem_dwconv_kernel<TIN, TOUT, CP, TW, R, kConvMinBlocks>, grid, dim3(256), 0, s,
+                    reinterpret_cast<const TIN*>(x), w, bias, reinterpret_cast<TOUT*>(y), B, Hg, Wg, C, mode);
 }
 
 cudaError_t launch_srem(const void* x, const float* w, const float* bias, void* y, int B, int Hg, int Wg, int C,
