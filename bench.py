@@ -191,7 +191,9 @@ def _config(w, world):
                         "epilogue + bwd + SREM 3x3 dwconv (C=%d); scan mode cycles over the 4 DiG directions"
                         % (w.name, w.B, w.grid_h, w.grid_w, w.L, w.H, w.dk, w.dv, w.conv_C),
             "global_batch": w.B * world, "seq_len": w.L, "parallelism": "replicas x%d" % world,
-            "l2": "flushed (512 MiB write) before every step, outside the timed events"}
+            "l2": "flushed (512 MiB write) before every step, outside the timed events",
+            "e2e": "all inputs copied in and all outputs copied out every step (pinned host buffers); copies on "
+                   "their own streams overlap the neighbouring steps' compute, two device buffer sets alternate"}
 
 
 def run_ours(args, rank, world, local_rank):
@@ -215,20 +217,26 @@ def run_ours(args, rank, world, local_rank):
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(i, ev=None):
+    def step(i, ev=None, t=None, strm=None):
+        """One step: forward + epilogue, backward from the forward's records, SREM conv."""
+        t = t or {"q": q, "k": k, "v": v, "z": z, "r": r, "dO": dO, "x": xc, "w": wc,
+                  "o": o, "y": y, "dq": dq, "dk": dk_, "dv": dv_, "dla": dla, "yc": yc}
+        strm = strm or stream
         mode = i % 4
         if ev:
-            ev[0].record(stream)
-        dig.dig_gla_fwd(q, k, v, z, w.inv_tau, o, w.grid_h, w.grid_w, mode, ws_f, r=r, y=y)
+            ev[0].record(strm)
+        dig.dig_gla_fwd(t["q"], t["k"], t["v"], t["z"], w.inv_tau, t["o"], w.grid_h, w.grid_w, mode, ws_f,
+                        r=t["r"], y=t["y"], stream=strm)
         if ev:
-            ev[1].record(stream)
+            ev[1].record(strm)
         # the backward of a training step reuses the forward's gate factors and chunk states
-        dig.dig_gla_bwd_saved(q, k, v, z, w.inv_tau, dO, dq, dk_, dv_, dla, w.grid_h, w.grid_w, mode, ws_f, ws_b)
+        dig.dig_gla_bwd_saved(t["q"], t["k"], t["v"], t["z"], w.inv_tau, t["dO"], t["dq"], t["dk"], t["dv"], t["dla"],
+                              w.grid_h, w.grid_w, mode, ws_f, ws_b, stream=strm)
         if ev:
-            ev[2].record(stream)
-        dig.dig_srem_reorient_dwconv(xc, wc, None, yc, mode)
+            ev[2].record(strm)
+        dig.dig_srem_reorient_dwconv(t["x"], t["w"], None, t["yc"], mode, stream=strm)
         if ev:
-            ev[3].record(stream)
+            ev[3].record(strm)
 
     for i in range(args.warmup):
         flush.fill_(float(i))
@@ -261,31 +269,53 @@ def run_ours(args, rank, world, local_rank):
         if st != dig.DIG_OK:
             raise RuntimeError("device status after timing: %s" % dig.lib.dig_status_string(st).decode())
 
-    # end to end: the same step through the C ABI with pinned host buffers
-    host_in = {n: a.cpu().pin_memory() for n, a in (("q", q), ("k", k), ("v", v), ("z", z), ("r", r), ("dO", dO),
-                                                     ("x", xc), ("w", wc))}
-    outs = (o, y, dq, dk_, dv_, dla, yc)
-    host_out = [a.cpu().pin_memory() for a in outs]
-    dev_in = {"q": q, "k": k, "v": v, "z": z, "r": r, "dO": dO, "x": xc, "w": wc}
+    # end to end: steps through the C ABI with pinned host buffers.  Every step
+    # copies all its inputs in (H2D stream), runs on the compute stream and copies
+    # all its outputs back (D2H stream).  Two device buffer sets alternate, so a
+    # step's copies overlap its neighbours' compute, as a training loop's input
+    # feed does; the time is that of the whole run from the first copy in to the
+    # last copy out, divided by the steps.
+    names_in = ("q", "k", "v", "z", "r", "dO", "x", "w")
+    cur = {"q": q, "k": k, "v": v, "z": z, "r": r, "dO": dO, "x": xc, "w": wc,
+           "o": o, "y": y, "dq": dq, "dk": dk_, "dv": dv_, "dla": dla, "yc": yc}
+    names_out = ("o", "y", "dq", "dk", "dv", "dla", "yc")
+    host_in = {n: cur[n].cpu().pin_memory() for n in names_in}
+    host_out = {n: cur[n].cpu().pin_memory() for n in names_out}
+    sets = [cur, {n: torch.empty_like(a) for n, a in cur.items()}]
     h2d = sum(a.numel() * a.element_size() for a in host_in.values())
-    d2h = sum(a.numel() * a.element_size() for a in outs)
-    e2e_steps = max(3, min(args.steps, 10))
+    d2h = sum(a.numel() * a.element_size() for a in host_out.values())
+    s_h2d, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    done = {kind: [torch.cuda.Event(), torch.cuda.Event()] for kind in ("h2d", "cmp", "d2h")}
+
+    def e2e_run(n, first):
+        for i in range(first, first + n):
+            b, t = i % 2, sets[i % 2]
+            if i - first >= 2:
+                s_h2d.wait_event(done["cmp"][b])  # step i-2 has consumed this set's inputs
+            with torch.cuda.stream(s_h2d):
+                for n_ in names_in:
+                    t[n_].copy_(host_in[n_], non_blocking=True)
+            done["h2d"][b].record(s_h2d)
+            stream.wait_event(done["h2d"][b])
+            if i - first >= 2:
+                stream.wait_event(done["d2h"][b])  # step i-2's outputs are back on the host
+            step(i, t=t, strm=stream)
+            done["cmp"][b].record(stream)
+            s_d2h.wait_event(done["cmp"][b])
+            with torch.cuda.stream(s_d2h):
+                for n_ in names_out:
+                    host_out[n_].copy_(t[n_], non_blocking=True)
+            done["d2h"][b].record(s_d2h)
+
+    e2e_steps = max(4, min(args.steps, 12))
+    e2e_run(2, 0)  # warm-up
+    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2e_ms = []
-    for i in range(e2e_steps + 1):
-        flush.fill_(float(i))
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for n_, hbuf in host_in.items():
-            dev_in[n_].copy_(hbuf, non_blocking=True)
-        step(i)
-        for hb, a in zip(host_out, outs):
-            hb.copy_(a, non_blocking=True)
-        e1.record(stream)
-        e1.synchronize()
-        if i > 0:
-            e2e_ms.append(e0.elapsed_time(e1))
-    e2e_step_ms = float(np.mean(e2e_ms))
+    e0.record(s_h2d)
+    e2e_run(e2e_steps, 2)
+    e1.record(s_d2h)
+    e1.synchronize()
+    e2e_step_ms = e0.elapsed_time(e1) / e2e_steps
     if world > 1:
         tt = torch.tensor([e2e_step_ms], device=dev)
         torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
