@@ -259,8 +259,6 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  griddep_wait();  // the kernels before this one have completed
-  griddep_launch_dependents();
   const uint32_t tmem = sh.tmem;
   const uint32_t sbase = smem_u32(smem);
   const uint64_t dQk = sdesc(sbase + BC::OFF_Q, 128, K::SBO_K), dQm = sdesc(sbase + BC::OFF_Q, K::SBO_K, 128);
@@ -327,15 +325,18 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
       pc1[j].load(ch + DK, in);
     }
   };
+  // The kernel before this one is the state scan, which writes only the chunk
+  // states and state gradients; everything older has completed.  So the first
+  // unit's other rows are requested before the wait for that scan.
   if ((int)blockIdx.x < nunits) {
     const int h0 = Unit(a, blockIdx.x).h;
-    if constexpr (PRE) {
-      issue_qk(blockIdx.x, sh.rows[0]);
-      issue_s(blockIdx.x);
-    }
+    if constexpr (PRE) issue_qk(blockIdx.x, sh.rows[0]);
     load_v_rows_t<C, DK, DV, TIN>(a, h0, sh.rows[0], a.v, sbase + BC::OFF_V);
     load_v_rows_t<C, DK, DV, TIN>(a, h0, sh.rows[0], a.dO, sbase + BC::OFF_DO);
   }
+  griddep_wait();  // the kernels before this one have completed
+  griddep_launch_dependents();
+  if (PRE && (int)blockIdx.x < nunits) issue_s(blockIdx.x);
 
   for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
     const Unit U(a, u);

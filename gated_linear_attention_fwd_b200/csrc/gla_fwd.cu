@@ -229,8 +229,6 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  griddep_wait();  // the kernels before this one have completed
-  griddep_launch_dependents();
   const int t = tid & 127, wq = (tid >> 5) & 3, half = tid >> 7;
   const uint32_t lane_base = static_cast<uint32_t>(32 * wq) << 16;
   const uint32_t tmem = sh.tmem;
@@ -271,9 +269,17 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
       const int i = tid + 256 * j;
       int jr, g;
       piece_of<Cfg::NGS>(i, jr, g);
+      pc[j].load(a.gCH + ((size_t)U.bz * a.nchunks + U.n) * 4 * DK + 4 * g, i < DV * Cfg::NGS);
+    }
+  };
+  auto issue_s = [&](int u) {  // entry-state rows (written by the scan before this kernel)
+#pragma unroll
+    for (int j = 0; j < Cfg::NPS; ++j) {
+      const int i = tid + 256 * j;
+      int jr, g;
+      piece_of<Cfg::NGS>(i, jr, g);
       const bool in = i < DV * Cfg::NGS;
       ps[j].load_cg(a.dsn + ((size_t)u * DV + (in ? jr : 0)) * DK + 4 * g, in);
-      pc[j].load(a.gCH + ((size_t)U.bz * a.nchunks + U.n) * 4 * DK + 4 * g, in);
     }
   };
   auto issue_r = [&](int h, const long long* rows) {
@@ -290,12 +296,18 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
   // Loading one unit ahead holds two units' pieces in registers; with 8-byte
   // pieces (d_k not a multiple of 8) that spills, so those variants load per unit.
   constexpr bool kAhead = PSK == 8;
+  // The kernel before this one is the state scan, which writes only the chunk
+  // states; everything older has completed.  So the first unit's other rows are
+  // requested before the wait for that scan.
   if (kAhead && (int)blockIdx.x < nunits) {
     const int h0 = Unit(a, blockIdx.x).h;
     issue_rows(blockIdx.x, sh.rows[0]);
     load_v_rows_t<C, DK, DV, TIN>(a, h0, sh.rows[0], a.v, sbase + OC::OFF_VR);
     issue_r(h0, sh.rows[0]);
   }
+  griddep_wait();  // the kernels before this one have completed
+  griddep_launch_dependents();
+  if (kAhead && (int)blockIdx.x < nunits) issue_s(blockIdx.x);
 
   int it = 0;
   for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
@@ -310,6 +322,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
         __syncthreads();
       }
       issue_rows(u, rows);
+      issue_s(u);
       load_v_rows_t<C, DK, DV, TIN>(a, U.h, rows, a.v, sbase + OC::OFF_VR);
     }
     if (has_next) fill_rows(a, un, C, rows_next);  // visible after the next barrier
@@ -368,7 +381,10 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
                                     idesc_bf16(128, OC::NB), false);  // [P | O] = qbar [kbar | S'^T]^T
       mma_commit(&sh.bar_a);
     }
-    if (has_next) issue_rows(un, rows_next);  // this unit's row pieces are consumed
+    if (has_next) {  // this unit's row pieces are consumed
+      issue_rows(un, rows_next);
+      issue_s(un);
+    }
     if (!mbar_wait(&sh.bar_a, ph, kSpinLimitNs)) timed_out = true;
     tc_fence_after();
     // ---- mask P (s <= t) and store it as bf16 terms in TMEM, one K-step of 16 at a time
