@@ -22,6 +22,12 @@
  *     never allocates, frees or keeps device memory, and never synchronises
  *     (except dig_read_status).  Work is enqueued on `stream` (a cudaStream_t;
  *     NULL = legacy default stream) and the call returns without waiting.
+ *     Stream order holds as for plain launches: the kernels are launched with
+ *     programmatic stream serialization, so one may be scheduled while the
+ *     previous kernel of the stream finishes, but each reads or writes global
+ *     memory written by that kernel only after waiting for its completion, and
+ *     writes nothing before then (any caller-side kernel that precedes a call
+ *     has completed before the call's first kernel touches memory).
  *   - Tensors are dense, row-major, tokens in GRID row-major order
  *     (token g = row * grid_w + col, L = grid_h * grid_w).  Pointers must be
  *     16-byte aligned.
