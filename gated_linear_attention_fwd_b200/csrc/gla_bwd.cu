@@ -75,6 +75,10 @@ struct BwdCfg {
   static constexpr int NSG = 256 / DK;  // token segments of the d log alpha reverse cumsum
   static constexpr int SEGL = cdiv(C, NSG);
   static_assert(OFF_SK + C * KSB <= END_OPS && OFF_SV + C * VSB <= END_OPS, "staging");
+  // the unit's state blocks (DV x DK fp32) land by bulk copy in the S', Gt and
+  // qbar slots and are converted in place
+  static_assert(DV * DK * 4 <= NTG * K::SPT_SZ && DV * DK * 4 <= NTG * K::AQ_SZ && (DV * DK * 4) % 16 == 0,
+                "state landing");
   static_assert(TM_DV + K::DVP <= TM_COLS, "TMEM budget");
   static_assert(SMEM <= 225 * 1024, "shared-memory budget");
   static_assert(C == bwd_chunk_len(DK, DV, std::is_same<TIN, float>::value), "chunk length");
@@ -82,9 +86,11 @@ struct BwdCfg {
 
 struct GradSmem {
   long long rows[2][128];  // grid tokens of the current and the next unit (by unit parity)
+  alignas(16) float gch[128];  // the unit's chunk constants: 2^r (d_k values), then 2^(Gamma - r) (bulk copy)
   float segtot[8][64];  // reverse-cumsum totals of the token segments
   float bnd[2][64];     // rowsum(S_{n+1} o G_n), double-buffered by unit parity
   uint64_t bar[6];      // completion of the six product groups of a unit
+  uint64_t sbar;        // completion of the unit's bulk copies (states and chunk constants)
   uint32_t tmem;
 };
 
@@ -252,6 +258,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
   }
   if (tid == 0) {
     for (int i = 0; i < 6; ++i) mbar_init(&sh.bar[i], 1);
+    mbar_init(&sh.sbar, 1);
     fence_mbar_init();
   }
   if (tid < 128) sh.bnd[tid >> 6][tid & 63] = 0.f;
@@ -282,16 +289,15 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
     tc_fence_after();
   };
 
-  // Row pieces of a unit (q, k, EQ; S_n, G_n, S_{n+1} and chunk constants).
-  // With 128-token chunks (where they fit 72 registers) they are loaded one unit
-  // ahead: issued while the previous unit's d log alpha is formed, consumed as
-  // the unit's operands.  Otherwise (64-token chunks, whose wider rows leave no
-  // room) each group is loaded when the unit starts, just before its use.
-  constexpr int RQ = K::NPK * (2 * PSK * (int)sizeof(TIN) / 4 + PSK), RS = K::NPS * 20;
-  constexpr bool PRE = C == 128 && RQ + RS <= 72;
+  // Row pieces of a unit (q, k, EQ).  With 128-token chunks (where they fit 40
+  // registers) they are loaded one unit ahead: issued while the previous unit's
+  // d log alpha is formed, consumed as the unit's operands.  Otherwise
+  // (64-token chunks, whose wider rows leave no room) they are loaded when the
+  // unit starts.
+  constexpr int RQ = K::NPK * (2 * PSK * (int)sizeof(TIN) / 4 + PSK);
+  constexpr bool PRE = C == 128 && RQ <= 40;
   Piece<TIN, PSK> pq[K::NPK], pk[K::NPK];
   Piece<float, PSK> pe[K::NPK];
-  Piece<float, 4> ps[K::NPS], pg[K::NPS], pn[K::NPS], pc0[K::NPS], pc1[K::NPS];
   auto issue_qk = [&](int u, const long long* rows) {
     const Unit U(a, u);
 #pragma unroll
@@ -307,23 +313,20 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
       pe[j].load(a.gEQ + ((size_t)U.bz * a.L + (valid ? U.n * C + tt : 0)) * DK + g * PSK, valid);
     }
   };
-  auto issue_s = [&](int u) {
+  // The unit's contiguous blocks by bulk copy (one thread; they bypass the
+  // load/store path): S_n into the S' slot, G_n into the Gt slot, S_{n+1} (not
+  // for the last chunk) into the qbar slot, and the chunk constants.  Issued for
+  // the next unit once this unit's gradient rows have left the staging over
+  // those slots, so they land while this unit's d log alpha is formed.
+  constexpr uint32_t SB = DV * DK * 4;
+  auto issue_states = [&](int u) {
     const Unit U(a, u);
     const bool has_next_chunk = U.n + 1 < a.nchunks;  // G of the last chunk is zero
-#pragma unroll
-    for (int j = 0; j < K::NPS; ++j) {
-      const int i = tid + 256 * j;
-      int jr, g;
-      piece_of<K::NGS>(i, jr, g);
-      const bool in = i < DV * K::NGS;
-      const size_t row = ((size_t)u * DV + (in ? jr : 0)) * DK + 4 * g;
-      ps[j].load_cg(a.dsn + row, in);
-      pg[j].load_cg(a.dhn + row, in);
-      pn[j].load_cg(a.dsn + row + (size_t)DV * DK, in && has_next_chunk);
-      const float* ch = a.gCH + ((size_t)U.bz * a.nchunks + U.n) * 4 * DK + 4 * g;
-      pc0[j].load(ch, in);
-      pc1[j].load(ch + DK, in);
-    }
+    mbar_arrive_expect_tx(&sh.sbar, 2 * SB + (has_next_chunk ? SB : 0u) + 2 * DK * 4);
+    bulk_copy_g2s(sbase + BC::OFF_SP, a.dsn + (size_t)u * DV * DK, SB, &sh.sbar);
+    bulk_copy_g2s(sbase + BC::OFF_GT, a.dhn + (size_t)u * DV * DK, SB, &sh.sbar);
+    if (has_next_chunk) bulk_copy_g2s(sbase + BC::OFF_Q, a.dsn + (size_t)(u + 1) * DV * DK, SB, &sh.sbar);
+    bulk_copy_g2s(smem_u32(sh.gch), a.gCH + ((size_t)U.bz * a.nchunks + U.n) * 4 * DK, 2 * DK * 4, &sh.sbar);
   };
   // The kernel before this one is the state scan, which writes only the chunk
   // states and state gradients; everything older has completed.  So the first
@@ -336,7 +339,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
   }
   griddep_wait();  // the kernels before this one have completed
   griddep_launch_dependents();
-  if (PRE && (int)blockIdx.x < nunits) issue_s(blockIdx.x);
+  if (tid == 0 && (int)blockIdx.x < nunits) issue_states(blockIdx.x);
 
   for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
     const Unit U(a, u);
@@ -347,8 +350,57 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
     const long long* rows = sh.rows[it & 1];  // this unit's grid tokens
     long long* rows_next = sh.rows[(it + 1) & 1];
     if (has_next) fill_rows(a, un, C, rows_next);  // read after the operand barrier
+    // ---- the state blocks, read in place: S' and Gt rows (to registers) and the boundary term
+    const bool has_next_chunk = U.n + 1 < a.nchunks;
+    if (!mbar_wait(&sh.sbar, ph, kSpinLimitNs)) timed_out = true;
+    float spv[K::NPS][4], gtv[K::NPS][4];
+#pragma unroll
+    for (int j = 0; j < K::NPS; ++j) {
+      const int i = tid + 256 * j;
+      int jr, g;
+      piece_of<K::NGS>(i, jr, g);
+      const bool in = i < DV * K::NGS;
+      const int off = (in ? jr * DK : 0) + 4 * g;
+      const float4 sv = *reinterpret_cast<const float4*>(smem + BC::OFF_SP + 4 * off);
+      const float4 gv = *reinterpret_cast<const float4*>(smem + BC::OFF_GT + 4 * off);
+      const float4 nv = has_next_chunk ? *reinterpret_cast<const float4*>(smem + BC::OFF_Q + 4 * off)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 c0 = *reinterpret_cast<const float4*>(&sh.gch[4 * g]);
+      const float4 c1 = *reinterpret_cast<const float4*>(&sh.gch[DK + 4 * g]);
+      spv[j][0] = sv.x * c0.x;  // S' = 2^r S_n
+      spv[j][1] = sv.y * c0.y;
+      spv[j][2] = sv.z * c0.z;
+      spv[j][3] = sv.w * c0.w;
+      gtv[j][0] = gv.x * c1.x;  // Gt = 2^(Gamma - r) G_n
+      gtv[j][1] = gv.y * c1.y;
+      gtv[j][2] = gv.z * c1.z;
+      gtv[j][3] = gv.w * c1.w;
+      float bp[4] = {in ? nv.x * gv.x : 0.f, in ? nv.y * gv.y : 0.f, in ? nv.z * gv.z : 0.f, in ? nv.w * gv.w : 0.f};
+      // sum over the 8 rows of this lane group (lanes i..i+7 share the channel group)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        bp[e] += __shfl_xor_sync(0xffffffffu, bp[e], 1);
+        bp[e] += __shfl_xor_sync(0xffffffffu, bp[e], 2);
+        bp[e] += __shfl_xor_sync(0xffffffffu, bp[e], 4);
+      }
+      if (in && (i & 7) == 0) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) atomicAdd(&bnd[4 * g + e], bp[e]);
+      }
+    }
+    __syncthreads();  // every state row read: the slots take the operands
+    // ---- operands: S' and Gt rows; qbar, kbar rows and EQ (from the q / k pieces)
+#pragma unroll
+    for (int j = 0; j < K::NPS; ++j) {
+      const int i = tid + 256 * j;
+      int jr, g;
+      piece_of<K::NGS>(i, jr, g);
+      if (i < DV * K::NGS) {
+        st_piece<NTG, 4>(sbase + BC::OFF_SP, jr, K::SBO_K, 4 * g, K::SPT_SZ, spv[j]);
+        st_piece<NTG, 4>(sbase + BC::OFF_GT, jr, K::SBO_K, 4 * g, K::SPT_SZ, gtv[j]);
+      }
+    }
     if constexpr (!PRE) issue_qk(u, rows);
-    // ---- operands from the prefetched pieces: qbar, kbar rows and EQ; S' and Gt rows; the boundary term
 #pragma unroll
     for (int j = 0; j < K::NPK; ++j) {
       const int i = tid + 256 * j;
@@ -372,42 +424,6 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
         for (int e = 0; e < PSK; e += 4)
           *reinterpret_cast<float4*>(EQ + tt * BC::EP + g * PSK + e) =
               make_float4(ev[e], ev[e + 1], ev[e + 2], ev[e + 3]);
-      }
-    }
-    if constexpr (!PRE) issue_s(u);  // after the q / k pieces are consumed (register budget)
-#pragma unroll
-    for (int j = 0; j < K::NPS; ++j) {
-      const int i = tid + 256 * j;
-      int jr, g;
-      piece_of<K::NGS>(i, jr, g);
-      const bool in = i < DV * K::NGS;
-      float sv[4], gv[4], nv[4], c0[4], c1[4];
-      ps[j].unpack(sv);
-      pg[j].unpack(gv);
-      pn[j].unpack(nv);
-      pc0[j].unpack(c0);
-      pc1[j].unpack(c1);
-      float bp[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        bp[e] = nv[e] * gv[e];  // zero outside the rows and for the last chunk
-        sv[e] *= c0[e];         // S' = 2^r S_n
-        gv[e] *= c1[e];         // Gt = 2^(Gamma - r) G_n
-      }
-      if (in) {
-        st_piece<NTG, 4>(sbase + BC::OFF_SP, jr, K::SBO_K, 4 * g, K::SPT_SZ, sv);
-        st_piece<NTG, 4>(sbase + BC::OFF_GT, jr, K::SBO_K, 4 * g, K::SPT_SZ, gv);
-      }
-      // sum over the 8 rows of this lane group (lanes i..i+7 share the channel group)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        bp[e] += __shfl_xor_sync(0xffffffffu, bp[e], 1);
-        bp[e] += __shfl_xor_sync(0xffffffffu, bp[e], 2);
-        bp[e] += __shfl_xor_sync(0xffffffffu, bp[e], 4);
-      }
-      if (in && (i & 7) == 0) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) atomicAdd(&bnd[4 * g + e], bp[e]);
       }
     }
     {  // zero padding: key channels DK..DKP of every row; value rows DV..DVP of S' and Gt
@@ -509,10 +525,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
     tc_fence_before();
     __syncthreads();
     // ---- the next unit's row pieces start to arrive; dq, dk (and dv) rows as coalesced pieces
-    if (PRE && has_next) {
-      issue_qk(un, rows_next);
-      issue_s(un);
-    }
+    if (PRE && has_next) issue_qk(un, rows_next);
     constexpr int KPB = PSK * (int)sizeof(TOUT), VPB = 8 * (int)sizeof(TOUT);
 #pragma unroll
     for (int j = 0; j < K::NPK; ++j) {
@@ -559,7 +572,9 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
       sh.segtot[sg][sc] = acc;
     }
     if (tid < 64) sh.bnd[(it + 1) & 1][tid] = 0.f;  // the next unit's accumulator
+    fence_async_smem();  // the staging reads precede the next unit's bulk copies into the same slots
     __syncthreads();
+    if (tid == 0 && has_next) issue_states(un);  // they land while d log alpha is finished
     if (sg < BC::NSG) {
       float post = bnd[sc];
       for (int s2 = sg + 1; s2 < BC::NSG; ++s2) post += sh.segtot[s2][sc];
