@@ -95,9 +95,9 @@ struct GradSmem {
 };
 
 // Masks one C x C product in TMEM (lane = row r; keep column c >= r when
-// `upper`, else c <= r) and rewrites it as two bf16 terms in place, 16 columns
-// (one K-step) at a time.  This thread covers the columns of its half; all of
-// its loads are issued before the one wait.
+// `upper`, else c <= r) and rewrites it as two bf16 terms in place, one K-step
+// of 16 columns at a time.  This thread covers the columns of its half.  (One
+// wait per 16-column load measured faster than waiting once for all of them.)
 template <int C, int PT_STRIDE>
 __device__ __forceinline__ void mask_to_terms(uint32_t tmem, uint32_t region, bool upper) {
   const int tid = threadIdx.x, t = tid & 127, wq = t >> 5, half = tid >> 7;
@@ -524,7 +524,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
     }
     tc_fence_before();
     __syncthreads();
-    // ---- the next unit's row pieces start to arrive; dq, dk (and dv) rows as coalesced pieces
+    // ---- the next unit's q, k and EQ pieces start to arrive; dq, dk (and dv) rows as coalesced pieces
     if (PRE && has_next) issue_qk(un, rows_next);
     constexpr int KPB = PSK * (int)sizeof(TOUT), VPB = 8 * (int)sizeof(TOUT);
 #pragma unroll
