@@ -61,7 +61,7 @@ def algorithmic_bytes(w):
 
 # This library's kernels per op, in launch order, and the sources they are built from.
 OP_KERNELS = {
-    "fwd": ["gla_chunk_state_kernel", "gla_state_scan_kernel", "gla_chunk_out_kernel"],
+    "fwd": ["gla_gate_kernel", "gla_chunk_state_kernel", "gla_state_scan_kernel", "gla_chunk_out_kernel"],
     "bwd": ["gla_chunk_dh_kernel", "gla_state_scan_kernel", "gla_chunk_grad_kernel"],
     "conv": ["srem_dwconv_kernel"],
 }

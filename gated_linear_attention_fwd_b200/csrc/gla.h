@@ -54,10 +54,10 @@ struct WsLayout {
 WsLayout ws_layout(int B, int H, int gate_heads, int L, int nchunks, int dk, int dv, bool backward);
 
 // Launch helpers; return cudaSuccess or the launch error.  The forward enqueues
-// its three kernels (chunk states, state scan, outputs); the backward its three
-// (chunk states and state gradients, the forward and reverse scans, gradients),
-// or with `saved` (gEQ, gCH and dsn from the forward) only the state gradients,
-// their reverse scan and the gradients.
+// its four kernels (gate factors, chunk states, state scan, outputs); the
+// backward its four (gate factors, chunk states and state gradients, the
+// forward and reverse scans, gradients), or with `saved` (gEQ, gCH and dsn from
+// the forward) only the state gradients, their reverse scan and the gradients.
 cudaError_t launch_gla_fwd(const GlaVariant& var, const GlaArgs& a, cudaStream_t s);
 cudaError_t launch_gla_bwd(const GlaVariant& var, const GlaArgs& a, bool saved, cudaStream_t s);
 bool gla_variant_built(int dk, int dv);

@@ -15,8 +15,8 @@
 // the state leaving the chunk by e^delta is the same as shifting every later
 // log-decay cumsum by delta (natural-log units throughout).
 //
-// Kernels: the forward's chunk-state kernel in backward mode (dS_n and dH_n per
-// chunk), the state scan forward over dS (entry states S_n) and in reverse over
+// Kernels: the forward's gate kernel and its chunk-state kernel in backward mode
+// (dS_n and dH_n per chunk), the state scan forward over dS (entry states S_n) and in reverse over
 // dH (exit gradients G_n), then gla_chunk_grad_kernel over independent
 // (sequence, chunk) units.  P^T, dP^T and dP are formed by separate tensor-core
 // products so none needs a transpose.  They take turns in one TMEM region: each

@@ -1,7 +1,8 @@
 // gla_chunk.cuh -- pieces shared by the chunk-parallel GLA kernels (forward
-// and backward): operand layouts, the unit decomposition, row loads, and the
-// chunk-state kernel (gate cumsum, per-chunk state contribution, and for the
-// backward the per-chunk state-gradient contribution).
+// and backward): operand layouts, the unit decomposition, row loads, the gate
+// kernel (per gate head and chunk: the cumsum of the log decays as gate
+// factors) and the chunk-state kernel (per-chunk state contribution, and for
+// the backward the per-chunk state-gradient contribution).
 //
 // A unit is one chunk of C consecutive scan positions of one (batch, head)
 // sequence.  Units are independent: kernels loop over them persistently and
@@ -61,27 +62,23 @@ struct StateCfg {
   static constexpr int OFF_VR = OFF_QB + (BWD ? K::NTG * K::AQ_SZ : 0);
   static constexpr int OFF_DO = OFF_VR + K::NTV * K::VR_SZ;  // BWD: dO
   static constexpr int END_ROWS = OFF_DO + (BWD ? K::NTV * K::VR_SZ : 0);
-  static constexpr int GP = DK + 4;                 // row pitch (floats) of the cumsum buffer
-  static constexpr int OFF_G = cround(END_ROWS, 16);
   static constexpr int SDP = DK + 4;                // row pitch of the dS / dH staging rows
-  static constexpr int OFF_SD = OFF_G + C * GP * 4;
+  static constexpr int OFF_SD = cround(END_ROWS, 16);
   // the M = 128 reads of v^T / dO^T may run past their rows into the next
   // buffers (those lanes are unused); they only have to stay inside the allocation
   static constexpr int SMEM = cmax(cmax(OFF_SD + (BWD ? 2 : 1) * DV * SDP * 4, OFF_VR + K::VR_READ),
                                    BWD ? OFF_DO + K::VR_READ : 0);
-  static constexpr int NSG = 256 / DK;              // token segments of the cumsum
-  static constexpr int SEGL = cdiv(C, NSG);
   static constexpr int TM_DH = K::DKP;              // BWD: dH columns after dS
   static constexpr int TM_COLS = pow2ceil((BWD ? 2 : 1) * K::DKP);
-  static constexpr int PER_SM = SMEM <= 72 * 1024 ? 3 : SMEM <= 110 * 1024 ? 2 : 1;  // resident CTAs per SM
+  // resident CTAs per SM: by shared memory, and by registers (the forward kernel
+  // with d_k > 32 holds more row pieces than three CTAs' registers allow)
+  static constexpr int MINB = BWD ? 2 : (DK <= 32 ? 3 : 2);
+  static constexpr int PER_SM = cmax(1, SMEM <= 72 * 1024 ? cmin(3, MINB) : SMEM <= 110 * 1024 ? cmin(2, MINB) : 1);
   static_assert(SMEM <= 225 * 1024, "shared-memory budget");
-  static_assert(NSG <= 8, "cumsum segments");
 };
 
 struct StateSmem {
   long long rows[2][128];  // grid tokens of the units whose loads are in flight (by unit parity)
-  float segtot[8][64];  // cumsum totals of the token segments
-  float gam[64];        // chunk decay Gamma (log2)
   uint64_t bar;
   uint32_t tmem;
 };
@@ -191,15 +188,109 @@ __device__ __forceinline__ void stage_rows_dk(uint32_t tmem, int col0, float* sd
   }
 }
 
-// Per unit: the gate of the chunk (inclusive cumsum b of the base-2 log decays
-// over its tokens, per key channel), stored once per gate head as the factors
-// EQ = 2^(b - r) and the chunk constants {2^r, 2^(Gamma - r), 2^Gamma, Gamma};
-// and the chunk's state contribution dS = khat^T v with khat = k 2^(Gamma - b)
-// (value-major rows, to `dsn`).  With BWD it also forms the chunk's
-// state-gradient contribution dH = (q 2^b)^T dO (to `dhn`), which the reverse
+// ============================================================== gate
+// Per (gate head, chunk): the inclusive cumsum b of the base-2 log decays over
+// the chunk's tokens, per key channel, stored as the factors EQ = 2^(b - r)
+// (r = b at the chunk's middle token) and the chunk constants {2^r,
+// 2^(Gamma - r), 2^Gamma, Gamma}.  Computed once; every head that shares the
+// gate reads them.  Tokens past the sequence end do not decay.  A factor
+// outside 2^+-115 sets DIG_ERR_GATE_RANGE.
+template <int C, int DK>
+__global__ void __launch_bounds__(256) gla_gate_kernel(const GlaArgs a) {
+  constexpr int GP = DK + 4;     // row pitch (floats) of the cumsum buffer
+  constexpr int NSG = 256 / DK;  // token segments of the cumsum
+  constexpr int SEGL = cdiv(C, NSG);
+  constexpr int NG = DK / 4;     // 4-channel groups of a token row
+  static_assert(NSG <= 8 && DK <= 64, "cumsum segments");
+  __shared__ __align__(16) float G[C * GP];
+  __shared__ float segtot[8][64];
+  __shared__ float gam[64];
+  __shared__ long long grows[C];
+  griddep_wait();  // the kernels before this one have completed
+  griddep_launch_dependents();
+  const int tid = threadIdx.x;
+  const int nunits = a.B * a.gate_heads * a.nchunks;
+  bool bad = false;
+  for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+    const int bz = u / a.nchunks, n = u - bz * a.nchunks;
+    const int b = bz / a.gate_heads, hz = bz - b * a.gate_heads;
+    if (tid < C) {
+      const int p = n * C + tid;
+      grows[tid] = p < a.L ? (long long)b * a.L + scan_to_grid(p, a.L, a.Hg, a.Wg, a.mode) : -1;
+    }
+    __syncthreads();
+    // ---- base-2 log decays of the chunk's tokens (consecutive threads: consecutive channel groups of a token)
+    for (int i = tid; i < C * NG; i += 256) {
+      const int t = i / NG, g = i - t * NG;
+      const long long gr = grows[t];
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);  // padding tokens do not decay
+      if (gr >= 0) {
+        const float4 zz = __ldg(reinterpret_cast<const float4*>(a.z + ((size_t)gr * a.gate_heads + hz) * DK) + g);
+        x = make_float4(log2_decay(zz.x, a.inv_tau), log2_decay(zz.y, a.inv_tau), log2_decay(zz.z, a.inv_tau),
+                        log2_decay(zz.w, a.inv_tau));
+      }
+      *reinterpret_cast<float4*>(G + t * GP + 4 * g) = x;
+    }
+    __syncthreads();
+    // ---- inclusive cumsum over the tokens, per key channel: token segments, then their prefixes
+    const int sc = tid % DK, sg = tid / DK;
+    const int t0 = sg * SEGL, t1 = min(C, t0 + SEGL);
+    if (sg < NSG) {
+      float acc = 0.f;
+      for (int t = t0; t < t1; ++t) {
+        acc += G[t * GP + sc];
+        G[t * GP + sc] = acc;
+      }
+      segtot[sg][sc] = acc;
+    }
+    __syncthreads();
+    if (sg < NSG) {
+      float pre = 0.f, tot = 0.f;
+      for (int s2 = 0; s2 < NSG; ++s2) {
+        const float x = segtot[s2][sc];
+        pre += s2 < sg ? x : 0.f;
+        tot += x;
+      }
+      if (sg > 0)
+        for (int t = t0; t < t1; ++t) G[t * GP + sc] += pre;
+      if (sg == 0) gam[sc] = tot;
+    }
+    __syncthreads();
+    // ---- gate factors and chunk constants
+    const float* Gr = G + (C / 2 - 1) * GP;  // b at the reference token
+    for (int i = tid; i < C * NG; i += 256) {
+      const int t = i / NG, g = i - t * NG;
+      const int p = n * C + t;
+      if (p < a.L) {
+        const float4 bt = *reinterpret_cast<const float4*>(G + t * GP + 4 * g);
+        const float4 rr = *reinterpret_cast<const float4*>(Gr + 4 * g);
+        const float d0 = bt.x - rr.x, d1 = bt.y - rr.y, d2 = bt.z - rr.z, d3 = bt.w - rr.w;
+        bad |= fmaxf(fmaxf(fabsf(d0), fabsf(d1)), fmaxf(fabsf(d2), fabsf(d3))) > 115.f;
+        *reinterpret_cast<float4*>(a.gEQ + ((size_t)bz * a.L + p) * DK + 4 * g) =
+            make_float4(ex2(d0), ex2(d1), ex2(d2), ex2(d3));
+      }
+    }
+    if (tid < DK) {
+      float* ch = a.gCH + ((size_t)bz * a.nchunks + n) * 4 * DK + tid;
+      const float r = Gr[tid], gm = gam[tid];
+      ch[0 * DK] = exp2f(r);
+      ch[1 * DK] = exp2f(gm - r);
+      ch[2 * DK] = exp2f(gm);
+      ch[3 * DK] = gm;
+    }
+    __syncthreads();  // the cumsum buffer, token table and segment totals are reused by the next unit
+  }
+  if (bad) set_status(a.status, DIG_ERR_GATE_RANGE);
+}
+
+// ============================================================== chunk state
+// Per unit: the chunk's state contribution dS = khat^T v with khat =
+// k 2^(Gamma - b) = k 2^(Gamma - r) / EQ (value-major rows, to `dsn`), from the
+// gate kernel's factors.  With BWD it also forms the chunk's state-gradient
+// contribution dH = (q 2^b)^T dO, q 2^b = q EQ 2^r (to `dhn`), which the reverse
 // scan turns into the gradient of every chunk's exit state.
 template <int C, int DK, int DV, typename TIN, bool BWD>
-__global__ void __launch_bounds__(256, BWD ? 2 : 3) gla_chunk_state_kernel(const GlaArgs a) {
+__global__ void __launch_bounds__(256, StateCfg<C, DK, DV, TIN, BWD>::MINB) gla_chunk_state_kernel(const GlaArgs a) {
   using Cfg = ChunkCfg<C, DK, DV, TIN>;
   using SC = StateCfg<C, DK, DV, TIN, BWD>;
   constexpr int NTG = Cfg::NTG, NTV = Cfg::NTV, DKP = Cfg::DKP, PSK = Cfg::PSK;
@@ -222,7 +313,6 @@ __global__ void __launch_bounds__(256, BWD ? 2 : 3) gla_chunk_state_kernel(const
   griddep_launch_dependents();
   const uint32_t tmem = sh.tmem;
   const uint32_t sbase = smem_u32(smem);
-  float* G = reinterpret_cast<float*>(smem + SC::OFF_G);    // [C][GP] cumsum of log2 decays
   float* SD = reinterpret_cast<float*>(smem + SC::OFF_SD);  // [DV][SDP] dS staging, then dH
   const uint64_t dVRm = sdesc(sbase + SC::OFF_VR, Cfg::SBO_V, 128);
   const uint64_t dKHm = sdesc(sbase + SC::OFF_KH, Cfg::SBO_K, 128);
@@ -230,33 +320,34 @@ __global__ void __launch_bounds__(256, BWD ? 2 : 3) gla_chunk_state_kernel(const
   const uint64_t dQBm = sdesc(sbase + SC::OFF_QB, Cfg::SBO_K, 128);
   const int nunits = a.B * a.H * a.nchunks;
   uint32_t ph = 0;
-  bool timed_out = false, bad = false;
+  bool timed_out = false;
 
-  // Row pieces of a unit, loaded one unit ahead: gate logits, k (and q) are
-  // issued once the current unit's operands are written, v (and dO) once its
-  // products have completed.
-  Piece<float, 4> pz[Cfg::NPZ];
+  // Row pieces of a unit, loaded one unit ahead: gate factors EQ = 2^(b - r),
+  // the chunk constants and k (and q) are issued once the current unit's
+  // operands are written, v (and dO) once its products have completed.
+  // all of a thread's pieces share one channel group when the groups divide 32
+  // (piece_of), and then one load of the chunk constants serves them all
+  constexpr int NPC = 32 % Cfg::NGK == 0 ? 1 : Cfg::NPK;
+  Piece<float, PSK> pe[Cfg::NPK], pc[NPC], pc0[BWD ? NPC : 1];
   Piece<TIN, PSK> pk[Cfg::NPK], pq[BWD ? Cfg::NPK : 1];
   auto issue_rows = [&](int u, const long long* rows) {
     const Unit U(a, u);
-    const int hz = U.bz - U.b * a.gate_heads;
-#pragma unroll
-    for (int j = 0; j < Cfg::NPZ; ++j) {
-      const int i = tid + 256 * j;
-      int t, g;
-      piece_of<Cfg::NGZ>(i, t, g);
-      const long long gr = i < C * Cfg::NGZ ? rows[t] : -1;
-      pz[j].load(a.z + ((size_t)(gr >= 0 ? gr : 0) * a.gate_heads + hz) * DK + 4 * g, gr >= 0);
-    }
 #pragma unroll
     for (int j = 0; j < Cfg::NPK; ++j) {
       const int i = tid + 256 * j;
       int t, g;
       piece_of<Cfg::NGK>(i, t, g);
       const long long gr = i < C * Cfg::NGK ? rows[t] : -1;
+      const bool valid = gr >= 0;
       const size_t off = tok_row(gr, a, U.h) * DK + g * PSK;
-      pk[j].load(reinterpret_cast<const TIN*>(a.k) + off, gr >= 0);
-      if constexpr (BWD) pq[j].load(reinterpret_cast<const TIN*>(a.q) + off, gr >= 0);
+      pk[j].load(reinterpret_cast<const TIN*>(a.k) + off, valid);
+      if constexpr (BWD) pq[j].load(reinterpret_cast<const TIN*>(a.q) + off, valid);
+      pe[j].load(a.gEQ + ((size_t)U.bz * a.L + (valid ? U.n * C + t : 0)) * DK + g * PSK, valid);
+      if (j < NPC) {
+        const float* ch = a.gCH + ((size_t)U.bz * a.nchunks + U.n) * 4 * DK + g * PSK;
+        pc[j].load(ch + DK, i < C * Cfg::NGK);  // 2^(Gamma - r)
+        if constexpr (BWD) pc0[j].load(ch, i < C * Cfg::NGK);  // 2^r
+      }
     }
   };
   auto issue_vd = [&](int u, const long long* rows) {
@@ -272,95 +363,31 @@ __global__ void __launch_bounds__(256, BWD ? 2 : 3) gla_chunk_state_kernel(const
   int it = 0;
   for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
     const Unit U(a, u);
-    const bool writer = a.gate_heads != 1 || U.h == 0;  // one unit per gate head stores the factors
     const int un = u + gridDim.x;
     const bool has_next = un < nunits;
     long long* rows_next = sh.rows[(it + 1) & 1];
-    if (has_next) fill_rows(a, un, C, rows_next);  // read after this unit's next barrier
-    // ---- inclusive cumsum over the chunk's tokens, per key channel (shared memory)
-#pragma unroll
-    for (int j = 0; j < Cfg::NPZ; ++j) {
-      const int i = tid + 256 * j;
-      int t, g;
-      piece_of<Cfg::NGZ>(i, t, g);
-      if (i < C * Cfg::NGZ) {
-        const int p = U.n * C + t;
-        float zz[4];
-        pz[j].unpack(zz);
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);  // padding tokens do not decay
-        if (p < a.L)
-          x = make_float4(log2_decay(zz[0], a.inv_tau), log2_decay(zz[1], a.inv_tau), log2_decay(zz[2], a.inv_tau),
-                          log2_decay(zz[3], a.inv_tau));
-        *reinterpret_cast<float4*>(G + t * SC::GP + 4 * g) = x;
-      }
-    }
-    __syncthreads();
-    const int sc = tid % DK, sg = tid / DK;
-    const int t0 = sg * SC::SEGL, t1 = min(C, t0 + SC::SEGL);
-    if (sg < SC::NSG) {
-      float acc = 0.f;
-      for (int t = t0; t < t1; ++t) {
-        acc += G[t * SC::GP + sc];
-        G[t * SC::GP + sc] = acc;
-      }
-      sh.segtot[sg][sc] = acc;
-    }
-    __syncthreads();
-    if (sg < SC::NSG) {
-      float pre = 0.f, tot = 0.f;
-      for (int s2 = 0; s2 < SC::NSG; ++s2) {
-        const float x = sh.segtot[s2][sc];
-        pre += s2 < sg ? x : 0.f;
-        tot += x;
-      }
-      if (sg > 0)
-        for (int t = t0; t < t1; ++t) G[t * SC::GP + sc] += pre;
-      if (sg == 0) sh.gam[sc] = tot;
-    }
-    __syncthreads();
-    const float* Gr = G + (C / 2 - 1) * SC::GP;  // b at the reference token
-    // ---- gate factors (one writer per gate head)
-#pragma unroll
-    for (int j = 0; j < Cfg::NPZ; ++j) {
-      const int i = tid + 256 * j;
-      int t, g;
-      piece_of<Cfg::NGZ>(i, t, g);
-      const int p = U.n * C + t;
-      if (i < C * Cfg::NGZ && p < a.L) {
-        const float4 bt = *reinterpret_cast<const float4*>(G + t * SC::GP + 4 * g);
-        const float4 rr = *reinterpret_cast<const float4*>(Gr + 4 * g);
-        const float d0 = bt.x - rr.x, d1 = bt.y - rr.y, d2 = bt.z - rr.z, d3 = bt.w - rr.w;
-        bad |= fmaxf(fmaxf(fabsf(d0), fabsf(d1)), fmaxf(fabsf(d2), fabsf(d3))) > 115.f;
-        if (writer)
-          *reinterpret_cast<float4*>(a.gEQ + ((size_t)U.bz * a.L + p) * DK + 4 * g) =
-              make_float4(ex2(d0), ex2(d1), ex2(d2), ex2(d3));
-      }
-    }
-    if (writer && tid < DK) {
-      float* ch = a.gCH + ((size_t)U.bz * a.nchunks + U.n) * 4 * DK + tid;
-      const float r = Gr[tid], gm = sh.gam[tid];
-      ch[0 * DK] = exp2f(r);
-      ch[1 * DK] = exp2f(gm - r);
-      ch[2 * DK] = exp2f(gm);
-      ch[3 * DK] = gm;
-    }
-    // ---- khat = k 2^(Gamma - b)   (BWD: and q 2^b)
+    if (has_next) fill_rows(a, un, C, rows_next);  // read after the barrier before this unit's products
+    // ---- khat = k 2^(Gamma - b) = k 2^(Gamma - r) / EQ   (BWD: and q 2^b = q EQ 2^r)
 #pragma unroll
     for (int j = 0; j < Cfg::NPK; ++j) {
       const int i = tid + 256 * j;
       int t, g;
       piece_of<Cfg::NGK>(i, t, g);
       if (i < C * Cfg::NGK) {
-        float kv[PSK];
+        const bool valid = U.n * C + t < a.L;  // padding tokens hold zeros
+        float kv[PSK], ev[PSK], cv[PSK];
         pk[j].unpack(kv);
+        pe[j].unpack(ev);
+        pc[NPC == 1 ? 0 : j].unpack(cv);
 #pragma unroll
-        for (int e = 0; e < PSK; ++e) kv[e] *= ex2(sh.gam[g * PSK + e] - G[t * SC::GP + g * PSK + e]);
+        for (int e = 0; e < PSK; ++e) kv[e] *= valid ? __fdividef(cv[e], ev[e]) : 0.f;
         st_piece<NTG, PSK>(sbase + SC::OFF_KH, t, Cfg::SBO_K, g * PSK, Cfg::AQ_SZ, kv);
         if constexpr (BWD) {
-          float qv[PSK];
+          float qv[PSK], c0[PSK];
           pq[j].unpack(qv);
+          pc0[NPC == 1 ? 0 : j].unpack(c0);
 #pragma unroll
-          for (int e = 0; e < PSK; ++e) qv[e] *= ex2(G[t * SC::GP + g * PSK + e]);
+          for (int e = 0; e < PSK; ++e) qv[e] *= valid ? ev[e] * c0[e] : 0.f;
           st_piece<NTG, PSK>(sbase + SC::OFF_QB, t, Cfg::SBO_K, g * PSK, Cfg::AQ_SZ, qv);
         }
       }
@@ -373,13 +400,15 @@ __global__ void __launch_bounds__(256, BWD ? 2 : 3) gla_chunk_state_kernel(const
           st_piece<NTG, 4>(sbase + SC::OFF_QB, i / Cfg::NPAD, Cfg::SBO_K, DK + 4 * (i % Cfg::NPAD), Cfg::AQ_SZ, zz);
       }
     }
-    if (has_next) issue_rows(un, rows_next);  // this unit's row pieces are consumed
     cp_async_wait_all();
     // ---- dS = v^T khat, dH = dO^T (q 2^b)  (M = value channels, N = key channels, K = tokens)
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // this unit's row pieces are consumed, and the next unit's row table (filled
+    // at the top of this iteration) is visible after the barrier above
+    if (has_next) issue_rows(un, rows_next);
     if (tid == 0) {
       mma_issue<NTV, NTG, C / 16>(tmem, dVRm, Cfg::VR_SZ, 2 * Cfg::SBO_V, dKHm, Cfg::AQ_SZ, 2 * Cfg::SBO_K,
                                   idesc_bf16(128, DKP, true, true), false);
@@ -417,7 +446,6 @@ __global__ void __launch_bounds__(256, BWD ? 2 : 3) gla_chunk_state_kernel(const
     }
     __syncthreads();  // operands, staging and the cumsum buffer are reused by the next unit
   }
-  if (bad) set_status(a.status, DIG_ERR_GATE_RANGE);
   if (timed_out) set_status(a.status, DIG_ERR_DEVICE_TIMEOUT);
   tc_fence_before();
   __syncthreads();
@@ -458,15 +486,17 @@ inline int persistent_grid(int per_sm, long long units) {
   return (int)(units < slots ? units : slots);
 }
 
-// Chunk-state kernel launch (sets its shared-memory limit first).
+// Gate kernel, then chunk-state kernel (which reads the gate factors).
 template <int C, int DK, int DV, typename TIN, bool BWD>
 cudaError_t launch_chunk_state(const GlaArgs& a, cudaStream_t s) {
   using SC = StateCfg<C, DK, DV, TIN, BWD>;
   const long long units = (long long)a.B * a.H * a.nchunks;
   if (units <= 0) return cudaSuccess;
-  auto k1 = gla_chunk_state_kernel<C, DK, DV, TIN, BWD>;
-  cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, SC::SMEM);
+  const long long gunits = (long long)a.B * a.gate_heads * a.nchunks;
+  cudaError_t e = launch_pdl(gla_gate_kernel<C, DK>, dim3(persistent_grid(4, gunits)), dim3(256), 0, s, a);
   if (e != cudaSuccess) return e;
+  auto k1 = gla_chunk_state_kernel<C, DK, DV, TIN, BWD>;
+  if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, SC::SMEM)) != cudaSuccess) return e;
   return launch_pdl(k1, persistent_grid(SC::PER_SM, units), 256, SC::SMEM, s, a);
 }
 

@@ -12,6 +12,7 @@ namespace dig {
 
 __host__ __device__ constexpr int cround(int x, int m) { return (x + m - 1) / m * m; }
 __host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
+__host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 __host__ __device__ constexpr int pow2ceil(int x) {
   int p = 32;
   while (p < x) p <<= 1;

@@ -14,16 +14,17 @@
 //     S_{n+1} = diag(2^Gamma) S_n + khat^T V
 // which equals the recurrence in exact arithmetic.
 //
-// Three kernels, each over independent (sequence, chunk) units (the first two
-// are shared with the backward, gla_chunk.cuh):
-//   1. gla_chunk_state_kernel: the gate of the chunk (cumsum over its tokens),
-//      written once per gate head as per-token factors 2^(b - r) and per-chunk
-//      constants; and the chunk's state contribution dS_n = khat^T V.
-//   2. gla_state_scan_kernel: S_{n+1} = diag(2^Gamma_n) S_n + dS_n over the
+// Four kernels, each over independent units (the first three are shared with
+// the backward, gla_chunk.cuh):
+//   1. gla_gate_kernel: per (gate head, chunk), the gate of the chunk (cumsum
+//      over its tokens) as per-token factors 2^(b - r) and per-chunk constants.
+//   2. gla_chunk_state_kernel: per (sequence, chunk), the chunk's state
+//      contribution dS_n = khat^T V.
+//   3. gla_state_scan_kernel: S_{n+1} = diag(2^Gamma_n) S_n + dS_n over the
 //      chunks, an associative scan (sixteen chunk ranges per state element,
 //      then a carry fold), overwriting dS_n with the entry state S_n.
-//   3. gla_chunk_out_kernel: the outputs of every chunk from its entry state,
-//      and the fused Swish(r) * RMSNorm(o) epilogue.
+//   4. gla_chunk_out_kernel: per (sequence, chunk), the outputs from the
+//      chunk's entry state, and the fused Swish(r) * RMSNorm(o) epilogue.
 // No unit waits on another, so several CTAs share an SM and hide each other's
 // memory latency; there is no inter-CTA signalling.
 //
