@@ -16,7 +16,6 @@
  *   - SREM: slide "SREM (Spatial Reorient & Enhancement Module) の導入": a 3x3
  *     depthwise conv on the 2-D token grid followed by a transpose / flip of the
  *     scan order.
- * Every reading of a garbled or silent passage is listed in the design doc.
  *
  * Layouts (all fp64, row-major, tokens in grid row-major order g = row*Wg + col):
  *   q, k        [B][L][H][dk]
