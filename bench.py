@@ -37,6 +37,15 @@ WORKLOAD_INDEX = 3  # DiG-S/2 at 1792^2: the configuration that carries every ho
 L2_FLUSH_BYTES = 512 << 20
 
 
+def max_over_ranks(value, world, device):
+    """The largest of `value` over the ranks: the time of the slowest replica."""
+    if world <= 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -259,11 +268,7 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(3)] for i in range(args.steps)])  # ms
-    step_ms = float(per.sum(axis=1).mean())
-    if world > 1:
-        tt = torch.tensor([step_ms], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        step_ms = float(tt.item())
+    step_ms = max_over_ranks(float(per.sum(axis=1).mean()), world, dev)
     for ws in (ws_f, ws_b):
         st = dig.dig_read_status(ws)
         if st != dig.DIG_OK:
@@ -315,11 +320,7 @@ def run_ours(args, rank, world, local_rank):
     e2e_run(e2e_steps, 2)
     e1.record(s_d2h)
     e1.synchronize()
-    e2e_step_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        tt = torch.tensor([e2e_step_ms], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        e2e_step_ms = float(tt.item())
+    e2e_step_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
 
     if rank != 0:
         return None
