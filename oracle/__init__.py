@@ -17,6 +17,10 @@ Parity status of each function (what pins it is in tests/test_oracle_pins.py):
                  permutation, all-ones kernel on a constant grid (9/6/4)
   epilogue       pinned: unit RMS of the normalised row, Swish(0) = 0,
                  positive scale invariance
+  epilogue_bwd   pinned: central finite differences of sum(dy * epilogue) in o, r
+                 and gamma; d_o orthogonal to o when eps = 0 (scale invariance)
+  srem_dwconv_bwd pinned: adjoint identity <conv(x), dy> = <x, dx>; dw and dbias
+                 from the forward conv with one-tap kernels / zero kernel
   scan_index     pinned: bijection, inverse restores the grid, transpose on
                  square grids, a hand-derived 3x4 fixture
 """
@@ -49,6 +53,10 @@ def _load():
                                        dp, dp, dp, dp, L, L, L, L, L, L, L, ctypes.c_int]
         lib.oracle_epilogue.restype = ctypes.c_int
         lib.oracle_epilogue.argtypes = [dp, dp, dp, ctypes.c_double, dp, L, L]
+        lib.oracle_epilogue_bwd.restype = ctypes.c_int
+        lib.oracle_epilogue_bwd.argtypes = [dp, dp, dp, ctypes.c_double, dp, dp, dp, dp, L, L]
+        lib.oracle_srem_dwconv_bwd.restype = ctypes.c_int
+        lib.oracle_srem_dwconv_bwd.argtypes = [dp, dp, dp, dp, dp, dp, L, L, L, L, ctypes.c_int]
         lib.oracle_srem_dwconv.restype = ctypes.c_int
         lib.oracle_srem_dwconv.argtypes = [dp, dp, dp, dp, L, L, L, L, ctypes.c_int]
         _lib = lib
@@ -128,6 +136,36 @@ def epilogue(o, r, gamma=None, eps=1e-5):
     if rc:
         raise ValueError("oracle_epilogue rejected the arguments")
     return y
+
+
+def epilogue_bwd(o, r, dy, gamma=None, eps=1e-5):
+    """Gradients (d_o, d_r, d_gamma) of sum(dy * epilogue(o, r, gamma, eps))."""
+    o, r, dy = _f64(o), _f64(r), _f64(dy)
+    dv = o.shape[-1]
+    rows = o.size // dv if dv else 0
+    g = None if gamma is None else _f64(gamma)
+    d_o, d_r = np.zeros_like(o), np.zeros_like(o)
+    d_gamma = np.zeros(dv, dtype=np.float64)
+    rc = _load().oracle_epilogue_bwd(_ptr(o), _ptr(r), _ptr(g), float(eps), _ptr(dy), _ptr(d_o), _ptr(d_r),
+                                     _ptr(d_gamma), rows, dv)
+    if rc:
+        raise ValueError("oracle_epilogue_bwd rejected the arguments")
+    return d_o, d_r, d_gamma
+
+
+def srem_dwconv_bwd(x, w, dy, mode):
+    """Gradients (dx [B,Hg,Wg,C] grid order, dw [C,3,3], dbias [C]) of sum(dy * srem_dwconv(x, w, bias, mode))
+    for dy [B,L,C] in scan order."""
+    x, w, dy = _f64(x), _f64(w), _f64(dy)
+    B, Hg, Wg, C = x.shape
+    dx = np.zeros_like(x)
+    dw = np.zeros((C, 3, 3), dtype=np.float64)
+    db = np.zeros(C, dtype=np.float64)
+    rc = _load().oracle_srem_dwconv_bwd(_ptr(x), _ptr(w), _ptr(dy), _ptr(dx), _ptr(dw), _ptr(db),
+                                        B, Hg, Wg, C, int(mode))
+    if rc:
+        raise ValueError("oracle_srem_dwconv_bwd rejected the arguments (rc=%d)" % rc)
+    return dx, dw, db
 
 
 def srem_dwconv(x, w, bias, mode):

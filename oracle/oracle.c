@@ -257,6 +257,53 @@ int oracle_epilogue(const double *o, const double *r, const double *gamma, doubl
     return 0;
 }
 
+/* Backward of the epilogue above (same slide, eq. (9)-(10)), by the chain rule.
+ * Per row, with s_j = Swish(r_j) = r_j sigmoid(r_j), inv = 1/sqrt(mean(o^2) + eps)
+ * and y_j = s_j o_j inv gamma_j:
+ *   dy_j/do_m    = s_j gamma_j (delta_jm inv + o_j dinv/do_m),  dinv/do_m = -inv^3 o_m / dv
+ *   dy_j/dr_j    = o_j inv gamma_j Swish'(r_j),  Swish'(x) = sigmoid(x) (1 + x (1 - sigmoid(x)))
+ *   dy_j/dgamma_j = s_j o_j inv
+ * d_o, d_r are per row; d_gamma sums over rows (NULL skips it). */
+int oracle_epilogue_bwd(const double *o, const double *r, const double *gamma, double eps,
+                        const double *dy, double *d_o, double *d_r, double *d_gamma,
+                        long rows, long dv)
+{
+    if (rows < 0 || dv <= 0) return 1;
+#pragma omp parallel for schedule(static)
+    for (long i = 0; i < rows; ++i) {
+        const double *oi = o + i * dv, *ri = r + i * dv, *gi = dy + i * dv;
+        double ms = 0.0;
+        for (long j = 0; j < dv; ++j) ms += oi[j] * oi[j];
+        double inv = 1.0 / sqrt(ms / (double)dv + eps);
+        double dinv_sum = 0.0;  /* sum_j dy_j s_j gamma_j o_j: the weight of dinv/do_m */
+        for (long j = 0; j < dv; ++j) {
+            double sig = 1.0 / (1.0 + exp(-ri[j]));
+            double gm = gamma ? gamma[j] : 1.0;
+            dinv_sum += gi[j] * ri[j] * sig * gm * oi[j];
+        }
+        for (long m = 0; m < dv; ++m) {
+            double sig = 1.0 / (1.0 + exp(-ri[m]));
+            double gm = gamma ? gamma[m] : 1.0;
+            double direct = gi[m] * ri[m] * sig * gm * inv;
+            double through_inv = dinv_sum * (-inv * inv * inv * oi[m] / (double)dv);
+            d_o[i * dv + m] = direct + through_inv;
+            d_r[i * dv + m] = gi[m] * oi[m] * inv * gm * sig * (1.0 + ri[m] * (1.0 - sig));
+        }
+    }
+    if (d_gamma) {
+        for (long j = 0; j < dv; ++j) d_gamma[j] = 0.0;
+        for (long i = 0; i < rows; ++i) {
+            const double *oi = o + i * dv, *ri = r + i * dv, *gi = dy + i * dv;
+            double ms = 0.0;
+            for (long j = 0; j < dv; ++j) ms += oi[j] * oi[j];
+            double inv = 1.0 / sqrt(ms / (double)dv + eps);
+            for (long j = 0; j < dv; ++j)
+                d_gamma[j] += gi[j] * ri[j] / (1.0 + exp(-ri[j])) * oi[j] * inv;
+        }
+    }
+    return 0;
+}
+
 /* SREM: 3x3 depthwise cross-correlation with zero "same" padding on the grid,
  * result written in scan order: y[b][t][ch] = conv(x)[b][grid(t)][ch]. */
 int oracle_srem_dwconv(const double *x, const double *w, const double *bias, double *y,
@@ -280,5 +327,63 @@ int oracle_srem_dwconv(const double *x, const double *w, const double *bias, dou
             y[(b * L + t) * C + ch] = acc;
         }
     }
+    return 0;
+}
+
+/* Backward of the SREM conv above: gradients of sum_t dy[b][t][ch] y[b][t][ch].
+ * The scan-order gradient is first put back on the grid (dyg[b][pi(t)] = dy[b][t]);
+ * then, from y_g = bias + sum_{di,dj} w[di,dj] x[g + (di,dj)],
+ *   dx[g]       = sum_{di,dj} w[di,dj] dyg[g - (di,dj)]   (terms inside the grid)
+ *   dw[di,dj]   = sum_{b,g} dyg[g] x[g + (di,dj)]            (zero outside the grid)
+ *   dbias       = sum_{b,g} dyg[g]
+ * dx is in grid order [B][Hg][Wg][C]; dw [C][3][3]; dbias [C] (NULL skips it). */
+int oracle_srem_dwconv_bwd(const double *x, const double *w, const double *dy,
+                           double *dx, double *dw, double *dbias,
+                           long B, long Hg, long Wg, long C, int mode)
+{
+    if (B < 0 || Hg < 0 || Wg < 0 || C <= 0 || mode < 0 || mode > 3) return 1;
+    long L = Hg * Wg;
+    double *dyg = (double *)malloc(sizeof(double) * (size_t)(B * L * C > 0 ? B * L * C : 1));
+    if (!dyg) return 2;
+    for (long b = 0; b < B; ++b)
+        for (long t = 0; t < L; ++t) {
+            long g = oracle_scan_index(mode, Hg, Wg, t);
+            for (long ch = 0; ch < C; ++ch) dyg[(b * L + g) * C + ch] = dy[(b * L + t) * C + ch];
+        }
+#pragma omp parallel for schedule(static)
+    for (long bg = 0; bg < B * L; ++bg) {
+        long b = bg / L, g = bg % L, r0 = g / Wg, c0 = g % Wg;
+        for (long ch = 0; ch < C; ++ch) {
+            double acc = 0.0;
+            for (long di = -1; di <= 1; ++di)
+                for (long dj = -1; dj <= 1; ++dj) {
+                    long rr = r0 - di, cc = c0 - dj;  /* output pixel that read x[g] through tap (di,dj) */
+                    if (rr < 0 || rr >= Hg || cc < 0 || cc >= Wg) continue;
+                    acc += w[ch * 9 + (di + 1) * 3 + (dj + 1)] * dyg[((b * Hg + rr) * Wg + cc) * C + ch];
+                }
+            dx[bg * C + ch] = acc;
+        }
+    }
+#pragma omp parallel for schedule(static)
+    for (long ch = 0; ch < C; ++ch) {
+        for (long tap = 0; tap < 9; ++tap) {
+            long di = tap / 3 - 1, dj = tap % 3 - 1;
+            double acc = 0.0;
+            for (long b = 0; b < B; ++b)
+                for (long rr = 0; rr < Hg; ++rr)
+                    for (long cc = 0; cc < Wg; ++cc) {
+                        long xr = rr + di, xc = cc + dj;
+                        if (xr < 0 || xr >= Hg || xc < 0 || xc >= Wg) continue;
+                        acc += dyg[((b * Hg + rr) * Wg + cc) * C + ch] * x[((b * Hg + xr) * Wg + xc) * C + ch];
+                    }
+            dw[ch * 9 + tap] = acc;
+        }
+        if (dbias) {
+            double acc = 0.0;
+            for (long bg = 0; bg < B * L; ++bg) acc += dyg[bg * C + ch];
+            dbias[ch] = acc;
+        }
+    }
+    free(dyg);
     return 0;
 }

@@ -322,3 +322,117 @@ def test_epilogue_scale_invariance_gamma_and_sign():
     # Swish(r) = r * sigmoid(r): negative r gives a small negative gate
     yn = oracle.epilogue(np.ones((1, 2)), np.array([[-1.0, 1.0]]), None, eps=0.0)
     assert np.allclose(yn, [[-1.0 / (1 + np.e), 1.0 / (1 + np.exp(-1.0))]], rtol=1e-12)
+
+
+# ----------------------------------------------------------------------------- epilogue backward
+
+def _epi_loss(o, r, gamma, dy, eps):
+    return float(np.sum(dy * oracle.epilogue(o, r, gamma, eps=eps)))
+
+
+@pytest.mark.parametrize("with_gamma", [True, False])
+def test_epilogue_bwd_matches_finite_differences(with_gamma):
+    rng = np.random.default_rng(72 + with_gamma)
+    rows, dv, eps = 3, 5, 1e-3
+    o = rng.standard_normal((rows, dv))
+    r = 2.0 * rng.standard_normal((rows, dv))
+    dy = rng.standard_normal((rows, dv))
+    gamma = rng.standard_normal(dv) if with_gamma else None
+    d_o, d_r, d_g = oracle.epilogue_bwd(o, r, dy, gamma, eps=eps)
+    h = 1e-6
+    for name, arr, grad in (("o", o, d_o), ("r", r, d_r)):
+        for idx in np.ndindex(arr.shape):
+            p, m = arr.copy(), arr.copy()
+            p[idx] += h
+            m[idx] -= h
+            args_p = (p, r) if name == "o" else (o, p)
+            args_m = (m, r) if name == "o" else (o, m)
+            fd = (_epi_loss(*args_p, gamma, dy, eps) - _epi_loss(*args_m, gamma, dy, eps)) / (2 * h)
+            assert abs(grad[idx] - fd) <= 1e-7 * max(1.0, abs(fd)), (name, idx, grad[idx], fd)
+    g0 = np.ones(dv) if gamma is None else gamma
+    for j in range(dv):
+        p, m = g0.copy(), g0.copy()
+        p[j] += h
+        m[j] -= h
+        fd = (_epi_loss(o, r, p, dy, eps) - _epi_loss(o, r, m, dy, eps)) / (2 * h)
+        assert abs(d_g[j] - fd) <= 1e-7 * max(1.0, abs(fd))
+
+
+def test_epilogue_bwd_grad_orthogonal_to_o_without_eps():
+    # eps = 0 makes y invariant to o -> c o, so the o-gradient has no component along o
+    rng = np.random.default_rng(74)
+    o = rng.standard_normal((6, 16))
+    r = rng.standard_normal((6, 16))
+    dy = rng.standard_normal((6, 16))
+    d_o, _, _ = oracle.epilogue_bwd(o, r, dy, rng.standard_normal(16), eps=0.0)
+    assert np.max(np.abs(np.sum(d_o * o, axis=-1))) <= 1e-12 * np.max(np.abs(d_o)) * 16
+    assert np.max(np.abs(d_o)) > 1e-3
+
+
+def test_epilogue_bwd_zero_gate_passes_only_r_gradient():
+    # Swish(0) = 0 and Swish'(0) = 1/2: with r = 0 the o- and gamma-gradients vanish and
+    # d_r = dy * RMSNorm(o) * gamma / 2
+    rng = np.random.default_rng(75)
+    o = rng.standard_normal((4, 8))
+    dy = rng.standard_normal((4, 8))
+    gamma = rng.standard_normal(8)
+    d_o, d_r, d_g = oracle.epilogue_bwd(o, np.zeros_like(o), dy, gamma, eps=0.0)
+    assert np.all(d_o == 0.0) and np.all(d_g == 0.0)
+    n = o / np.sqrt(np.mean(o * o, axis=-1, keepdims=True))
+    assert np.allclose(d_r, dy * n * gamma * 0.5, rtol=1e-13, atol=1e-15)
+
+
+# ----------------------------------------------------------------------------- SREM conv backward
+
+@pytest.mark.parametrize("mode", range(4))
+@pytest.mark.parametrize("hw", [(5, 7), (1, 4), (6, 1), (3, 3)])
+def test_conv_bwd_dx_is_adjoint_of_forward(mode, hw):
+    rng = np.random.default_rng(80 + mode)
+    Hg, Wg = hw
+    B, C = 2, 3
+    w = rng.standard_normal((C, 3, 3))
+    dy = rng.standard_normal((B, Hg * Wg, C))
+    dx, _, _ = oracle.srem_dwconv_bwd(rng.standard_normal((B, Hg, Wg, C)), w, dy, mode)
+    # <conv(e), dy> = <e, dx> for every basis input e: the forward applied to each unit input
+    for b in range(B):
+        for r in range(Hg):
+            for c in range(Wg):
+                for ch in range(C):
+                    e = np.zeros((B, Hg, Wg, C))
+                    e[b, r, c, ch] = 1.0
+                    ref = np.sum(oracle.srem_dwconv(e, w, None, mode) * dy)
+                    assert abs(dx[b, r, c, ch] - ref) <= 1e-12 * max(1.0, abs(ref))
+
+
+@pytest.mark.parametrize("mode", range(4))
+def test_conv_bwd_dw_dbias_from_one_tap_kernels(mode):
+    rng = np.random.default_rng(84 + mode)
+    B, Hg, Wg, C = 2, 4, 6, 3
+    x = rng.standard_normal((B, Hg, Wg, C))
+    dy = rng.standard_normal((B, Hg * Wg, C))
+    _, dw, db = oracle.srem_dwconv_bwd(x, rng.standard_normal((C, 3, 3)), dy, mode)
+    # the loss is linear in w and bias: each coefficient is the forward with a one-tap kernel
+    for tap in range(9):
+        wt = np.zeros((C, 3, 3))
+        wt[:, tap // 3, tap % 3] = 1.0
+        ref = np.sum(oracle.srem_dwconv(x, wt, None, mode) * dy, axis=(0, 1))
+        assert np.allclose(dw[:, tap // 3, tap % 3], ref, rtol=1e-12, atol=1e-12)
+    ref_b = np.sum(oracle.srem_dwconv(x, np.zeros((C, 3, 3)), np.ones(C), mode) * dy, axis=(0, 1))
+    assert np.allclose(db, ref_b, rtol=1e-12, atol=1e-12)
+
+
+def test_conv_bwd_matches_scipy_full_correlation():
+    # dx of a 'same' correlation is a 'same' convolution of the grid gradient with the kernel
+    rng = np.random.default_rng(88)
+    B, Hg, Wg, C = 1, 5, 4, 2
+    x = rng.standard_normal((B, Hg, Wg, C))
+    w = rng.standard_normal((C, 3, 3))
+    dy = rng.standard_normal((B, Hg * Wg, C))
+    mode = 3
+    dx, _, _ = oracle.srem_dwconv_bwd(x, w, dy, mode)
+    perm = oracle.scan_index(mode, Hg, Wg)
+    dyg = np.zeros((Hg * Wg, C))
+    dyg[perm] = dy[0]
+    for c in range(C):
+        ref = scipy.signal.convolve2d(dyg[:, c].reshape(Hg, Wg), w[c], mode="same", boundary="fill")
+        assert np.allclose(dx[0, :, :, c], ref, rtol=1e-13, atol=1e-13)
