@@ -65,7 +65,11 @@ def algorithmic_bytes(w):
     fwd = 2 * qk + vv + z + vv + 2 * vv        # q k v z r in; o y out
     bwd = 2 * qk + vv + z + vv + 2 * qk + vv + z  # q k v z dO in; dq dk dv dlogalpha out
     conv = 2 * BL * w.conv_C * e
-    return {"fwd": fwd, "bwd": bwd, "conv": conv}
+    # the backward ops outside the step: the epilogue's (o r dY in; d_o d_r out) and the
+    # conv's (x dY in; dx out); the fp32 parameter vectors are a few KB
+    epi_bwd = 5 * vv
+    conv_bwd = 3 * BL * w.conv_C * e
+    return {"fwd": fwd, "bwd": bwd, "conv": conv, "epi_bwd": epi_bwd, "conv_bwd": conv_bwd}
 
 
 # This library's kernels per op, in launch order, and the sources they are built from.
@@ -73,13 +77,20 @@ OP_KERNELS = {
     "fwd": ["gla_gate_kernel", "gla_chunk_state_kernel", "gla_state_scan_kernel", "gla_chunk_out_kernel"],
     "bwd": ["gla_chunk_dh_kernel", "gla_state_scan_kernel", "gla_chunk_grad_kernel"],
     "conv": ["srem_dwconv_kernel"],
+    "epi_bwd": ["epilogue_bwd_kernel"],
+    "conv_bwd": ["srem_dwconv_bwd_kernel"],
 }
+STEP_OPS = ("fwd", "bwd", "conv")  # the ops of one timed step
 _CHUNK_SRC = ["gla_chunk.cuh", "gla_common.cuh", "sm100.cuh", "dig_common.cuh", "gla.h"]
 OP_SOURCES = {
     "fwd": ["gla_fwd.cu"] + _CHUNK_SRC,
     "bwd": ["gla_bwd.cu", "gla_fwd.cu"] + _CHUNK_SRC,
-    "conv": ["srem.cu", "dig_common.cuh", "gla.h"],
+    "conv": ["srem.cu", "srem.cuh", "dig_common.cuh", "gla.h"],
+    "epi_bwd": ["epilogue_bwd.cu", "gla_common.cuh", "sm100.cuh", "dig_common.cuh", "bwd_ops.h"],
+    "conv_bwd": ["srem_bwd.cu", "srem.cuh", "gla_common.cuh", "sm100.cuh", "dig_common.cuh", "bwd_ops.h"],
 }
+OP_NAMES = {"fwd": "dig_gla_fwd", "bwd": "dig_gla_bwd_saved", "conv": "dig_srem_reorient_dwconv",
+            "epi_bwd": "dig_epilogue_bwd", "conv_bwd": "dig_srem_reorient_dwconv_bwd"}
 
 
 def _src_hash(names):
@@ -205,6 +216,34 @@ def _config(w, world):
                    "their own streams overlap the neighbouring steps' compute, two device buffer sets alternate"}
 
 
+def time_backward_ops(dig, w, dev, stream, o, r, dY, xc, wc, flush, warmup, iters):
+    """Mean event-timed seconds of one dig_epilogue_bwd and one
+    dig_srem_reorient_dwconv_bwd call (with d_gamma, dw and dbias)."""
+    g = torch.Generator(device=dev).manual_seed(1)
+    d_o, d_r = torch.empty_like(o), torch.empty_like(o)
+    d_gamma = torch.empty(w.dv, device=dev)
+    dyc = torch.randn(w.B, w.L, w.conv_C, device=dev, generator=g).to(xc.dtype)
+    dx = torch.empty_like(xc)
+    dw, db = torch.empty(w.conv_C, 3, 3, device=dev), torch.empty(w.conv_C, device=dev)
+    calls = {
+        "epi_bwd": lambda i: dig.dig_epilogue_bwd(o, r, dY, d_o, d_r, None, 1e-5, d_gamma, stream=stream),
+        "conv_bwd": lambda i: dig.dig_srem_reorient_dwconv_bwd(xc, wc, dyc, dx, i % 4, dw, db, stream=stream),
+    }
+    out = {}
+    for op, call in calls.items():
+        for i in range(warmup):
+            call(i)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+        for i in range(iters):
+            flush.fill_(float(i))
+            evs[i][0].record(stream)
+            call(i)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        out[op] = float(np.mean([a.elapsed_time(b) for a, b in evs])) * 1e-3
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
     from gated_linear_attention_fwd_b200 import dig
     dev = torch.device("cuda", local_rank)
@@ -322,10 +361,16 @@ def run_ours(args, rank, world, local_rank):
     e1.synchronize()
     e2e_step_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
 
+    # the backward ops of the epilogue and the conv (outside the step): each timed
+    # alone with CUDA events, L2 flushed before every call, on the bench's workload
+    aux_t = time_backward_ops(dig, w, dev, stream, o, r, dO, xc, wc, flush, args.warmup, max(args.steps, 10))
+    aux_t = {op: max_over_ranks(tv, world, dev) for op, tv in aux_t.items()}
+
     if rank != 0:
         return None
     hbm, tflops, peak_kind = _peaks()
     algo = algorithmic_bytes(w)
+    step_algo = sum(algo[op] for op in STEP_OPS)
     t_f, t_b, t_c = [float(per[:, j].mean()) * 1e-3 for j in range(3)]
     # Each op is a short sequence of this library's kernels launched by one C-ABI
     # call; its roofline is taken over the whole sequence (algorithmic bytes of
@@ -347,12 +392,17 @@ def run_ours(args, rank, world, local_rank):
                      "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": _traffic(kname, srcs, 1.0),
                      "algorithmic_bytes": algo[dom], "peak_source": peak_kind,
-                     "step_frac": (sum(algo.values()) / hbm / 1e9) / (step_ms * 1e-3)},
+                     "step_frac": (step_algo / hbm / 1e9) / (step_ms * 1e-3)},
         "ops_us": {"dig_gla_fwd": t_f * 1e6, "dig_gla_bwd_saved": t_b * 1e6, "dig_srem_reorient_dwconv": t_c * 1e6},
         "e2e": {"value": tokens / (e2e_step_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": sum(len(k) for k in OP_KERNELS.values()) * args.steps,
+        "gpu_launches": sum(len(OP_KERNELS[op]) for op in STEP_OPS) * args.steps,
         "clocks": clk.summary(),
+        "backward_ops": {OP_NAMES[op]: {"us": t * 1e6, "achieved": algo[op] / t / 1e9, "unit": "GB/s",
+                                        "frac": algo[op] / t / 1e9 / hbm, "algorithmic_bytes": algo[op],
+                                        "traffic": _traffic(OP_NAMES[op], OP_SOURCES[op], 1.0),
+                                        "kernels": OP_KERNELS[op]}
+                         for op, t in aux_t.items()},
     }
     if world == 1 and not args.no_cpu_baseline:
         tps, dt, cores, n = cpu_sample(w, x, steps=1, min_seconds=10.0)

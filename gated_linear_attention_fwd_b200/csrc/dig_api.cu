@@ -7,6 +7,7 @@
 
 #include "../../include/dig.h"
 #include "dig_common.cuh"
+#include "bwd_ops.h"
 #include "gla.h"
 
 namespace dig {
@@ -212,6 +213,54 @@ dig_status dig_srem_reorient_dwconv(const void* x, const float* w, const float* 
   const cudaError_t e =
       launch_srem(x, w, bias, y, B, grid_h, grid_w, C, scan_mode, dtype, out_dtype, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "srem launch: %s", cudaGetErrorString(e));
+  return DIG_OK;
+}
+
+dig_status dig_srem_reorient_dwconv_bwd(const void* x, const float* w, const void* dY, void* dx, float* dw,
+                                        float* dbias, int B, int grid_h, int grid_w, int C, int scan_mode, int dtype,
+                                        int out_dtype, void* stream) {
+  if (B < 0 || grid_h < 0 || grid_w < 0 || C <= 0)
+    return fail(DIG_ERR_INVALID_ARGUMENT, "bad size (B=%d grid=%dx%d C=%d)", B, grid_h, grid_w, C);
+  if (scan_mode < 0 || scan_mode > 3) return fail(DIG_ERR_INVALID_ARGUMENT, "scan_mode %d not in 0..3", scan_mode);
+  if ((dtype != DIG_F32 && dtype != DIG_BF16) || (out_dtype != DIG_F32 && out_dtype != DIG_BF16))
+    return fail(DIG_ERR_INVALID_ARGUMENT, "dtype %d / out_dtype %d not DIG_F32 or DIG_BF16", dtype, out_dtype);
+  if ((long long)B * grid_h * grid_w * C >= (1ll << 40)) return fail(DIG_ERR_INVALID_ARGUMENT, "tensor too large");
+  if ((long long)grid_h * grid_w >= (1ll << 31)) return fail(DIG_ERR_INVALID_ARGUMENT, "grid too large");
+  if (!w) return fail(DIG_ERR_INVALID_ARGUMENT, "w must be non-NULL");
+  if (!aligned16(x) || !aligned16(w) || !aligned16(dY) || !aligned16(dx) || !aligned16(dw) || !aligned16(dbias))
+    return fail(DIG_ERR_MISALIGNED, "a tensor pointer is not 16-byte aligned");
+  if (B == 0 || grid_h == 0 || grid_w == 0) {  // no pixels: the parameter gradients are zero
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = dw ? cudaMemsetAsync(dw, 0, (size_t)C * 9 * sizeof(float), s) : cudaSuccess;
+    if (e == cudaSuccess && dbias) e = cudaMemsetAsync(dbias, 0, (size_t)C * sizeof(float), s);
+    if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
+    return DIG_OK;
+  }
+  if (!dY || !dx) return fail(DIG_ERR_INVALID_ARGUMENT, "dY and dx must be non-NULL");
+  if ((dw || dbias) && !x) return fail(DIG_ERR_INVALID_ARGUMENT, "x must be non-NULL when dw or dbias is wanted");
+  const cudaError_t e = launch_srem_bwd(x, w, dY, dx, dw, dbias, B, grid_h, grid_w, C, scan_mode, dtype, out_dtype,
+                                        static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "srem backward launch: %s", cudaGetErrorString(e));
+  return DIG_OK;
+}
+
+dig_status dig_epilogue_bwd(const void* o, const void* r, const float* gamma, float eps, const void* dY, void* d_o,
+                            void* d_r, float* d_gamma, long long rows, int d_v, int dtype, int out_dtype,
+                            void* stream) {
+  if (rows < 0 || d_v <= 0) return fail(DIG_ERR_INVALID_ARGUMENT, "bad size (rows=%lld d_v=%d)", rows, d_v);
+  if (d_v > 8192) return fail(DIG_ERR_UNSUPPORTED, "d_v=%d above 8192", d_v);
+  if (!(eps >= 0.f)) return fail(DIG_ERR_INVALID_ARGUMENT, "eps must be >= 0");
+  if ((dtype != DIG_F32 && dtype != DIG_BF16) || (out_dtype != DIG_F32 && out_dtype != DIG_BF16))
+    return fail(DIG_ERR_INVALID_ARGUMENT, "dtype %d / out_dtype %d not DIG_F32 or DIG_BF16", dtype, out_dtype);
+  if (rows >= (1ll << 40) / d_v) return fail(DIG_ERR_INVALID_ARGUMENT, "tensor too large");
+  if (rows > 0 && (!o || !r || !dY || !d_o || !d_r))
+    return fail(DIG_ERR_INVALID_ARGUMENT, "o, r, dY, d_o and d_r must be non-NULL");
+  if (!aligned16(o) || !aligned16(r) || !aligned16(dY) || !aligned16(d_o) || !aligned16(d_r) ||
+      !aligned16(gamma) || !aligned16(d_gamma))
+    return fail(DIG_ERR_MISALIGNED, "a tensor pointer is not 16-byte aligned");
+  const cudaError_t e = launch_epilogue_bwd(o, r, gamma, eps, dY, d_o, d_r, d_gamma, rows, d_v, dtype, out_dtype,
+                                            static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "epilogue backward launch: %s", cudaGetErrorString(e));
   return DIG_OK;
 }
 

@@ -60,6 +60,10 @@ lib.dig_gla_bwd_saved.argtypes = [_vp, _vp, _vp, _vp, _i, _f, _vp, _vp, _vp, _vp
                                   _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp, _sz, _vp]
 lib.dig_srem_reorient_dwconv.restype = _i
 lib.dig_srem_reorient_dwconv.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
+lib.dig_srem_reorient_dwconv_bwd.restype = _i
+lib.dig_srem_reorient_dwconv_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
+lib.dig_epilogue_bwd.restype = _i
+lib.dig_epilogue_bwd.argtypes = [_vp, _vp, _vp, _f, _vp, _vp, _vp, _vp, ctypes.c_longlong, _i, _i, _i, _vp]
 lib.dig_read_status.restype = _i
 lib.dig_read_status.argtypes = [_vp, _vp]
 lib.dig_status_string.restype = ctypes.c_char_p
@@ -176,6 +180,23 @@ def dig_srem_reorient_dwconv(x, w, bias, y, scan_mode, stream=None):
     st = lib.dig_srem_reorient_dwconv(_ptr(x), _ptr(w), _ptr(bias), _ptr(y), B, Hg, Wg, C, scan_mode,
                                       _code(x.dtype), _code(y.dtype), _stream(stream))
     _check(st, "dig_srem_reorient_dwconv")
+
+
+def dig_srem_reorient_dwconv_bwd(x, w, dY, dx, scan_mode, dw=None, dbias=None, stream=None):
+    """x, dx [B,Hg,Wg,C] grid order; w [C,3,3] fp32; dY [B,L,C] scan order; dw [C,3,3], dbias [C] fp32 or None."""
+    B, Hg, Wg, C = dx.shape
+    st = lib.dig_srem_reorient_dwconv_bwd(_ptr(x), _ptr(w), _ptr(dY), _ptr(dx), _ptr(dw), _ptr(dbias),
+                                          B, Hg, Wg, C, scan_mode, _code(dY.dtype), _code(dx.dtype), _stream(stream))
+    _check(st, "dig_srem_reorient_dwconv_bwd")
+
+
+def dig_epilogue_bwd(o, r, dY, d_o, d_r, gamma=None, eps=1e-5, d_gamma=None, stream=None):
+    """o, r, dY [..., d_v] (same dtype); d_o, d_r [..., d_v]; gamma, d_gamma [d_v] fp32 or None."""
+    d_v = o.shape[-1]
+    rows = o.numel() // d_v if d_v else 0
+    st = lib.dig_epilogue_bwd(_ptr(o), _ptr(r), _ptr(gamma), float(eps), _ptr(dY), _ptr(d_o), _ptr(d_r),
+                              _ptr(d_gamma), rows, d_v, _code(o.dtype), _code(d_o.dtype), _stream(stream))
+    _check(st, "dig_epilogue_bwd")
 
 
 def dig_read_status(workspace, stream=None) -> int:

@@ -14,7 +14,7 @@ from . import dig, inputs
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", choices=["fwd", "bwd", "conv"], default="fwd")
+    ap.add_argument("--op", choices=["fwd", "bwd", "conv", "epi_bwd", "conv_bwd"], default="fwd")
     ap.add_argument("--workload", type=int, default=3)
     ap.add_argument("--iters", type=int, default=4)
     ap.add_argument("--mode", type=int, default=0)
@@ -31,6 +31,24 @@ def main():
         y = torch.empty(B, L, C, device="cuda", dtype=dt)
         for _ in range(args.iters):
             dig.dig_srem_reorient_dwconv(x, wc, None, y, args.mode)
+        torch.cuda.synchronize()
+        print("ok")
+        return
+    if args.op == "conv_bwd":
+        C = w.conv_C or H * dv
+        x, wc = rnd(B, w.grid_h, w.grid_w, C), torch.randn(C, 3, 3, device="cuda", generator=g) * 0.1
+        dy, dx = rnd(B, L, C), torch.empty(B, w.grid_h, w.grid_w, C, device="cuda", dtype=dt)
+        dw, db = torch.empty(C, 3, 3, device="cuda"), torch.empty(C, device="cuda")
+        for _ in range(args.iters):
+            dig.dig_srem_reorient_dwconv_bwd(x, wc, dy, dx, args.mode, dw, db)
+        torch.cuda.synchronize()
+        print("ok")
+        return
+    if args.op == "epi_bwd":
+        o, r, dy = rnd(B, L, H, dv), rnd(B, L, H, dv), rnd(B, L, H, dv)
+        d_o, d_r, d_g = torch.empty_like(o), torch.empty_like(o), torch.empty(dv, device="cuda")
+        for _ in range(args.iters):
+            dig.dig_epilogue_bwd(o, r, dy, d_o, d_r, None, 1e-5, d_g)
         torch.cuda.synchronize()
         print("ok")
         return

@@ -90,10 +90,10 @@ def traffic(args):
             rd += _value(r)
         elif r["Metric Name"] == "dram__bytes_write.sum":
             wr += _value(r)
-    name = {"fwd": "dig_gla_fwd", "bwd": "dig_gla_bwd_saved", "conv": "dig_srem_reorient_dwconv"}[args.op]
+    name = bench.OP_NAMES[args.op]
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     d = json.load(open(path)) if os.path.exists(path) else {}
-    d = {k: v for k, v in d.items() if k in ("dig_gla_fwd", "dig_gla_bwd_saved", "dig_srem_reorient_dwconv")}
+    d = {k: v for k, v in d.items() if k in bench.OP_NAMES.values()}
     d[name] = {
         "source_sha": bench._src_hash(bench.OP_SOURCES[args.op]),
         "dram_bytes_per_call": int((rd + wr) / args.calls),
@@ -118,7 +118,7 @@ def main():
     a.add_argument("--command", required=True)
     t = sub.add_parser("traffic")
     t.add_argument("csv")
-    t.add_argument("--op", choices=["fwd", "bwd", "conv"], required=True)
+    t.add_argument("--op", choices=["fwd", "bwd", "conv", "epi_bwd", "conv_bwd"], required=True)
     t.add_argument("--calls", type=int, required=True)
     t.add_argument("--workload", required=True)
     t.add_argument("--command", required=True)

@@ -16,6 +16,8 @@
  *   SREM       slide "SREM (Spatial Reorient & Enhancement Module) の導入" and the
  *              paper's "DiG Block" section: 3x3 depthwise conv on the 2-D token grid
  *              and one of four scan orders (transpose / flip)
+ *   backward   gradients of the three operations by the chain rule, for training
+ *              (the paper trains DiG end to end)
  *
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
@@ -180,6 +182,42 @@ dig_status dig_gla_bwd_saved(const void *q, const void *k, const void *v, const 
 dig_status dig_srem_reorient_dwconv(const void *x, const float *w, const float *bias, void *y,
                                     int B, int grid_h, int grid_w, int C, int scan_mode,
                                     int dtype, int out_dtype, void *stream);
+
+/* Backward of dig_srem_reorient_dwconv: gradients of sum(dY * y).
+ *   x      [B, grid_h, grid_w, C] dtype, grid order: the forward's input (only read
+ *          for dw; may be NULL when dw and dbias are both NULL)
+ *   w      [C, 3, 3] fp32: the forward's weights
+ *   dY     [B, L, C] dtype, SCAN order (the layout of the forward's y)
+ *   dx     [B, grid_h, grid_w, C] out_dtype, grid order:
+ *          dx[g] = sum_{di,dj} w[di+1, dj+1] * dY at the scan position of g - (di, dj)
+ *   dw     [C, 3, 3] fp32 or NULL; dbias [C] fp32 or NULL: sums over B and the
+ *          grid.  Overwritten: the call zeroes them on `stream` first.  With an
+ *          even C the partial sums of the thread blocks are added with
+ *          floating-point atomics, so their last bits may differ between runs.
+ * Same element types, alignment and stream rules as the forward. */
+dig_status dig_srem_reorient_dwconv_bwd(const void *x, const float *w, const void *dY, void *dx,
+                                        float *dw, float *dbias,
+                                        int B, int grid_h, int grid_w, int C, int scan_mode,
+                                        int dtype, int out_dtype, void *stream);
+
+/* Backward of the epilogue (slide eq. (9)-(10)): gradients of sum(dY * y) for
+ * y = Swish(r) * o / sqrt(mean(o^2) + eps) * gamma, taken row by row over d_v as
+ * dig_gla_fwd computes it (rows = B * L * H for its [B, L, H, d_v] tensors; any
+ * row order, as long as o, r, dY, d_o and d_r share it).
+ *   o, r, dY   [rows, d_v] dtype       the forward's o and r, and dLoss/dy
+ *   gamma      [d_v] fp32 or NULL (ones)
+ *   eps        the forward's eps (>= 0)
+ *   d_o        [rows, d_v] out_dtype   dLoss/do: the dO to pass to dig_gla_bwd
+ *   d_r        [rows, d_v] out_dtype   dLoss/dr
+ *   d_gamma    [d_v] fp32 or NULL: dLoss/dgamma summed over the rows.  Overwritten:
+ *              the call zeroes it on `stream` first, then adds the thread blocks'
+ *              partial sums with floating-point atomics (last bits may differ
+ *              between runs).
+ * d_v up to 8192 (DIG_ERR_UNSUPPORTED above).  Same element types, alignment and
+ * stream rules as the forward. */
+dig_status dig_epilogue_bwd(const void *o, const void *r, const float *gamma, float eps,
+                            const void *dY, void *d_o, void *d_r, float *d_gamma,
+                            long long rows, int d_v, int dtype, int out_dtype, void *stream);
 
 /* Synchronises `stream`, returns the device status word kept in `workspace`
  * (DIG_OK, DIG_ERR_DEVICE_TIMEOUT or DIG_ERR_GATE_RANGE) and clears it. */

@@ -26,6 +26,7 @@ def _fwd(**kw):
 def test_exports_every_declared_function():
     names = dig.header_functions()
     assert {"dig_gla_fwd", "dig_gla_bwd", "dig_srem_reorient_dwconv", "dig_gla_workspace_bytes",
+            "dig_epilogue_bwd", "dig_srem_reorient_dwconv_bwd",
             "dig_read_status", "dig_status_string", "dig_last_error", "dig_gla_supported"} <= set(names)
     for n in names:
         assert hasattr(dig.lib, n), n
@@ -90,6 +91,33 @@ def test_bwd_and_conv_reject_bad_arguments_on_host():
     assert dig.lib.dig_srem_reorient_dwconv(1024, 1024, N, 1032, 1, 3, 4, 8, 0, 1, 1, N) == dig.DIG_ERR_MISALIGNED
     assert dig.lib.dig_srem_reorient_dwconv(1024, 1024, N, 1024, 1, 3, 4, 0, 0, 1, 1, N) == \
         dig.DIG_ERR_INVALID_ARGUMENT
+
+
+def test_backward_helpers_reject_bad_arguments_on_host():
+    E = dig.lib.dig_epilogue_bwd
+    ok = dict(o=1024, r=1024, gamma=N, eps=1e-5, dY=1024, d_o=1024, d_r=1024, d_gamma=N, rows=4, d_v=64,
+              dtype=1, out_dtype=1)
+
+    def epi(**kw):
+        a = dict(ok, **kw)
+        return E(a["o"], a["r"], a["gamma"], a["eps"], a["dY"], a["d_o"], a["d_r"], a["d_gamma"], a["rows"],
+                 a["d_v"], a["dtype"], a["out_dtype"], N)
+    assert epi(d_v=0) == dig.DIG_ERR_INVALID_ARGUMENT
+    assert epi(rows=-1) == dig.DIG_ERR_INVALID_ARGUMENT
+    assert epi(d_v=8193) == dig.DIG_ERR_UNSUPPORTED
+    assert epi(eps=-1.0) == dig.DIG_ERR_INVALID_ARGUMENT
+    assert epi(dtype=7) == dig.DIG_ERR_INVALID_ARGUMENT
+    assert epi(o=N) == dig.DIG_ERR_INVALID_ARGUMENT
+    assert epi(d_r=1032) == dig.DIG_ERR_MISALIGNED
+    assert epi(d_gamma=1028) == dig.DIG_ERR_MISALIGNED
+    C = dig.lib.dig_srem_reorient_dwconv_bwd
+    # x, w, dY, dx, dw, dbias, B, grid_h, grid_w, C, mode, dtype, out_dtype, stream
+    assert C(1024, 1024, 1024, 1024, N, N, 1, 3, 4, 0, 0, 1, 1, N) == dig.DIG_ERR_INVALID_ARGUMENT
+    assert C(1024, 1024, 1024, 1024, N, N, 1, 3, 4, 8, 4, 1, 1, N) == dig.DIG_ERR_INVALID_ARGUMENT
+    assert C(N, 1024, 1024, 1024, 1024, N, 1, 3, 4, 8, 0, 1, 1, N) == dig.DIG_ERR_INVALID_ARGUMENT  # dw needs x
+    assert C(1024, N, 1024, 1024, N, N, 1, 3, 4, 8, 0, 1, 1, N) == dig.DIG_ERR_INVALID_ARGUMENT
+    assert C(1024, 1024, 1024, 1024, 1036, N, 1, 3, 4, 8, 0, 1, 1, N) == dig.DIG_ERR_MISALIGNED
+    assert C(1024, 1024, 1024, 1024, N, N, 1, 3, 4, 8, 0, 1, 2, N) == dig.DIG_ERR_INVALID_ARGUMENT
 
 
 def test_workspace_bytes():
