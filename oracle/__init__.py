@@ -19,6 +19,9 @@ Parity status of each function (what pins it is in tests/test_oracle_pins.py):
                  positive scale invariance
   epilogue_bwd   pinned: central finite differences of sum(dy * epilogue) in o, r
                  and gamma; d_o orthogonal to o when eps = 0 (scale invariance)
+  gate_proj_fwd  pinned: numpy matmul (x @ W1) @ W2 + b; rank-one closed form
+  gate_proj_bwd  pinned: central finite differences of sum(dla * inv_tau * logsigmoid(z))
+                 in x, W1, W2 and b
   srem_dwconv_bwd pinned: adjoint identity <conv(x), dy> = <x, dx>; dw and dbias
                  from the forward conv with one-tap kernels / zero kernel
   scan_index     pinned: bijection, inverse restores the grid, transpose on
@@ -57,6 +60,10 @@ def _load():
         lib.oracle_epilogue_bwd.argtypes = [dp, dp, dp, ctypes.c_double, dp, dp, dp, dp, L, L]
         lib.oracle_srem_dwconv_bwd.restype = ctypes.c_int
         lib.oracle_srem_dwconv_bwd.argtypes = [dp, dp, dp, dp, dp, dp, L, L, L, L, ctypes.c_int]
+        lib.oracle_gate_proj_fwd.restype = ctypes.c_int
+        lib.oracle_gate_proj_fwd.argtypes = [dp, dp, dp, dp, dp, dp, L, L, L, L]
+        lib.oracle_gate_proj_bwd.restype = ctypes.c_int
+        lib.oracle_gate_proj_bwd.argtypes = [dp, dp, dp, dp, dp, ctypes.c_double, dp, dp, dp, dp, L, L, L, L]
         lib.oracle_srem_dwconv.restype = ctypes.c_int
         lib.oracle_srem_dwconv.argtypes = [dp, dp, dp, dp, L, L, L, L, ctypes.c_int]
         _lib = lib
@@ -166,6 +173,34 @@ def srem_dwconv_bwd(x, w, dy, mode):
     if rc:
         raise ValueError("oracle_srem_dwconv_bwd rejected the arguments (rc=%d)" % rc)
     return dx, dw, db
+
+
+def gate_proj_fwd(x, W1, W2, b=None):
+    """z = (x W1) W2 + b over the last axis of x [..., D]; returns (z [..., dk], u = x W1 [..., R])."""
+    x, W1, W2 = _f64(x), _f64(W1), _f64(W2)
+    D, R, dk = W1.shape[0], W1.shape[1], W2.shape[1]
+    rows = x.size // D
+    bb = None if b is None else _f64(b)
+    z = np.zeros(x.shape[:-1] + (dk,), dtype=np.float64)
+    u = np.zeros(x.shape[:-1] + (R,), dtype=np.float64)
+    rc = _load().oracle_gate_proj_fwd(_ptr(x), _ptr(W1), _ptr(W2), _ptr(bb), _ptr(z), _ptr(u), rows, D, R, dk)
+    if rc:
+        raise ValueError("oracle_gate_proj_fwd rejected the arguments")
+    return z, u
+
+
+def gate_proj_bwd(x, W1, W2, z, dlog_alpha, inv_tau):
+    """Gradients (dx, dW1, dW2, db) of sum(dlog_alpha * inv_tau * logsigmoid(z)) for z = gate_proj_fwd(x, W1, W2, b)."""
+    x, W1, W2, z, dla = _f64(x), _f64(W1), _f64(W2), _f64(z), _f64(dlog_alpha)
+    D, R, dk = W1.shape[0], W1.shape[1], W2.shape[1]
+    rows = x.size // D
+    dx = np.zeros_like(x)
+    dW1, dW2, db = np.zeros((D, R)), np.zeros((R, dk)), np.zeros(dk)
+    rc = _load().oracle_gate_proj_bwd(_ptr(x), _ptr(W1), _ptr(W2), _ptr(z), _ptr(dla), float(inv_tau), _ptr(dx),
+                                      _ptr(dW1), _ptr(dW2), _ptr(db), rows, D, R, dk)
+    if rc:
+        raise ValueError("oracle_gate_proj_bwd rejected the arguments (rc=%d)" % rc)
+    return dx, dW1, dW2, db
 
 
 def srem_dwconv(x, w, bias, mode):

@@ -387,3 +387,82 @@ int oracle_srem_dwconv_bwd(const double *x, const double *w, const double *dy,
     free(dyg);
     return 0;
 }
+
+/* Gate projection (slide "Gated Linear Attention Transformer (GLA) の導入", eq. (5):
+ * the gate logits come from the block input through a low-rank projection):
+ *   u = x W1   [rows][R],   z = u W2 + b   [rows][dk]
+ * x [rows][D], W1 [D][R], W2 [R][dk], b [dk] (NULL = 0).  u may be NULL. */
+int oracle_gate_proj_fwd(const double *x, const double *W1, const double *W2, const double *b,
+                         double *z, double *u, long rows, long D, long R, long dk)
+{
+    if (rows < 0 || D <= 0 || R <= 0 || dk <= 0) return 1;
+#pragma omp parallel for schedule(static)
+    for (long t = 0; t < rows; ++t) {
+        double ut[64];
+        if (R > 64) continue;
+        for (long r = 0; r < R; ++r) {
+            double acc = 0.0;
+            for (long d = 0; d < D; ++d) acc += x[t * D + d] * W1[d * R + r];
+            ut[r] = acc;
+            if (u) u[t * R + r] = acc;
+        }
+        for (long k = 0; k < dk; ++k) {
+            double acc = b ? b[k] : 0.0;
+            for (long r = 0; r < R; ++r) acc += ut[r] * W2[r * dk + k];
+            z[t * dk + k] = acc;
+        }
+    }
+    return R > 64 ? 1 : 0;
+}
+
+/* Its backward from the GLA backward's d log(alpha): log(alpha) = inv_tau * logsigmoid(z),
+ * so dz = dlog_alpha * inv_tau * sigmoid(-z); then, by the chain rule through z = (x W1) W2 + b,
+ *   du = dz W2^T,  dx = du W1^T,  dW1 = x^T du,  dW2 = u^T dz (u = x W1),  db = sum_t dz. */
+int oracle_gate_proj_bwd(const double *x, const double *W1, const double *W2, const double *z,
+                         const double *dla, double inv_tau, double *dx, double *dW1, double *dW2,
+                         double *db, long rows, long D, long R, long dk)
+{
+    if (rows < 0 || D <= 0 || R <= 0 || dk <= 0 || R > 64) return 1;
+    double *u = (double *)malloc(sizeof(double) * (size_t)(rows * R > 0 ? rows * R : 1));
+    double *du = (double *)malloc(sizeof(double) * (size_t)(rows * R > 0 ? rows * R : 1));
+    double *dz = (double *)malloc(sizeof(double) * (size_t)(rows * dk > 0 ? rows * dk : 1));
+    if (!u || !du || !dz) { free(u); free(du); free(dz); return 2; }
+#pragma omp parallel for schedule(static)
+    for (long t = 0; t < rows; ++t) {
+        for (long k = 0; k < dk; ++k)
+            dz[t * dk + k] = dla[t * dk + k] * inv_tau / (1.0 + exp(z[t * dk + k]));
+        for (long r = 0; r < R; ++r) {
+            double a = 0.0, g = 0.0;
+            for (long d = 0; d < D; ++d) a += x[t * D + d] * W1[d * R + r];
+            for (long k = 0; k < dk; ++k) g += dz[t * dk + k] * W2[r * dk + k];
+            u[t * R + r] = a;
+            du[t * R + r] = g;
+        }
+        for (long d = 0; d < D; ++d) {
+            double acc = 0.0;
+            for (long r = 0; r < R; ++r) acc += du[t * R + r] * W1[d * R + r];
+            dx[t * D + d] = acc;
+        }
+    }
+#pragma omp parallel for schedule(static)
+    for (long d = 0; d < D; ++d)
+        for (long r = 0; r < R; ++r) {
+            double acc = 0.0;
+            for (long t = 0; t < rows; ++t) acc += x[t * D + d] * du[t * R + r];
+            dW1[d * R + r] = acc;
+        }
+    for (long r = 0; r < R; ++r)
+        for (long k = 0; k < dk; ++k) {
+            double acc = 0.0;
+            for (long t = 0; t < rows; ++t) acc += u[t * R + r] * dz[t * dk + k];
+            dW2[r * dk + k] = acc;
+        }
+    if (db)
+        for (long k = 0; k < dk; ++k) {
+            double acc = 0.0;
+            for (long t = 0; t < rows; ++t) acc += dz[t * dk + k];
+            db[k] = acc;
+        }
+    free(u); free(du); free(dz);
+    return 0;
+}

@@ -436,3 +436,47 @@ def test_conv_bwd_matches_scipy_full_correlation():
     for c in range(C):
         ref = scipy.signal.convolve2d(dyg[:, c].reshape(Hg, Wg), w[c], mode="same", boundary="fill")
         assert np.allclose(dx[0, :, :, c], ref, rtol=1e-13, atol=1e-13)
+
+
+# ----------------------------------------------------------------------------- gate projection
+
+def test_gate_proj_fwd_matches_matmul_and_rank_one():
+    rng = np.random.default_rng(90)
+    x = rng.standard_normal((2, 7, 12))
+    W1, W2, b = rng.standard_normal((12, 4)), rng.standard_normal((4, 5)), rng.standard_normal(5)
+    z, u = oracle.gate_proj_fwd(x, W1, W2, b)
+    assert np.allclose(u, x @ W1, rtol=1e-13, atol=1e-13)
+    assert np.allclose(z, (x @ W1) @ W2 + b, rtol=1e-13, atol=1e-13)
+    # rank one: only row 3 of W1 and column 2 of W2 are non-zero, so z[..., 2] = x[..., 3] * (W1[3] . W2[:, 2])
+    # and every other column of z is 0
+    W1 = np.zeros((12, 4)); W1[3] = [1.0, 2.0, 0.0, -1.0]
+    W2 = np.zeros((4, 5)); W2[:, 2] = [0.5, 0.25, 7.0, 1.0]
+    z, _ = oracle.gate_proj_fwd(x, W1, W2)
+    assert np.array_equal(z[..., [0, 1, 3, 4]], np.zeros(z.shape[:-1] + (4,)))
+    assert np.allclose(z[..., 2], x[..., 3] * (0.5 + 0.5 + 0.0 - 1.0), atol=1e-15)
+
+
+def _gate_loss(x, W1, W2, b, dla, inv_tau):
+    z, _ = oracle.gate_proj_fwd(x, W1, W2, b)
+    return float(np.sum(dla * inv_tau * _logsig(z)))
+
+
+def test_gate_proj_bwd_matches_finite_differences():
+    rng = np.random.default_rng(91)
+    rows, D, R, dk, inv_tau = 5, 6, 3, 4, 1.0 / 16.0
+    x = rng.standard_normal((rows, D))
+    W1, W2, b = rng.standard_normal((D, R)), rng.standard_normal((R, dk)), rng.standard_normal(dk)
+    dla = rng.standard_normal((rows, dk))
+    z, _ = oracle.gate_proj_fwd(x, W1, W2, b)
+    dx, dW1, dW2, db = oracle.gate_proj_bwd(x, W1, W2, z, dla, inv_tau)
+    h = 1e-6
+    for arr, grad, slot in ((x, dx, 0), (W1, dW1, 1), (W2, dW2, 2), (b, db, 3)):
+        for idx in np.ndindex(arr.shape):
+            args_p = [x, W1, W2, b]
+            args_m = [x, W1, W2, b]
+            p, m = arr.copy(), arr.copy()
+            p[idx] += h
+            m[idx] -= h
+            args_p[slot], args_m[slot] = p, m
+            fd = (_gate_loss(*args_p, dla, inv_tau) - _gate_loss(*args_m, dla, inv_tau)) / (2 * h)
+            assert abs(grad[idx] - fd) <= 1e-7 * max(1.0, abs(fd)), (slot, idx, grad[idx], fd)
