@@ -69,7 +69,11 @@ def algorithmic_bytes(w):
     # conv's (x dY in; dx out); the fp32 parameter vectors are a few KB
     epi_bwd = 5 * vv
     conv_bwd = 3 * BL * w.conv_C * e
-    return {"fwd": fwd, "bwd": bwd, "conv": conv, "epi_bwd": epi_bwd, "conv_bwd": conv_bwd}
+    # the gate projection (D -> rank -> d_k): x in, z and u out; backward x u z dla in, dx out
+    gate_fwd = BL * (w.D * e + w.dk * 4 + w.rank * 4)
+    gate_bwd = BL * (2 * w.D * e + w.rank * 4 + 2 * w.dk * 4)
+    return {"fwd": fwd, "bwd": bwd, "conv": conv, "epi_bwd": epi_bwd, "conv_bwd": conv_bwd,
+            "gate_fwd": gate_fwd, "gate_bwd": gate_bwd}
 
 
 # This library's kernels per op, in launch order, and the sources they are built from.
@@ -79,6 +83,8 @@ OP_KERNELS = {
     "conv": ["srem_dwconv_kernel"],
     "epi_bwd": ["epilogue_bwd_kernel"],
     "conv_bwd": ["srem_dwconv_bwd_kernel"],
+    "gate_fwd": ["gate_proj_fwd_kernel"],
+    "gate_bwd": ["gate_proj_bwd_kernel"],
 }
 STEP_OPS = ("fwd", "bwd", "conv")  # the ops of one timed step
 _CHUNK_SRC = ["gla_chunk.cuh", "gla_common.cuh", "sm100.cuh", "dig_common.cuh", "gla.h"]
@@ -88,9 +94,12 @@ OP_SOURCES = {
     "conv": ["srem.cu", "srem.cuh", "dig_common.cuh", "gla.h"],
     "epi_bwd": ["epilogue_bwd.cu", "gla_common.cuh", "sm100.cuh", "dig_common.cuh", "bwd_ops.h"],
     "conv_bwd": ["srem_bwd.cu", "srem.cuh", "gla_common.cuh", "sm100.cuh", "dig_common.cuh", "bwd_ops.h"],
+    "gate_fwd": ["gate_proj.cu", "gate_proj.h", "gla_common.cuh", "sm100.cuh", "dig_common.cuh"],
+    "gate_bwd": ["gate_proj.cu", "gate_proj.h", "gla_common.cuh", "sm100.cuh", "dig_common.cuh"],
 }
 OP_NAMES = {"fwd": "dig_gla_fwd", "bwd": "dig_gla_bwd_saved", "conv": "dig_srem_reorient_dwconv",
-            "epi_bwd": "dig_epilogue_bwd", "conv_bwd": "dig_srem_reorient_dwconv_bwd"}
+            "epi_bwd": "dig_epilogue_bwd", "conv_bwd": "dig_srem_reorient_dwconv_bwd",
+            "gate_fwd": "dig_gate_proj_fwd", "gate_bwd": "dig_gate_proj_bwd"}
 
 
 def _src_hash(names):
@@ -216,10 +225,17 @@ def _config(w, world):
                    "their own streams overlap the neighbouring steps' compute, two device buffer sets alternate"}
 
 
-def time_backward_ops(dig, w, dev, stream, o, r, dY, xc, wc, flush, warmup, iters):
-    """Mean event-timed seconds of one dig_epilogue_bwd and one
-    dig_srem_reorient_dwconv_bwd call (with d_gamma, dw and dbias)."""
+def time_next_ops(dig, w, dev, stream, o, r, dY, xc, wc, dla, flush, warmup, iters):
+    """Mean event-timed seconds of one call of each op outside the step: the
+    epilogue backward (with d_gamma), the conv backward (with dw, dbias), and the
+    gate projection forward and backward (with u, dW1, dW2, db), on the step's
+    workload with synthetic tensors of its shapes."""
     g = torch.Generator(device=dev).manual_seed(1)
+    xg = torch.randn(w.B * w.L, w.D, device=dev, generator=g).to(xc.dtype)
+    W1 = 0.02 * torch.randn(w.D, w.rank, device=dev, generator=g)
+    W2 = 0.02 * torch.randn(w.rank, w.dk, device=dev, generator=g)
+    zg, ug = torch.empty(w.B * w.L, w.dk, device=dev), torch.empty(w.B * w.L, w.rank, device=dev)
+    dxg, dW1, dW2, dbg = torch.empty_like(xg), torch.empty_like(W1), torch.empty_like(W2), torch.empty(w.dk, device=dev)
     d_o, d_r = torch.empty_like(o), torch.empty_like(o)
     d_gamma = torch.empty(w.dv, device=dev)
     dyc = torch.randn(w.B, w.L, w.conv_C, device=dev, generator=g).to(xc.dtype)
@@ -228,6 +244,9 @@ def time_backward_ops(dig, w, dev, stream, o, r, dY, xc, wc, flush, warmup, iter
     calls = {
         "epi_bwd": lambda i: dig.dig_epilogue_bwd(o, r, dY, d_o, d_r, None, 1e-5, d_gamma, stream=stream),
         "conv_bwd": lambda i: dig.dig_srem_reorient_dwconv_bwd(xc, wc, dyc, dx, i % 4, dw, db, stream=stream),
+        "gate_fwd": lambda i: dig.dig_gate_proj_fwd(xg, W1, W2, zg, None, ug, stream=stream),
+        "gate_bwd": lambda i: dig.dig_gate_proj_bwd(xg, W1, W2, ug, zg, dla.view(-1, w.dk), w.inv_tau, dxg, dW1, dW2,
+                                                    dbg, stream=stream),
     }
     out = {}
     for op, call in calls.items():
@@ -361,9 +380,10 @@ def run_ours(args, rank, world, local_rank):
     e1.synchronize()
     e2e_step_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
 
-    # the backward ops of the epilogue and the conv (outside the step): each timed
-    # alone with CUDA events, L2 flushed before every call, on the bench's workload
-    aux_t = time_backward_ops(dig, w, dev, stream, o, r, dO, xc, wc, flush, args.warmup, max(args.steps, 10))
+    # the ops outside the step (backward of the epilogue and the conv, the gate
+    # projection and its backward): each timed alone with CUDA events, L2 flushed
+    # before every call, on the bench's workload
+    aux_t = time_next_ops(dig, w, dev, stream, o, r, dO, xc, wc, dla, flush, args.warmup, max(args.steps, 10))
     aux_t = {op: max_over_ranks(tv, world, dev) for op, tv in aux_t.items()}
 
     if rank != 0:
@@ -398,7 +418,7 @@ def run_ours(args, rank, world, local_rank):
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": sum(len(OP_KERNELS[op]) for op in STEP_OPS) * args.steps,
         "clocks": clk.summary(),
-        "backward_ops": {OP_NAMES[op]: {"us": t * 1e6, "achieved": algo[op] / t / 1e9, "unit": "GB/s",
+        "next_ops": {OP_NAMES[op]: {"us": t * 1e6, "achieved": algo[op] / t / 1e9, "unit": "GB/s",
                                         "frac": algo[op] / t / 1e9 / hbm, "algorithmic_bytes": algo[op],
                                         "traffic": _traffic(OP_NAMES[op], OP_SOURCES[op], 1.0),
                                         "kernels": OP_KERNELS[op]}

@@ -8,6 +8,7 @@
 #include "../../include/dig.h"
 #include "dig_common.cuh"
 #include "bwd_ops.h"
+#include "gate_proj.h"
 #include "gla.h"
 
 namespace dig {
@@ -261,6 +262,52 @@ dig_status dig_epilogue_bwd(const void* o, const void* r, const float* gamma, fl
   const cudaError_t e = launch_epilogue_bwd(o, r, gamma, eps, dY, d_o, d_r, d_gamma, rows, d_v, dtype, out_dtype,
                                             static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "epilogue backward launch: %s", cudaGetErrorString(e));
+  return DIG_OK;
+}
+
+static dig_status check_gate_shape(long long rows, int D, int R, int d_k, bool backward) {
+  if (rows < 0 || D <= 0 || R <= 0 || d_k <= 0)
+    return fail(DIG_ERR_INVALID_ARGUMENT, "bad size (rows=%lld D=%d R=%d d_k=%d)", rows, D, R, d_k);
+  if (D % 8 != 0 || R > 32 || d_k > 128)
+    return fail(DIG_ERR_UNSUPPORTED, "gate projection built for D %% 8 == 0, R <= 32, d_k <= 128 (D=%d R=%d d_k=%d)",
+                D, R, d_k);
+  if (gate_proj_smem_bytes(D, R, d_k, backward) > 227u * 1024u)
+    return fail(DIG_ERR_UNSUPPORTED, "gate projection weights do not fit shared memory (D=%d R=%d d_k=%d)", D, R,
+                d_k);
+  if (rows >= (1ll << 40) / D) return fail(DIG_ERR_INVALID_ARGUMENT, "tensor too large");
+  return DIG_OK;
+}
+
+dig_status dig_gate_proj_fwd(const void* x, const float* W1, const float* W2, const float* b, float* z, float* u,
+                             long long rows, int D, int R, int d_k, int dtype, void* stream) {
+  const dig_status st = check_gate_shape(rows, D, R, d_k, false);
+  if (st != DIG_OK) return st;
+  if (dtype != DIG_F32 && dtype != DIG_BF16) return fail(DIG_ERR_INVALID_ARGUMENT, "dtype %d not DIG_F32 or DIG_BF16", dtype);
+  if (rows > 0 && (!x || !W1 || !W2 || !z)) return fail(DIG_ERR_INVALID_ARGUMENT, "x, W1, W2 and z must be non-NULL");
+  if (!aligned16(x) || !aligned16(W1) || !aligned16(W2) || !aligned16(b) || !aligned16(z) || !aligned16(u))
+    return fail(DIG_ERR_MISALIGNED, "a tensor pointer is not 16-byte aligned");
+  const cudaError_t e = launch_gate_proj_fwd(x, W1, W2, b, z, u, rows, D, R, d_k, dtype, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "gate projection launch: %s", cudaGetErrorString(e));
+  return DIG_OK;
+}
+
+dig_status dig_gate_proj_bwd(const void* x, const float* W1, const float* W2, const float* u, const float* z,
+                             const float* dlog_alpha, float inv_tau, void* dx, float* dW1, float* dW2, float* db,
+                             long long rows, int D, int R, int d_k, int dtype, int out_dtype, void* stream) {
+  const dig_status st = check_gate_shape(rows, D, R, d_k, true);
+  if (st != DIG_OK) return st;
+  if ((dtype != DIG_F32 && dtype != DIG_BF16) || (out_dtype != DIG_F32 && out_dtype != DIG_BF16))
+    return fail(DIG_ERR_INVALID_ARGUMENT, "dtype %d / out_dtype %d not DIG_F32 or DIG_BF16", dtype, out_dtype);
+  if (!(inv_tau > 0.f && inv_tau < 1e30f)) return fail(DIG_ERR_INVALID_ARGUMENT, "inv_tau must be positive and finite");
+  if (!dW1 || !dW2) return fail(DIG_ERR_INVALID_ARGUMENT, "dW1 and dW2 must be non-NULL");
+  if (rows > 0 && (!x || !W1 || !W2 || !u || !z || !dlog_alpha || !dx))
+    return fail(DIG_ERR_INVALID_ARGUMENT, "x, W1, W2, u, z, dlog_alpha and dx must be non-NULL");
+  if (!aligned16(x) || !aligned16(W1) || !aligned16(W2) || !aligned16(u) || !aligned16(z) || !aligned16(dlog_alpha) ||
+      !aligned16(dx) || !aligned16(dW1) || !aligned16(dW2) || !aligned16(db))
+    return fail(DIG_ERR_MISALIGNED, "a tensor pointer is not 16-byte aligned");
+  const cudaError_t e = launch_gate_proj_bwd(x, W1, W2, u, z, dlog_alpha, inv_tau, dx, dW1, dW2, db, rows, D, R, d_k,
+                                             dtype, out_dtype, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "gate projection backward launch: %s", cudaGetErrorString(e));
   return DIG_OK;
 }
 

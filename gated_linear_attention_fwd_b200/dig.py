@@ -64,6 +64,11 @@ lib.dig_srem_reorient_dwconv_bwd.restype = _i
 lib.dig_srem_reorient_dwconv_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
 lib.dig_epilogue_bwd.restype = _i
 lib.dig_epilogue_bwd.argtypes = [_vp, _vp, _vp, _f, _vp, _vp, _vp, _vp, ctypes.c_longlong, _i, _i, _i, _vp]
+lib.dig_gate_proj_fwd.restype = _i
+lib.dig_gate_proj_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_longlong, _i, _i, _i, _i, _vp]
+lib.dig_gate_proj_bwd.restype = _i
+lib.dig_gate_proj_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp, _vp, ctypes.c_longlong,
+                                  _i, _i, _i, _i, _i, _vp]
 lib.dig_read_status.restype = _i
 lib.dig_read_status.argtypes = [_vp, _vp]
 lib.dig_status_string.restype = ctypes.c_char_p
@@ -197,6 +202,27 @@ def dig_epilogue_bwd(o, r, dY, d_o, d_r, gamma=None, eps=1e-5, d_gamma=None, str
     st = lib.dig_epilogue_bwd(_ptr(o), _ptr(r), _ptr(gamma), float(eps), _ptr(dY), _ptr(d_o), _ptr(d_r),
                               _ptr(d_gamma), rows, d_v, _code(o.dtype), _code(d_o.dtype), _stream(stream))
     _check(st, "dig_epilogue_bwd")
+
+
+def dig_gate_proj_fwd(x, W1, W2, z, b=None, u=None, stream=None):
+    """x [..., D]; W1 [D,R], W2 [R,d_k] fp32; z [..., d_k] fp32; b [d_k] or None; u [..., R] fp32 or None."""
+    D, R = W1.shape
+    d_k = W2.shape[1]
+    rows = x.numel() // D
+    st = lib.dig_gate_proj_fwd(_ptr(x), _ptr(W1), _ptr(W2), _ptr(b), _ptr(z), _ptr(u), rows, D, R, d_k,
+                               _code(x.dtype), _stream(stream))
+    _check(st, "dig_gate_proj_fwd")
+
+
+def dig_gate_proj_bwd(x, W1, W2, u, z, dlog_alpha, inv_tau, dx, dW1, dW2, db=None, stream=None):
+    """Gradients of the gate projection from d log(alpha) (see include/dig.h)."""
+    D, R = W1.shape
+    d_k = W2.shape[1]
+    rows = x.numel() // D
+    st = lib.dig_gate_proj_bwd(_ptr(x), _ptr(W1), _ptr(W2), _ptr(u), _ptr(z), _ptr(dlog_alpha), float(inv_tau),
+                               _ptr(dx), _ptr(dW1), _ptr(dW2), _ptr(db), rows, D, R, d_k, _code(x.dtype),
+                               _code(dx.dtype), _stream(stream))
+    _check(st, "dig_gate_proj_bwd")
 
 
 def dig_read_status(workspace, stream=None) -> int:

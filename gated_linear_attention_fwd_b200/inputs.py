@@ -128,6 +128,20 @@ def make_inputs(w: Workload, seed: int | None = None, with_conv: bool | None = N
     return out
 
 
+def gate_proj_inputs(w: Workload, seed: int, dtype: str | None = None, with_bias: bool = False) -> dict:
+    """Inputs of the gate projection for workload w: x [B, L, D] ~ N(0,1) (stored in
+    the workload's dtype), W1 [D, rank] and W2 [rank, dk] ~ N(0, 0.02^2) and, when
+    asked for, b [dk] ~ N(0, 1), all float32 numpy arrays (bf16-exact x for bf16)."""
+    rng = np.random.default_rng(seed)
+    D = w.D or 384
+    out = {"x": _store(rng.standard_normal((w.B, w.L, D)), dtype or w.dtype),
+           "W1": np.ascontiguousarray(0.02 * rng.standard_normal((D, w.rank)), dtype=np.float32),
+           "W2": np.ascontiguousarray(0.02 * rng.standard_normal((w.rank, w.dk)), dtype=np.float32)}
+    if with_bias:
+        out["b"] = np.ascontiguousarray(rng.standard_normal(w.dk), dtype=np.float32)
+    return out
+
+
 def custom(B, H, grid_h, grid_w, dk, dv, dtype="bf16", gate="direct", inv_tau=1.0 / 16.0,
            D=384, conv_C=0) -> Workload:
     """A workload of arbitrary shape with the same generators (parity edge cases)."""

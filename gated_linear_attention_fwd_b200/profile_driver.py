@@ -14,7 +14,8 @@ from . import dig, inputs
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", choices=["fwd", "bwd", "conv", "epi_bwd", "conv_bwd"], default="fwd")
+    ap.add_argument("--op", choices=["fwd", "bwd", "conv", "epi_bwd", "conv_bwd", "gate_fwd", "gate_bwd"],
+                    default="fwd")
     ap.add_argument("--workload", type=int, default=3)
     ap.add_argument("--iters", type=int, default=4)
     ap.add_argument("--mode", type=int, default=0)
@@ -41,6 +42,23 @@ def main():
         dw, db = torch.empty(C, 3, 3, device="cuda"), torch.empty(C, device="cuda")
         for _ in range(args.iters):
             dig.dig_srem_reorient_dwconv_bwd(x, wc, dy, dx, args.mode, dw, db)
+        torch.cuda.synchronize()
+        print("ok")
+        return
+    if args.op in ("gate_fwd", "gate_bwd"):
+        D, R = w.D or 384, w.rank
+        xg = rnd(B * L, D)
+        W1 = 0.02 * torch.randn(D, R, device="cuda", generator=g)
+        W2 = 0.02 * torch.randn(R, dk, device="cuda", generator=g)
+        zg, ug = torch.empty(B * L, dk, device="cuda"), torch.empty(B * L, R, device="cuda")
+        dig.dig_gate_proj_fwd(xg, W1, W2, zg, None, ug)
+        dla = torch.randn(B * L, dk, device="cuda", generator=g)
+        dxg, dW1, dW2 = torch.empty_like(xg), torch.empty_like(W1), torch.empty_like(W2)
+        for _ in range(args.iters):
+            if args.op == "gate_fwd":
+                dig.dig_gate_proj_fwd(xg, W1, W2, zg, None, ug)
+            else:
+                dig.dig_gate_proj_bwd(xg, W1, W2, ug, zg, dla, w.inv_tau, dxg, dW1, dW2)
         torch.cuda.synchronize()
         print("ok")
         return

@@ -109,6 +109,12 @@ def traffic(args):
     print(json.dumps(d[name], indent=1))
 
 
+def bench_ops():
+    sys.path.insert(0, ROOT)
+    import bench  # noqa: E402
+    return bench.OP_NAMES.keys()
+
+
 def main():
     ap = argparse.ArgumentParser()
     sub = ap.add_subparsers(dest="cmd", required=True)
@@ -118,7 +124,7 @@ def main():
     a.add_argument("--command", required=True)
     t = sub.add_parser("traffic")
     t.add_argument("csv")
-    t.add_argument("--op", choices=["fwd", "bwd", "conv", "epi_bwd", "conv_bwd"], required=True)
+    t.add_argument("--op", choices=sorted(bench_ops()), required=True)
     t.add_argument("--calls", type=int, required=True)
     t.add_argument("--workload", required=True)
     t.add_argument("--command", required=True)

@@ -219,6 +219,35 @@ dig_status dig_epilogue_bwd(const void *o, const void *r, const float *gamma, fl
                             const void *dY, void *d_o, void *d_r, float *d_gamma,
                             long long rows, int d_v, int dtype, int out_dtype, void *stream);
 
+/* Gate projection (slide eq. (5): the gate logits are a projection of the block
+ * input, low-rank in DiG: D -> R -> d_k):
+ *   u = x W1,   z = u W2 + b
+ *   x    [rows, D] dtype          rows = B * L tokens (grid order), D % 8 == 0
+ *   W1   [D, R] fp32;  W2 [R, d_k] fp32;  b [d_k] fp32 or NULL (zero)
+ *   z    [rows, d_k] fp32         the z of dig_gla_fwd with gate_heads = 1
+ *   u    [rows, R] fp32 or NULL   x W1, kept for dig_gate_proj_bwd
+ * Built for R <= 32 and d_k <= 128 with the weights in shared memory (D * R
+ * floats, plus D * R more for the backward, up to 227 KB): DIG_ERR_UNSUPPORTED
+ * otherwise.  Same alignment and stream rules as the other calls. */
+dig_status dig_gate_proj_fwd(const void *x, const float *W1, const float *W2, const float *b,
+                             float *z, float *u, long long rows, int D, int R, int d_k,
+                             int dtype, void *stream);
+
+/* Backward of the gate projection from the GLA backward's dlog_alpha (the gate
+ * is log(alpha) = inv_tau * logsigmoid(z), so dz = dlog_alpha * inv_tau * sigmoid(-z)):
+ *   x, W1, W2   as passed to dig_gate_proj_fwd;  u, z its outputs
+ *   dlog_alpha  [rows, d_k] fp32 (dig_gla_bwd with gate_heads = 1)
+ *   dx          [rows, D] out_dtype:  dz W2^T W1^T
+ *   dW1 [D, R], dW2 [R, d_k], db [d_k] (db may be NULL) fp32: sums over the rows.
+ *               Overwritten (zeroed on `stream` first); the thread blocks' partial
+ *               sums are added with floating-point atomics, so their last bits may
+ *               differ between runs. */
+dig_status dig_gate_proj_bwd(const void *x, const float *W1, const float *W2, const float *u,
+                             const float *z, const float *dlog_alpha, float inv_tau,
+                             void *dx, float *dW1, float *dW2, float *db,
+                             long long rows, int D, int R, int d_k, int dtype, int out_dtype,
+                             void *stream);
+
 /* Synchronises `stream`, returns the device status word kept in `workspace`
  * (DIG_OK, DIG_ERR_DEVICE_TIMEOUT or DIG_ERR_GATE_RANGE) and clears it. */
 dig_status dig_read_status(void *workspace, void *stream);

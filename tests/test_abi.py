@@ -26,7 +26,7 @@ def _fwd(**kw):
 def test_exports_every_declared_function():
     names = dig.header_functions()
     assert {"dig_gla_fwd", "dig_gla_bwd", "dig_srem_reorient_dwconv", "dig_gla_workspace_bytes",
-            "dig_epilogue_bwd", "dig_srem_reorient_dwconv_bwd",
+            "dig_epilogue_bwd", "dig_srem_reorient_dwconv_bwd", "dig_gate_proj_fwd", "dig_gate_proj_bwd",
             "dig_read_status", "dig_status_string", "dig_last_error", "dig_gla_supported"} <= set(names)
     for n in names:
         assert hasattr(dig.lib, n), n
@@ -118,6 +118,29 @@ def test_backward_helpers_reject_bad_arguments_on_host():
     assert C(1024, N, 1024, 1024, N, N, 1, 3, 4, 8, 0, 1, 1, N) == dig.DIG_ERR_INVALID_ARGUMENT
     assert C(1024, 1024, 1024, 1024, 1036, N, 1, 3, 4, 8, 0, 1, 1, N) == dig.DIG_ERR_MISALIGNED
     assert C(1024, 1024, 1024, 1024, N, N, 1, 3, 4, 8, 0, 1, 2, N) == dig.DIG_ERR_INVALID_ARGUMENT
+
+
+def test_gate_projection_rejects_bad_arguments_on_host():
+    F, Bw = dig.lib.dig_gate_proj_fwd, dig.lib.dig_gate_proj_bwd
+    # x, W1, W2, b, z, u, rows, D, R, d_k, dtype, stream
+    assert F(1024, 1024, 1024, N, 1024, N, 4, 0, 16, 32, 1, N) == dig.DIG_ERR_INVALID_ARGUMENT
+    assert F(1024, 1024, 1024, N, 1024, N, 4, 12, 16, 32, 1, N) == dig.DIG_ERR_UNSUPPORTED      # D % 8
+    assert F(1024, 1024, 1024, N, 1024, N, 4, 384, 33, 32, 1, N) == dig.DIG_ERR_UNSUPPORTED     # R > 32
+    assert F(1024, 1024, 1024, N, 1024, N, 4, 384, 16, 129, 1, N) == dig.DIG_ERR_UNSUPPORTED    # d_k > 128
+    assert F(1024, 1024, 1024, N, 1024, N, 4, 8192, 32, 32, 1, N) == dig.DIG_ERR_UNSUPPORTED    # shared memory
+    assert F(1024, 1024, 1024, N, N, N, 4, 384, 16, 32, 1, N) == dig.DIG_ERR_INVALID_ARGUMENT
+    assert F(1024, 1024, 1024, N, 1032, N, 4, 384, 16, 32, 1, N) == dig.DIG_ERR_MISALIGNED
+    assert F(1024, 1024, 1024, N, 1024, N, 4, 384, 16, 32, 9, N) == dig.DIG_ERR_INVALID_ARGUMENT
+    # x, W1, W2, u, z, dla, inv_tau, dx, dW1, dW2, db, rows, D, R, d_k, dtype, out_dtype, stream
+    a = [1024] * 6 + [0.0625] + [1024] * 3 + [N, 4, 384, 16, 32, 1, 1, N]    # valid (not launched here)
+    bad = list(a); bad[6] = 0.0
+    assert Bw(*bad) == dig.DIG_ERR_INVALID_ARGUMENT                                          # inv_tau
+    bad = list(a); bad[8] = N
+    assert Bw(*bad) == dig.DIG_ERR_INVALID_ARGUMENT                                          # dW1
+    bad = list(a); bad[7] = 1040 + 4
+    assert Bw(*bad) == dig.DIG_ERR_MISALIGNED
+    bad = list(a); bad[12] = 20
+    assert Bw(*bad) == dig.DIG_ERR_UNSUPPORTED                                               # D % 8
 
 
 def test_workspace_bytes():
