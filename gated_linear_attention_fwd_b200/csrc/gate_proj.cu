@@ -21,6 +21,8 @@ namespace dig {
 namespace {
 
 constexpr int kTT = 64;  // tokens per tile
+constexpr int kXB = 8;   // forward: 8-value vectors of x loaded ahead per thread
+constexpr int kXT = 16;  // backward dW1: tokens of x loaded ahead per thread
 
 // 8 consecutive values of a row as fp32 (one 16-byte load for bf16, two for fp32)
 __device__ __forceinline__ void load8(const __nv_bfloat16* p, float* v) {
@@ -86,19 +88,26 @@ __global__ void __launch_bounds__(256) gate_proj_fwd_kernel(const TIN* __restric
     for (int j = 0; j < RQ; ++j) acc[j] = 0.f;
     if (row < rows) {
       const TIN* xr = x + (size_t)row * D;
-      for (int d0 = 0; d0 < D; d0 += 8) {
-        float xv[8];
-        load8(xr + d0, xv);
+      // kXB vectors of x in flight per thread before their products
+      for (int c0 = 0; c0 < D; c0 += 8 * kXB) {
+        float xv[kXB][8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float* wrow = W1s + (size_t)(d0 + e) * RT + g * RQ;
+        for (int q = 0; q < kXB; ++q)
+          if (c0 + 8 * q < D) load8(xr + c0 + 8 * q, xv[q]);
 #pragma unroll
-          for (int j = 0; j < RQ; j += 4) {
-            const float4 wv = *reinterpret_cast<const float4*>(wrow + j);
-            acc[j] = fmaf(xv[e], wv.x, acc[j]);
-            acc[j + 1] = fmaf(xv[e], wv.y, acc[j + 1]);
-            acc[j + 2] = fmaf(xv[e], wv.z, acc[j + 2]);
-            acc[j + 3] = fmaf(xv[e], wv.w, acc[j + 3]);
+        for (int q = 0; q < kXB; ++q) {
+          if (c0 + 8 * q >= D) break;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float* wrow = W1s + (size_t)(c0 + 8 * q + e) * RT + g * RQ;
+#pragma unroll
+            for (int j = 0; j < RQ; j += 4) {
+              const float4 wv = *reinterpret_cast<const float4*>(wrow + j);
+              acc[j] = fmaf(xv[q][e], wv.x, acc[j]);
+              acc[j + 1] = fmaf(xv[q][e], wv.y, acc[j + 1]);
+              acc[j + 2] = fmaf(xv[q][e], wv.z, acc[j + 2]);
+              acc[j + 3] = fmaf(xv[q][e], wv.w, acc[j + 3]);
+            }
           }
         }
       }
@@ -236,15 +245,22 @@ __global__ void __launch_bounds__(256) gate_proj_bwd_kernel(const TIN* __restric
       float a[RT];
 #pragma unroll
       for (int r = 0; r < RT; ++r) a[r] = 0.f;
-      for (int t = 0; t < nt; ++t) {
-        const float xv = static_cast<float>(x[(size_t)(row0 + t) * D + d]);
+      // kXT tokens of x in flight per thread; du rows at and past nt are zero
+      for (int t0 = 0; t0 < nt; t0 += kXT) {
+        float xv[kXT];
 #pragma unroll
-        for (int r = 0; r < RT; r += 4) {
-          const float4 g4 = *reinterpret_cast<const float4*>(dus + t * UP + r);
-          a[r] = fmaf(xv, g4.x, a[r]);
-          a[r + 1] = fmaf(xv, g4.y, a[r + 1]);
-          a[r + 2] = fmaf(xv, g4.z, a[r + 2]);
-          a[r + 3] = fmaf(xv, g4.w, a[r + 3]);
+        for (int j = 0; j < kXT; ++j)
+          xv[j] = t0 + j < nt ? static_cast<float>(x[(size_t)(row0 + t0 + j) * D + d]) : 0.f;
+#pragma unroll
+        for (int j = 0; j < kXT; ++j) {
+#pragma unroll
+          for (int r = 0; r < RT; r += 4) {
+            const float4 g4 = *reinterpret_cast<const float4*>(dus + (t0 + j) * UP + r);
+            a[r] = fmaf(xv[j], g4.x, a[r]);
+            a[r + 1] = fmaf(xv[j], g4.y, a[r + 1]);
+            a[r + 2] = fmaf(xv[j], g4.z, a[r + 2]);
+            a[r + 3] = fmaf(xv[j], g4.w, a[r + 3]);
+          }
         }
       }
 #pragma unroll
