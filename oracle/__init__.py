@@ -11,6 +11,9 @@ Parity status of each function (what pins it is in tests/test_oracle_pins.py):
   gla_fwd        pinned: brute-force quadratic form, alpha==1 causal linear
                  attention, alpha->0 diagonal case, constant-gate closed form,
                  causality and linearity
+  gla_fwd_ext    pinned: segment split (the second half started from the first half's
+                 final state equals the whole run), the S0-only closed form
+                 (k = 0), brute-force quadratic form with a value gate
   gla_bwd        pinned: central finite differences of a scalar loss, and the
                  reverse-cumsum identity for d log(alpha)
   srem_dwconv    pinned: scipy.signal.correlate2d, identity kernel = pure
@@ -51,6 +54,9 @@ def _load():
         lib.oracle_gla_fwd.restype = ctypes.c_int
         lib.oracle_gla_fwd.argtypes = [dp, dp, dp, dp, ctypes.c_int, ctypes.c_double, dp,
                                        L, L, L, L, L, L, L, ctypes.c_int]
+        lib.oracle_gla_fwd_ext.restype = ctypes.c_int
+        lib.oracle_gla_fwd_ext.argtypes = [dp, dp, dp, dp, dp, ctypes.c_int, ctypes.c_double, dp, dp, dp,
+                                           L, L, L, L, L, L, L, ctypes.c_int]
         lib.oracle_gla_bwd.restype = ctypes.c_int
         lib.oracle_gla_bwd.argtypes = [dp, dp, dp, dp, ctypes.c_int, ctypes.c_double, dp,
                                        dp, dp, dp, dp, L, L, L, L, L, L, L, ctypes.c_int]
@@ -112,6 +118,25 @@ def gla_fwd(q, k, v, z, inv_tau, grid_h, grid_w, mode):
     if rc:
         raise ValueError("oracle_gla_fwd rejected the arguments (rc=%d)" % rc)
     return o
+
+
+def gla_fwd_ext(q, k, v, z, inv_tau, Hg, Wg, mode, zb=None, S0=None):
+    """The recurrence with a value gate and state I/O: G_t = alpha_t^T beta_t, beta from
+    value-gate logits zb [B,L,Hz,dv] (None: beta = 1), initial state S0 [B,H,dk,dv]
+    (None: 0).  Returns (o [B,L,H,dv], S_final [B,H,dk,dv])."""
+    q, k, v, z = _f64(q), _f64(k), _f64(v), _f64(z)
+    B, L, H, dk = q.shape
+    dv = v.shape[3]
+    gh = z.shape[2]
+    zz = None if zb is None else _f64(zb)
+    s0 = None if S0 is None else _f64(S0)
+    o = np.zeros((B, L, H, dv), dtype=np.float64)
+    sf = np.zeros((B, H, dk, dv), dtype=np.float64)
+    rc = _load().oracle_gla_fwd_ext(_ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(zz), gh, float(inv_tau), _ptr(s0),
+                                    _ptr(o), _ptr(sf), B, H, L, dk, dv, Hg, Wg, int(mode))
+    if rc:
+        raise ValueError("oracle_gla_fwd_ext rejected the arguments")
+    return o, sf
 
 
 def gla_bwd(q, k, v, z, inv_tau, dO, grid_h, grid_w, mode):

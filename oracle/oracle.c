@@ -116,6 +116,56 @@ int oracle_gla_fwd(const double *q, const double *k, const double *v, const doub
     return 0;
 }
 
+/* The recurrence with the general gate and state I/O ([Slides] eq. (5)-(8) before
+ * the value gate is fixed to 1):
+ *   G_t = alpha_t^T beta_t (d_k x d_v),  S_t = G_t (*) S_{t-1} + k_t^T v_t,  o_t = q_t S_t
+ * with beta_t = sigmoid(zb_t)^(1/tau) from value-gate logits zb [B][L][Hz][dv]
+ * (NULL: beta = 1), S_0 from S0 [B*H][dk][dv] (NULL: 0), and the state after the
+ * last scan position written to S_final [B*H][dk][dv] (NULL: not written). */
+int oracle_gla_fwd_ext(const double *q, const double *k, const double *v, const double *z,
+                       const double *zb, int gate_heads, double inv_tau, const double *S0,
+                       double *o, double *S_final,
+                       long B, long H, long L, long dk, long dv, long Hg, long Wg, int mode)
+{
+    if (check_shape(B, H, L, dk, dv, Hg, Wg, mode, gate_heads)) return 1;
+    long n = B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < n; ++bh) {
+        long b = bh / H, h = bh % H, hz = (gate_heads == 1) ? 0 : h;
+        double *S = (double *)calloc((size_t)(dk * dv), sizeof(double));
+        double *alpha = (double *)malloc((size_t)dk * sizeof(double));
+        double *beta = (double *)malloc((size_t)dv * sizeof(double));
+        if (S0)
+            for (long e = 0; e < dk * dv; ++e) S[e] = S0[bh * dk * dv + e];
+        for (long t = 0; t < L; ++t) {
+            long g = oracle_scan_index(mode, Hg, Wg, t);
+            const double *qt = q + ((b * L + g) * H + h) * dk;
+            const double *kt = k + ((b * L + g) * H + h) * dk;
+            const double *vt = v + ((b * L + g) * H + h) * dv;
+            const double *zt = z + ((b * L + g) * gate_heads + hz) * dk;
+            double *ot = o + ((b * L + g) * H + h) * dv;
+            for (long c = 0; c < dk; ++c) alpha[c] = exp(inv_tau * log_sigmoid(zt[c]));
+            for (long j = 0; j < dv; ++j)
+                beta[j] = zb ? exp(inv_tau * log_sigmoid(zb[((b * L + g) * gate_heads + hz) * dv + j])) : 1.0;
+            /* S_t = (alpha_t^T beta_t) (*) S_{t-1} + k_t^T v_t */
+            for (long c = 0; c < dk; ++c)
+                for (long j = 0; j < dv; ++j)
+                    S[c * dv + j] = alpha[c] * beta[j] * S[c * dv + j] + kt[c] * vt[j];
+            for (long j = 0; j < dv; ++j) {
+                double acc = 0.0;
+                for (long c = 0; c < dk; ++c) acc += qt[c] * S[c * dv + j];
+                ot[j] = acc;
+            }
+        }
+        if (S_final)
+            for (long e = 0; e < dk * dv; ++e) S_final[bh * dk * dv + e] = S[e];
+        free(S);
+        free(alpha);
+        free(beta);
+    }
+    return 0;
+}
+
 /* Backward of the recurrence: a reverse sweep over the scan order carrying
  * dS = dLoss/dS_t.  The forward states are rebuilt from checkpoints taken every
  * CK steps.  dlogalpha is the gradient with respect to log(alpha_t); with one

@@ -480,3 +480,81 @@ def test_gate_proj_bwd_matches_finite_differences():
             args_p[slot], args_m[slot] = p, m
             fd = (_gate_loss(*args_p, dla, inv_tau) - _gate_loss(*args_m, dla, inv_tau)) / (2 * h)
             assert abs(grad[idx] - fd) <= 1e-7 * max(1.0, abs(fd)), (slot, idx, grad[idx], fd)
+
+
+# ----------------------------------------------------------------------------- value gate and state I/O
+
+def _quadratic_beta(q, k, v, z, zb, inv_tau, Hg, Wg, mode):
+    """Brute force with G_t = alpha_t^T beta_t: o_t[j] = sum_{s<=t} sum_c q_t[c] k_s[c] v_s[j]
+    prod_{s<u<=t} alpha_u[c] beta_u[j]."""
+    B, L, H, dk = q.shape
+    dv = v.shape[3]
+    perm = oracle.scan_index(mode, Hg, Wg)
+    o = np.zeros((B, L, H, dv))
+    for b in range(B):
+        for h in range(H):
+            hz = 0 if z.shape[2] == 1 else h
+            alpha = np.exp(inv_tau * _logsig(z[b, perm, hz, :]))
+            beta = np.exp(inv_tau * _logsig(zb[b, perm, hz, :]))
+            for t in range(L):
+                acc = np.zeros(dv)
+                for s in range(t + 1):
+                    da, db_ = np.ones(dk), np.ones(dv)
+                    for u in range(s + 1, t + 1):
+                        da, db_ = da * alpha[u], db_ * beta[u]
+                    acc += float(np.sum(q[b, perm[t], h] * da * k[b, perm[s], h])) * (db_ * v[b, perm[s], h])
+                o[b, perm[t], h] = acc
+    return o
+
+
+@pytest.mark.parametrize("mode", range(4))
+@pytest.mark.parametrize("gate_heads", [1, 2])
+def test_fwd_ext_value_gate_matches_quadratic_form(mode, gate_heads):
+    rng = np.random.default_rng(400 + mode + 10 * gate_heads)
+    q, k, v, z = _problem(rng, gate_heads=gate_heads)
+    zb = 2.0 * rng.standard_normal(z.shape[:3] + (v.shape[3],))
+    o, _ = oracle.gla_fwd_ext(q, k, v, z, 0.5, 3, 4, mode, zb=zb)
+    ref = _quadratic_beta(q, k, v, z, zb, 0.5, 3, 4, mode)
+    assert np.max(np.abs(o - ref)) <= 1e-12 * max(1.0, np.max(np.abs(ref)))
+
+
+def test_fwd_ext_without_value_gate_or_state_is_the_plain_recurrence():
+    rng = np.random.default_rng(410)
+    q, k, v, z = _problem(rng)
+    o, _ = oracle.gla_fwd_ext(q, k, v, z, 1.0 / 16.0, 3, 4, 2)
+    assert np.array_equal(o, oracle.gla_fwd(q, k, v, z, 1.0 / 16.0, 3, 4, 2))
+
+
+def test_fwd_ext_initial_state_closed_form():
+    # k = 0: the state is S0 decayed, S_t = (prod alpha)^T (prod beta) (*) S0, so
+    # o_t[j] = sum_c q_t[c] S0[c, j] prod_{u<=t} alpha_u[c] beta_u[j]
+    rng = np.random.default_rng(411)
+    q, k, v, z = _problem(rng, B=1, H=2, Hg=1, Wg=7, dk=3, dv=4)
+    zb = rng.standard_normal(z.shape[:3] + (4,))
+    S0 = rng.standard_normal((1, 2, 3, 4))
+    o, sf = oracle.gla_fwd_ext(q, np.zeros_like(k), v, z, 0.5, 1, 7, 0, zb=zb, S0=S0)
+    pa = np.cumprod(np.exp(0.5 * _logsig(z[0, :, 0, :])), axis=0)     # [L, dk]
+    pb = np.cumprod(np.exp(0.5 * _logsig(zb[0, :, 0, :])), axis=0)    # [L, dv]
+    for h in range(2):
+        ref = np.einsum("tc,cj,tc,tj->tj", q[0, :, h], S0[0, h], pa, pb)
+        assert np.allclose(o[0, :, h], ref, rtol=1e-13, atol=1e-14)
+        assert np.allclose(sf[0, h], S0[0, h] * np.outer(pa[-1], pb[-1]), rtol=1e-13, atol=1e-14)
+
+
+@pytest.mark.parametrize("with_beta", [False, True])
+def test_fwd_ext_segment_split_continues_the_state(with_beta):
+    # one row of tokens (scan order = token order): the second segment started from the
+    # first segment's final state gives the whole run's outputs and final state
+    rng = np.random.default_rng(412 + with_beta)
+    L, L1 = 11, 5
+    q, k, v, z = _problem(rng, B=2, H=2, Hg=1, Wg=L, dk=3, dv=4)
+    zb = rng.standard_normal(z.shape[:3] + (4,)) if with_beta else None
+    o, sf = oracle.gla_fwd_ext(q, k, v, z, 0.25, 1, L, 0, zb=zb)
+    part = lambda a, sl: None if a is None else np.ascontiguousarray(a[:, sl])
+    o1, s1 = oracle.gla_fwd_ext(part(q, slice(0, L1)), part(k, slice(0, L1)), part(v, slice(0, L1)),
+                                part(z, slice(0, L1)), 0.25, 1, L1, 0, zb=part(zb, slice(0, L1)))
+    o2, s2 = oracle.gla_fwd_ext(part(q, slice(L1, L)), part(k, slice(L1, L)), part(v, slice(L1, L)),
+                                part(z, slice(L1, L)), 0.25, 1, L - L1, 0, zb=part(zb, slice(L1, L)), S0=s1)
+    assert np.allclose(o[:, :L1], o1, rtol=1e-13, atol=1e-13)
+    assert np.allclose(o[:, L1:], o2, rtol=1e-12, atol=1e-12)
+    assert np.allclose(sf, s2, rtol=1e-12, atol=1e-12)
