@@ -14,6 +14,8 @@ Parity status of each function (what pins it is in tests/test_oracle_pins.py):
   gla_fwd_ext    pinned: segment split (the second half started from the first half's
                  final state equals the whole run), the S0-only closed form
                  (k = 0), brute-force quadratic form with a value gate
+  gla_bwd_ext    pinned: central finite differences of sum(o * dO) + sum(S_final * dSf)
+                 in q, k, v, z, zb and S0, across checkpoint blocks
   gla_bwd        pinned: central finite differences of a scalar loss, and the
                  reverse-cumsum identity for d log(alpha)
   srem_dwconv    pinned: scipy.signal.correlate2d, identity kernel = pure
@@ -57,6 +59,9 @@ def _load():
         lib.oracle_gla_fwd_ext.restype = ctypes.c_int
         lib.oracle_gla_fwd_ext.argtypes = [dp, dp, dp, dp, dp, ctypes.c_int, ctypes.c_double, dp, dp, dp,
                                            L, L, L, L, L, L, L, ctypes.c_int]
+        lib.oracle_gla_bwd_ext.restype = ctypes.c_int
+        lib.oracle_gla_bwd_ext.argtypes = [dp, dp, dp, dp, dp, ctypes.c_int, ctypes.c_double, dp, dp, dp,
+                                           dp, dp, dp, dp, dp, dp, L, L, L, L, L, L, L, ctypes.c_int]
         lib.oracle_gla_bwd.restype = ctypes.c_int
         lib.oracle_gla_bwd.argtypes = [dp, dp, dp, dp, ctypes.c_int, ctypes.c_double, dp,
                                        dp, dp, dp, dp, L, L, L, L, L, L, L, ctypes.c_int]
@@ -137,6 +142,28 @@ def gla_fwd_ext(q, k, v, z, inv_tau, Hg, Wg, mode, zb=None, S0=None):
     if rc:
         raise ValueError("oracle_gla_fwd_ext rejected the arguments")
     return o, sf
+
+
+def gla_bwd_ext(q, k, v, z, inv_tau, dO, Hg, Wg, mode, zb=None, S0=None, dSf=None):
+    """Gradients of sum(o * dO) + sum(S_final * dSf) for gla_fwd_ext.  Returns
+    (dq, dk, dv, dlogalpha, dlogbeta or None, dS0 [B,H,dk,dv])."""
+    q, k, v, z, dO = _f64(q), _f64(k), _f64(v), _f64(z), _f64(dO)
+    B, L, H, dk = q.shape
+    dv = v.shape[3]
+    gh = z.shape[2]
+    zz = None if zb is None else _f64(zb)
+    s0 = None if S0 is None else _f64(S0)
+    dsf = None if dSf is None else _f64(dSf)
+    dq, dkk, dvv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    dla = np.zeros_like(z)
+    dlb = None if zb is None else np.zeros((B, L, gh, dv), dtype=np.float64)
+    ds0 = np.zeros((B, H, dk, dv), dtype=np.float64)
+    rc = _load().oracle_gla_bwd_ext(_ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(zz), gh, float(inv_tau), _ptr(s0),
+                                    _ptr(dO), _ptr(dsf), _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dla), _ptr(dlb),
+                                    _ptr(ds0), B, H, L, dk, dv, Hg, Wg, int(mode))
+    if rc:
+        raise ValueError("oracle_gla_bwd_ext rejected the arguments (rc=%d)" % rc)
+    return dq, dkk, dvv, dla, dlb, ds0
 
 
 def gla_bwd(q, k, v, z, inv_tau, dO, grid_h, grid_w, mode):

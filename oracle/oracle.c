@@ -516,3 +516,138 @@ int oracle_gate_proj_bwd(const double *x, const double *W1, const double *W2, co
     free(u); free(du); free(dz);
     return 0;
 }
+
+/* Backward of oracle_gla_fwd_ext: gradients of sum_t o_t . dO_t + sum S_final (*) dSf
+ * (dSf [B*H][dk][dv], NULL = 0).  Reverse sweep carrying dS = dLoss/dS_t:
+ *   dS += q_t^T dO_t;  dq_t = dO_t S_t^T;  dk_t = v_t dS^T;  dv_t = k_t dS;
+ *   dlog(alpha_t)[c] = sum_j dS[c][j] G_t[c][j] S_{t-1}[c][j],
+ *   dlog(beta_t)[j]  = sum_c dS[c][j] G_t[c][j] S_{t-1}[c][j],
+ *   dS <- G_t (*) dS  (the gradient of S_{t-1});  after t = 0 it is dS0.
+ * Forward states are rebuilt from checkpoints every CK steps.  dlogalpha
+ * [B][L][Hz][dk] and dlogbeta [B][L][Hz][dv] (NULL: not formed) are summed over
+ * heads for a shared gate; dS0 [B*H][dk][dv] may be NULL. */
+int oracle_gla_bwd_ext(const double *q, const double *k, const double *v, const double *z,
+                       const double *zb, int gate_heads, double inv_tau, const double *S0,
+                       const double *dO, const double *dSf,
+                       double *dq, double *dk_out, double *dv_out, double *dlogalpha,
+                       double *dlogbeta, double *dS0,
+                       long B, long H, long L, long dk, long dv, long Hg, long Wg, int mode)
+{
+    if (check_shape(B, H, L, dk, dv, Hg, Wg, mode, gate_heads)) return 1;
+    long n = B * H;
+    long nblk = (L + CK - 1) / CK;
+    double *dla_h = (double *)calloc((size_t)(B * H * L * dk) + 1, sizeof(double));
+    double *dlb_h = (double *)calloc((size_t)(B * H * L * dv) + 1, sizeof(double));
+    if (!dla_h || !dlb_h) { free(dla_h); free(dlb_h); return 2; }
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < n; ++bh) {
+        long b = bh / H, h = bh % H, hz = (gate_heads == 1) ? 0 : h;
+        size_t ssz = (size_t)(dk * dv);
+        double *ckpt = (double *)calloc(ssz * (size_t)(nblk + 1), sizeof(double));
+        double *blk = (double *)malloc(ssz * CK * sizeof(double));
+        double *S = (double *)calloc(ssz, sizeof(double));
+        double *dS = (double *)calloc(ssz, sizeof(double));
+        double *G = (double *)malloc(ssz * sizeof(double));
+        /* the gate of token g: G[c][j] = alpha[c] beta[j] */
+        #define EXT_GATE(g_)                                                                        \
+            for (long c = 0; c < dk; ++c) {                                                         \
+                double a_ = exp(inv_tau * log_sigmoid(z[((b * L + (g_)) * gate_heads + hz) * dk + c])); \
+                for (long j = 0; j < dv; ++j)                                                       \
+                    G[c * dv + j] = a_ * (zb ? exp(inv_tau * log_sigmoid(                           \
+                                                   zb[((b * L + (g_)) * gate_heads + hz) * dv + j])) \
+                                             : 1.0);                                                \
+            }
+        if (S0) memcpy(S, S0 + bh * ssz, ssz * sizeof(double));
+        for (long t = 0; t < L; ++t) {
+            if (t % CK == 0) memcpy(ckpt + (size_t)(t / CK) * ssz, S, ssz * sizeof(double));
+            long g = oracle_scan_index(mode, Hg, Wg, t);
+            const double *kt = k + ((b * L + g) * H + h) * dk;
+            const double *vt = v + ((b * L + g) * H + h) * dv;
+            EXT_GATE(g)
+            for (long c = 0; c < dk; ++c)
+                for (long j = 0; j < dv; ++j) S[c * dv + j] = G[c * dv + j] * S[c * dv + j] + kt[c] * vt[j];
+        }
+        if (dSf) memcpy(dS, dSf + bh * ssz, ssz * sizeof(double));
+        for (long m = nblk - 1; m >= 0; --m) {
+            long t0 = m * CK, t1 = (t0 + CK < L) ? t0 + CK : L;
+            memcpy(S, ckpt + (size_t)m * ssz, ssz * sizeof(double));
+            for (long t = t0; t < t1; ++t) {
+                long g = oracle_scan_index(mode, Hg, Wg, t);
+                const double *kt = k + ((b * L + g) * H + h) * dk;
+                const double *vt = v + ((b * L + g) * H + h) * dv;
+                EXT_GATE(g)
+                for (long c = 0; c < dk; ++c)
+                    for (long j = 0; j < dv; ++j) S[c * dv + j] = G[c * dv + j] * S[c * dv + j] + kt[c] * vt[j];
+                memcpy(blk + (size_t)(t - t0) * ssz, S, ssz * sizeof(double));
+            }
+            for (long t = t1 - 1; t >= t0; --t) {
+                long g = oracle_scan_index(mode, Hg, Wg, t);
+                const double *qt = q + ((b * L + g) * H + h) * dk;
+                const double *kt = k + ((b * L + g) * H + h) * dk;
+                const double *vt = v + ((b * L + g) * H + h) * dv;
+                const double *dot = dO + ((b * L + g) * H + h) * dv;
+                const double *St = blk + (size_t)(t - t0) * ssz;
+                const double *Sp = (t > t0) ? blk + (size_t)(t - 1 - t0) * ssz : ckpt + (size_t)m * ssz;
+                double *dqt = dq + ((b * L + g) * H + h) * dk;
+                double *dkt = dk_out + ((b * L + g) * H + h) * dk;
+                double *dvt = dv_out + ((b * L + g) * H + h) * dv;
+                double *dlat = dla_h + ((b * H + h) * L + g) * dk;
+                double *dlbt = dlb_h + ((b * H + h) * L + g) * dv;
+                EXT_GATE(g)
+                for (long c = 0; c < dk; ++c)
+                    for (long j = 0; j < dv; ++j) dS[c * dv + j] += qt[c] * dot[j];
+                for (long c = 0; c < dk; ++c) {
+                    double acc = 0.0;
+                    for (long j = 0; j < dv; ++j) acc += dot[j] * St[c * dv + j];
+                    dqt[c] = acc;
+                }
+                for (long c = 0; c < dk; ++c) {
+                    double acc = 0.0;
+                    for (long j = 0; j < dv; ++j) acc += dS[c * dv + j] * vt[j];
+                    dkt[c] = acc;
+                }
+                for (long j = 0; j < dv; ++j) {
+                    double acc = 0.0;
+                    for (long c = 0; c < dk; ++c) acc += kt[c] * dS[c * dv + j];
+                    dvt[j] = acc;
+                }
+                for (long c = 0; c < dk; ++c) dlat[c] = 0.0;
+                for (long j = 0; j < dv; ++j) dlbt[j] = 0.0;
+                for (long c = 0; c < dk; ++c)
+                    for (long j = 0; j < dv; ++j) {
+                        double w = dS[c * dv + j] * G[c * dv + j] * Sp[c * dv + j];
+                        dlat[c] += w;
+                        dlbt[j] += w;
+                    }
+                for (long e = 0; e < (long)ssz; ++e) dS[e] *= G[e];
+            }
+        }
+        if (dS0) memcpy(dS0 + bh * ssz, dS, ssz * sizeof(double));
+        #undef EXT_GATE
+        free(ckpt); free(blk); free(S); free(dS); free(G);
+    }
+    long Hz = gate_heads;
+    if (dlogalpha)
+        for (long b = 0; b < B; ++b)
+            for (long g = 0; g < L; ++g)
+                for (long hz = 0; hz < Hz; ++hz)
+                    for (long c = 0; c < dk; ++c) {
+                        double acc = 0.0;
+                        for (long h = 0; h < H; ++h)
+                            if (Hz == 1 || h == hz) acc += dla_h[((b * H + h) * L + g) * dk + c];
+                        dlogalpha[((b * L + g) * Hz + hz) * dk + c] = acc;
+                    }
+    if (dlogbeta)
+        for (long b = 0; b < B; ++b)
+            for (long g = 0; g < L; ++g)
+                for (long hz = 0; hz < Hz; ++hz)
+                    for (long j = 0; j < dv; ++j) {
+                        double acc = 0.0;
+                        for (long h = 0; h < H; ++h)
+                            if (Hz == 1 || h == hz) acc += dlb_h[((b * H + h) * L + g) * dv + j];
+                        dlogbeta[((b * L + g) * Hz + hz) * dv + j] = acc;
+                    }
+    free(dla_h);
+    free(dlb_h);
+    return 0;
+}

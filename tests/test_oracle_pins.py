@@ -31,6 +31,10 @@ def _problem(rng, B=2, H=2, Hg=3, Wg=4, dk=3, dv=4, gate_heads=1, zscale=2.0):
     return q, k, v, z
 
 
+def _sig(x):
+    return 1.0 / (1.0 + np.exp(-x))
+
+
 def _logsig(x):
     return -np.logaddexp(0.0, -x)
 
@@ -558,3 +562,41 @@ def test_fwd_ext_segment_split_continues_the_state(with_beta):
     assert np.allclose(o[:, :L1], o1, rtol=1e-13, atol=1e-13)
     assert np.allclose(o[:, L1:], o2, rtol=1e-12, atol=1e-12)
     assert np.allclose(sf, s2, rtol=1e-12, atol=1e-12)
+
+
+def _ext_loss(q, k, v, z, zb, S0, dO, dSf, inv_tau, Hg, Wg, mode):
+    o, sf = oracle.gla_fwd_ext(q, k, v, z, inv_tau, Hg, Wg, mode, zb=zb, S0=S0)
+    return float(np.sum(o * dO) + np.sum(sf * dSf))
+
+
+@pytest.mark.parametrize("mode,gate_heads,hw,sample", [(0, 1, (3, 4), None), (3, 2, (3, 4), None),
+                                                       (2, 1, (7, 10), 12)])
+def test_bwd_ext_matches_finite_differences(mode, gate_heads, hw, sample):
+    """Every gradient of the value-gate / state-I/O recurrence, including an incoming
+    final-state gradient; the 70-token case crosses the backward's checkpoint blocks
+    (sampled elements)."""
+    rng = np.random.default_rng(500 + mode + 10 * gate_heads)
+    Hg, Wg = hw
+    inv_tau = 0.5
+    q, k, v, z = _problem(rng, B=1, H=2, Hg=Hg, Wg=Wg, dk=3, dv=4, gate_heads=gate_heads)
+    zb = rng.standard_normal(z.shape[:3] + (4,))
+    S0 = rng.standard_normal((1, 2, 3, 4))
+    dO = rng.standard_normal(v.shape)
+    dSf = rng.standard_normal((1, 2, 3, 4))
+    dq, dk_, dv_, dla, dlb, dS0 = oracle.gla_bwd_ext(q, k, v, z, inv_tau, dO, Hg, Wg, mode, zb=zb, S0=S0, dSf=dSf)
+    grads = {"q": dq, "k": dk_, "v": dv_, "z": dla * inv_tau * _sig(-z), "zb": dlb * inv_tau * _sig(-zb), "S0": dS0}
+    args = {"q": q, "k": k, "v": v, "z": z, "zb": zb, "S0": S0}
+    h = 1e-6
+    for name, arr in args.items():
+        idxs = list(np.ndindex(arr.shape))
+        if sample:
+            idxs = [idxs[i] for i in rng.choice(len(idxs), size=min(sample, len(idxs)), replace=False)]
+        for idx in idxs:
+            p, m = dict(args), dict(args)
+            p[name], m[name] = arr.copy(), arr.copy()
+            p[name][idx] += h
+            m[name][idx] -= h
+            fd = (_ext_loss(p["q"], p["k"], p["v"], p["z"], p["zb"], p["S0"], dO, dSf, inv_tau, Hg, Wg, mode) -
+                  _ext_loss(m["q"], m["k"], m["v"], m["z"], m["zb"], m["S0"], dO, dSf, inv_tau, Hg, Wg, mode)) / (2 * h)
+            got = grads[name][idx]
+            assert abs(got - fd) <= 1e-6 * max(1.0, abs(fd)), (name, idx, got, fd)
