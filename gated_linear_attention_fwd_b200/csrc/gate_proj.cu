@@ -40,6 +40,27 @@ __device__ __forceinline__ void load8(const float* p, float* v) {
   v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w, v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
 }
 
+// Copies a weight matrix into shared memory in the layout `dst[i] = src_at(i)` (0
+// where src_at returns a negative index), i < n, with 8 loads in flight per
+// thread: the copy costs a few memory round trips instead of one per element.
+template <typename F>
+__device__ __forceinline__ void stage_weights(float* dst, const float* __restrict__ src, int n, F src_at) {
+  for (int i0 = threadIdx.x; i0 < n; i0 += 8 * blockDim.x) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * blockDim.x;
+      const long long j = i < n ? src_at(i) : -1;
+      v[u] = j >= 0 ? __ldg(src + j) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * blockDim.x;
+      if (i < n) dst[i] = v[u];
+    }
+  }
+}
+
 __device__ __forceinline__ float sigmoid_neg(float z) {  // sigmoid(-z)
   return __fdividef(1.f, 1.f + ex2(z * kLog2e));
 }
@@ -69,14 +90,14 @@ __global__ void __launch_bounds__(256) gate_proj_fwd_kernel(const TIN* __restric
   float* us = W2s + (size_t)RT * dk;            // [kTT][RT + 1]
   griddep_wait();  // the kernels before this one have completed
   griddep_launch_dependents();
-  for (int i = threadIdx.x; i < D * RT; i += blockDim.x) {
+  stage_weights(W1s, W1, D * RT, [&](int i) -> long long {
     const int d = i / RT, r = i % RT;
-    W1s[i] = r < R ? W1[(size_t)d * R + r] : 0.f;
-  }
-  for (int i = threadIdx.x; i < RT * dk; i += blockDim.x) {
+    return r < R ? (long long)d * R + r : -1;
+  });
+  stage_weights(W2s, W2, RT * dk, [&](int i) -> long long {
     const int r = i / dk, k = i % dk;
-    W2s[i] = r < R ? W2[(size_t)r * dk + k] : 0.f;
-  }
+    return r < R ? (long long)r * dk + k : -1;
+  });
   __syncthreads();
   const int tl = threadIdx.x >> 2, g = threadIdx.x & 3;
   const long long ntiles = (rows + kTT - 1) / kTT;
@@ -174,15 +195,15 @@ __global__ void __launch_bounds__(256) gate_proj_bwd_kernel(const TIN* __restric
   float* dus = us + (size_t)kTT * UP;          // [kTT][UP]
   griddep_wait();  // the kernels before this one have completed
   griddep_launch_dependents();
-  for (int i = threadIdx.x; i < RT * D; i += blockDim.x) {
+  stage_weights(W1T, W1, RT * D, [&](int i) -> long long {
     const int r = i / D, d = i % D;
-    W1T[i] = r < R ? W1[(size_t)d * R + r] : 0.f;
-    G1T[i] = 0.f;
-  }
-  for (int i = threadIdx.x; i < dk * RT; i += blockDim.x) {
+    return r < R ? (long long)d * R + r : -1;
+  });
+  for (int i = threadIdx.x; i < RT * D; i += blockDim.x) G1T[i] = 0.f;
+  stage_weights(W2T, W2, dk * RT, [&](int i) -> long long {
     const int k = i / RT, r = i % RT;
-    W2T[i] = r < R ? W2[(size_t)r * dk + k] : 0.f;
-  }
+    return r < R ? (long long)r * dk + k : -1;
+  });
   float g2[NW2], gb = 0.f;
 #pragma unroll
   for (int j = 0; j < NW2; ++j) g2[j] = 0.f;
