@@ -383,8 +383,13 @@ def run_ours(args, rank, world, local_rank):
     # the ops outside the step (backward of the epilogue and the conv, the gate
     # projection and its backward): each timed alone with CUDA events, L2 flushed
     # before every call, on the bench's workload
-    aux_t = time_next_ops(dig, w, dev, stream, o, r, dO, xc, wc, dla, flush, args.warmup, max(args.steps, 10))
-    aux_t = {op: max_over_ranks(tv, world, dev) for op, tv in aux_t.items()}
+    # (an error there is reported in the line instead of costing the step's numbers)
+    try:
+        aux_t = time_next_ops(dig, w, dev, stream, o, r, dO, xc, wc, dla, flush, args.warmup, max(args.steps, 10))
+        aux_t = {op: max_over_ranks(tv, world, dev) for op, tv in aux_t.items()}
+        aux_err = None
+    except Exception as e:  # noqa: BLE001
+        aux_t, aux_err = {}, "%s: %s" % (type(e).__name__, str(e).splitlines()[0] if str(e) else "")
 
     if rank != 0:
         return None
@@ -422,7 +427,7 @@ def run_ours(args, rank, world, local_rank):
                                         "frac": algo[op] / t / 1e9 / hbm, "algorithmic_bytes": algo[op],
                                         "traffic": _traffic(OP_NAMES[op], OP_SOURCES[op], 1.0),
                                         "kernels": OP_KERNELS[op]}
-                         for op, t in aux_t.items()},
+                         for op, t in aux_t.items()} if aux_err is None else {"error": aux_err},
     }
     if world == 1 and not args.no_cpu_baseline:
         tps, dt, cores, n = cpu_sample(w, x, steps=1, min_seconds=10.0)
