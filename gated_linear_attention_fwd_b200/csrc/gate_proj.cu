@@ -67,8 +67,8 @@ __device__ __forceinline__ float sigmoid_neg(float z) {  // sigmoid(-z)
 
 }  // namespace
 
-// Shared memory of the forward (floats): W1 [D][RT] (columns >= R zero), W2 [RT][dk]
-// (rows >= R zero), u [kTT][RT + 1].
+// Dynamic shared memory of the forward, in bytes: fp32 W1 [D][RT] (columns >= R
+// zero), W2 [RT][dk] (rows >= R zero) and u [kTT][RT + 1].
 inline size_t gate_fwd_smem(int D, int RT, int dk) {
   return 4 * ((size_t)D * RT + (size_t)RT * dk + (size_t)kTT * (RT + 1));
 }
@@ -153,9 +153,9 @@ __global__ void __launch_bounds__(256) gate_proj_fwd_kernel(const TIN* __restric
   }
 }
 
-// Shared memory of the backward (floats): W1^T [RT][D], dW1^T partials [RT][D],
-// W2^T [dk][RT], dz [kTT][dk + 1], u and du [kTT][RT + 4] each (rows of u and du
-// start on 16-byte boundaries).
+// Dynamic shared memory of the backward, in bytes: fp32 W1^T [RT][D], dW1^T
+// partials [RT][D], W2^T [dk][RT], dz [kTT][dk + 1], u and du [kTT][RT + 4] each
+// (rows of u and du start on 16-byte boundaries).
 inline size_t gate_bwd_smem(int D, int RT, int dk) {
   return 4 * (2 * (size_t)RT * D + (size_t)dk * RT + (size_t)kTT * (dk + 1) + 2 * (size_t)kTT * (RT + 4));
 }
