@@ -76,6 +76,17 @@ def algorithmic_bytes(w):
             "gate_fwd": gate_fwd, "gate_bwd": gate_bwd}
 
 
+def metric_bytes(w):
+    """Bytes of the metric's GLA fwd and bwd with d log(alpha) counted once per head
+    (the per-token-head convention of the metric's roofline): fwd reads q k v z and
+    writes o; bwd reads q k v z dO and writes dq dk dv and a per-head d log(alpha)."""
+    BL, H, dk, dv = w.B * w.L, w.H, w.dk, w.dv
+    e = 2
+    fwd = BL * (H * (2 * dk + 2 * dv) * e + dk * 4)
+    bwd = BL * (H * (2 * dk + 2 * dv) * e + dk * 4 + H * (2 * dk + dv) * e + H * dk * 4)
+    return fwd, bwd
+
+
 # This library's kernels per op, in launch order, and the sources they are built from.
 OP_KERNELS = {
     "fwd": ["gla_gate_kernel", "gla_chunk_state_kernel", "gla_state_scan_kernel", "gla_chunk_out_kernel"],
@@ -263,6 +274,94 @@ def time_next_ops(dig, w, dev, stream, o, r, dY, xc, wc, dla, flush, warmup, ite
     return out
 
 
+# The metric's three shapes: L = 4096 (DiG-S/2 1024^2), 12544 (DiG-S/2 1792^2, the step
+# above) and 16384 (DiG-XL/2 2048^2).
+PER_CONFIG = (2, 3, 4)
+
+
+def time_gla_config(dig, index, dev, stream, flush, warmup, iters, seed_offset=0):
+    """Event-timed mean seconds of dig_gla_fwd (bf16 o; with the Swish*RMSNorm epilogue
+    where the workload has it) and of dig_gla_bwd_saved (bf16 dq dk dv) on one workload,
+    L2 flushed before every call pair, scan mode cycling."""
+    w = inputs.WORKLOADS[index]
+    x = inputs.make_inputs(w, seed=inputs.SEED_BASE + index + seed_offset, with_conv=False)
+    t = lambda a, dt=torch.bfloat16: torch.from_numpy(a).to(dev).to(dt).contiguous()
+    q, k, v, dO = t(x["q"]), t(x["k"]), t(x["v"]), t(x["dO"])
+    z = t(x["z"], torch.float32)
+    r = t(x["r"]) if w.epilogue else None
+    B, L, H = w.B, w.L, w.H
+    o = torch.empty(B, L, H, w.dv, device=dev, dtype=torch.bfloat16)
+    y = torch.empty_like(o) if w.epilogue else None
+    dq, dk_, dv_, dla = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(z)
+    ws_f = dig.new_workspace(B, H, L, w.dk, w.dv, device=dev)
+    ws_b = dig.new_workspace(B, H, L, w.dk, w.dv, backward=True, device=dev)
+
+    def call(i, ev=None):
+        mode = i % 4
+        if ev:
+            ev[0].record(stream)
+        dig.dig_gla_fwd(q, k, v, z, w.inv_tau, o, w.grid_h, w.grid_w, mode, ws_f, r=r, y=y, stream=stream)
+        if ev:
+            ev[1].record(stream)
+        dig.dig_gla_bwd_saved(q, k, v, z, w.inv_tau, dO, dq, dk_, dv_, dla, w.grid_h, w.grid_w, mode, ws_f, ws_b,
+                              stream=stream)
+        if ev:
+            ev[2].record(stream)
+
+    for i in range(warmup):
+        flush.fill_(float(i))
+        call(i)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(iters)]
+    for i in range(iters):
+        flush.fill_(float(i))
+        call(i, evs[i])
+    torch.cuda.synchronize()
+    for ws in (ws_f, ws_b):
+        st = dig.dig_read_status(ws)
+        if st != dig.DIG_OK:
+            raise RuntimeError("device status on %s: %s" % (w.name, dig.lib.dig_status_string(st).decode()))
+    t_f = float(np.mean([e[0].elapsed_time(e[1]) for e in evs])) * 1e-3
+    t_b = float(np.mean([e[1].elapsed_time(e[2]) for e in evs])) * 1e-3
+    return t_f, t_b
+
+
+def per_config_record(index, t_f, t_b, world, hbm, tflops):
+    """tokens/s of fwd+bwd and the fraction of roofline of each, with the metric's bytes."""
+    w = inputs.WORKLOADS[index]
+    fb, bb = metric_bytes(w)
+    epi = 2 * w.B * w.L * w.H * w.dv * 2 if w.epilogue else 0  # r in, y out (o is counted above)
+    roof_f = (fb + epi) / (hbm * 1e9)
+    roof_b = bb / (hbm * 1e9)
+    return {"workload": "%s: B=%d, %dx%d grid (L=%d), H=%d, d_k=%d, d_v=%d, bf16%s"
+                        % (w.name, w.B, w.grid_h, w.grid_w, w.L, w.H, w.dk, w.dv,
+                           ", fwd with Swish*RMSNorm epilogue" if w.epilogue else ""),
+            "seq_len": w.L, "tokens_per_s": w.B * w.L * world / (t_f + t_b),
+            "fwd_us": t_f * 1e6, "bwd_us": t_b * 1e6,
+            "fwd_bytes": fb + epi, "bwd_bytes": bb,
+            "fwd_frac": roof_f / t_f, "bwd_frac": roof_b / t_b,
+            "roofline_tokens_per_s": w.B * w.L * world / (roof_f + roof_b),
+            "frac": (roof_f + roof_b) / (t_f + t_b), "bound": "hbm", "peak_gbs": hbm}
+
+
+def run_guarded(fn, world, device):
+    """Runs fn() on every rank; returns (result, None) when it succeeded on all ranks and
+    ({}, message) otherwise, with every rank taking the same branch (one all-reduce of an
+    error flag) so that the collectives that follow stay paired.  A CUDA error leaves the
+    context unusable, so it is raised instead of being reported."""
+    result, err = {}, None
+    try:
+        result = fn()
+    except Exception as e:  # noqa: BLE001
+        torch.cuda.synchronize()  # raises if the error was a device fault
+        err = "%s: %s" % (type(e).__name__, str(e).splitlines()[0] if str(e) else "")
+    if world > 1:
+        flag = torch.tensor([1.0 if err else 0.0], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(flag, op=torch.distributed.ReduceOp.MAX)
+        if flag.item() and err is None:
+            err = "failed on another rank"
+    return (result, None) if err is None else ({}, err)
+
+
 def run_ours(args, rank, world, local_rank):
     from gated_linear_attention_fwd_b200 import dig
     dev = torch.device("cuda", local_rank)
@@ -384,12 +483,23 @@ def run_ours(args, rank, world, local_rank):
     # projection and its backward): each timed alone with CUDA events, L2 flushed
     # before every call, on the bench's workload
     # (an error there is reported in the line instead of costing the step's numbers)
-    try:
-        aux_t = time_next_ops(dig, w, dev, stream, o, r, dO, xc, wc, dla, flush, args.warmup, max(args.steps, 10))
-        aux_t = {op: max_over_ranks(tv, world, dev) for op, tv in aux_t.items()}
-        aux_err = None
-    except Exception as e:  # noqa: BLE001
-        aux_t, aux_err = {}, "%s: %s" % (type(e).__name__, str(e).splitlines()[0] if str(e) else "")
+    aux_t, aux_err = run_guarded(lambda: time_next_ops(dig, w, dev, stream, o, r, dO, xc, wc, dla, flush,
+                                                       args.warmup, max(args.steps, 10)), world, dev)
+    aux_t = {op: max_over_ranks(tv, world, dev) for op, tv in aux_t.items()} if aux_err is None else {}
+
+    # the metric's three shapes, each timed the same way (fwd + bwd from the forward's records)
+    cfg_t, cfg_err = {}, None
+    if not args.no_per_config:
+        def _cfgs():
+            out = {}
+            for idx in PER_CONFIG:
+                if idx == WORKLOAD_INDEX:
+                    continue
+                out[idx] = time_gla_config(dig, idx, dev, stream, flush, args.warmup, max(args.steps, 10), rank)
+            return out
+        cfg_t, cfg_err = run_guarded(_cfgs, world, dev)
+        if cfg_err is None:
+            cfg_t = {i: (max_over_ranks(a, world, dev), max_over_ranks(b, world, dev)) for i, (a, b) in cfg_t.items()}
 
     if rank != 0:
         return None
@@ -429,12 +539,34 @@ def run_ours(args, rank, world, local_rank):
                                         "kernels": OP_KERNELS[op]}
                          for op, t in aux_t.items()} if aux_err is None else {"error": aux_err},
     }
+    if not args.no_per_config:
+        t_step_fb = (t_f, t_b)
+        recs = {}
+        for idx in PER_CONFIG:
+            tf_, tb_ = t_step_fb if idx == WORKLOAD_INDEX else cfg_t.get(idx, (None, None))
+            if tf_ is not None:
+                recs[inputs.WORKLOADS[idx].name] = per_config_record(idx, tf_, tb_, world, hbm, tflops)
+        line["per_config"] = recs if cfg_err is None else dict(recs, error=cfg_err)
+        line["per_config_note"] = ("fwd+bwd (dig_gla_fwd + dig_gla_bwd_saved, bf16 outputs) per metric shape; "
+                                   "bytes count d log(alpha) once per head; fractions of the measured HBM copy "
+                                   "bandwidth")
     if world == 1 and not args.no_cpu_baseline:
         tps, dt, cores, n = cpu_sample(w, x, steps=1, min_seconds=10.0)
+        import oracle
+        nthreads = oracle.num_threads()
+        oracle.set_num_threads(1)
+        try:
+            tps1, dt1, _, n1 = cpu_sample(w, x, steps=1, min_seconds=5.0)
+        finally:
+            oracle.set_num_threads(nthreads)
         line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "nproc": os.cpu_count(),
                                 "sample": "oracle (fp64 C, OpenMP over heads) on batch element 0 of %s, all heads: "
                                           "%d steps (fwd+epilogue+bwd+conv, %d tokens each, scan modes cycling), "
-                                          "%.1f s" % (w.name, n, w.L, dt)}
+                                          "%.1f s" % (w.name, n, w.L, dt),
+                                "single_thread": {"value": tps1, "unit": "tokens/s", "cores": 1,
+                                                  "sample": "the same steps on one thread: %d steps, %.1f s"
+                                                            % (n1, dt1)}}
     return line
 
 
@@ -445,6 +577,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true", help="skip the L=4096 and L=16384 shapes")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -1,6 +1,8 @@
 // dig_api.cu -- the C ABI of libdig.so (include/dig.h): argument validation,
-// work decomposition, workspace layout, launches.  No allocation, no
-// synchronisation (except dig_read_status), no device state kept.
+// work decomposition, workspace layout, launches.  No allocation and no
+// synchronisation (except dig_read_status).  The library keeps no device state
+// of its own, with one exception: the 16 MiB scratch array of
+// dig_gla_fwd_noalloc (dig_noalloc.cu), held per device until the process exits.
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -95,24 +97,49 @@ size_t dig_gla_workspace_bytes(int B, int H, int gate_heads, int L, int d_k, int
   return ws_layout(B > 0 ? B : 1, H, gate_heads, L, nchunks, d_k, d_v, pass == 1).total;
 }
 
-dig_status dig_gla_fwd(const void* q, const void* k, const void* v, const float* z, int gate_heads, float inv_tau,
-                       void* o, const void* r, const float* gamma, float eps, void* y, int B, int H, int L, int d_k,
-                       int d_v, int grid_h, int grid_w, int scan_mode, int dtype, int out_dtype, void* workspace,
-                       size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace dig {
+// Every synchronous check of dig_gla_fwd (also run by dig_gla_fwd_noalloc before
+// it enqueues anything).  DIG_OK with *nothing_to_do set means an empty problem.
+dig_status gla_fwd_check(const void* q, const void* k, const void* v, const float* z, int gate_heads, void* o,
+                         const void* r, const float* gamma, void* y, int B, int H, int L, int d_k, int d_v,
+                         int grid_h, int grid_w, int scan_mode, int dtype, int out_dtype, const void* workspace,
+                         size_t workspace_bytes, bool* nothing_to_do) {
+  *nothing_to_do = false;
   dig_status st = check_common(B, H, L, d_k, d_v, grid_h, grid_w, scan_mode, dtype, out_dtype, gate_heads);
   if (st != DIG_OK) return st;
   if (!workspace) return fail(DIG_ERR_INVALID_ARGUMENT, "workspace is NULL");
   if (!aligned16(workspace)) return fail(DIG_ERR_MISALIGNED, "workspace not 16-byte aligned");
-  if (B == 0 || L == 0) return DIG_OK;
+  if (B == 0 || L == 0) {
+    *nothing_to_do = true;
+    return DIG_OK;
+  }
   if (!q || !k || !v || !z || !o) return fail(DIG_ERR_INVALID_ARGUMENT, "q, k, v, z and o must be non-NULL");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(z) || !aligned16(o) || !aligned16(r) ||
       !aligned16(gamma) || !aligned16(y))
     return fail(DIG_ERR_MISALIGNED, "a tensor pointer is not 16-byte aligned");
   const int C = chunk_len(dtype, false, d_k, d_v);
-  const int nchunks = (L + C - 1) / C;
-  const WsLayout lay = ws_layout(B, H, gate_heads, L, nchunks, d_k, d_v, false);
+  const WsLayout lay = ws_layout(B, H, gate_heads, L, (L + C - 1) / C, d_k, d_v, false);
   if (workspace_bytes < lay.total)
     return fail(DIG_ERR_WORKSPACE_TOO_SMALL, "workspace has %zu bytes, needs %zu", workspace_bytes, lay.total);
+  return DIG_OK;
+}
+}  // namespace dig
+
+extern "C" {
+
+dig_status dig_gla_fwd(const void* q, const void* k, const void* v, const float* z, int gate_heads, float inv_tau,
+                       void* o, const void* r, const float* gamma, float eps, void* y, int B, int H, int L, int d_k,
+                       int d_v, int grid_h, int grid_w, int scan_mode, int dtype, int out_dtype, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  bool empty = false;
+  const dig_status st = gla_fwd_check(q, k, v, z, gate_heads, o, r, gamma, y, B, H, L, d_k, d_v, grid_h, grid_w,
+                                      scan_mode, dtype, out_dtype, workspace, workspace_bytes, &empty);
+  if (st != DIG_OK || empty) return st;
+  const int C = chunk_len(dtype, false, d_k, d_v);
+  const int nchunks = (L + C - 1) / C;
+  const WsLayout lay = ws_layout(B, H, gate_heads, L, nchunks, d_k, d_v, false);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   GlaArgs a{};
   a.q = q; a.k = k; a.v = v; a.z = z; a.r = r; a.gamma = gamma; a.o = o; a.y = y;

@@ -27,7 +27,20 @@ void* g_scratch_ptr[kMaxDevices];  // device address of g_scratch, per device
 
 namespace dig {
 void set_last_error(const char* msg);  // dig_api.cu
+dig_status gla_fwd_check(const void* q, const void* k, const void* v, const float* z, int gate_heads, void* o,
+                         const void* r, const float* gamma, void* y, int B, int H, int L, int d_k, int d_v,
+                         int grid_h, int grid_w, int scan_mode, int dtype, int out_dtype, const void* workspace,
+                         size_t workspace_bytes, bool* nothing_to_do);  // dig_api.cu
 }
+
+namespace {
+dig_status cuda_fail(const char* step, cudaError_t e) {
+  char msg[256];
+  snprintf(msg, sizeof(msg), "dig_gla_fwd_noalloc: %s: %s", step, cudaGetErrorString(e));
+  dig::set_last_error(msg);
+  return DIG_ERR_CUDA;
+}
+}  // namespace
 
 extern "C" dig_status dig_gla_fwd_noalloc(const void* q, const void* k, const void* v, const float* z, int gate_heads,
                                           float inv_tau, void* o, const void* r, const float* gamma, float eps, void* y,
@@ -35,7 +48,15 @@ extern "C" dig_status dig_gla_fwd_noalloc(const void* q, const void* k, const vo
                                           int scan_mode, int dtype, int out_dtype, unsigned int* device_status,
                                           void* stream) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DIG_ERR_CUDA;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+  if (dev < 0 || dev >= kMaxDevices) {
+    char msg[160];
+    snprintf(msg, sizeof(msg), "dig_gla_fwd_noalloc: device %d is beyond the %d devices it keeps a scratch address for",
+             dev, kMaxDevices);
+    dig::set_last_error(msg);
+    return DIG_ERR_UNSUPPORTED;
+  }
   void* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_mu);
@@ -43,12 +64,18 @@ extern "C" dig_status dig_gla_fwd_noalloc(const void* q, const void* k, const vo
       // In host code g_scratch names a host-side stand-in; the kernel needs the
       // device address, resolved once per device with that device current.
       void* p = nullptr;
-      const cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
-      if (e != cudaSuccess || p == nullptr) return DIG_ERR_CUDA;
+      e = cudaGetSymbolAddress(&p, g_scratch);
+      if (e != cudaSuccess) return cuda_fail("cudaGetSymbolAddress of the scratch array", e);
+      if (p == nullptr) return cuda_fail("cudaGetSymbolAddress of the scratch array", cudaErrorInvalidSymbol);
       g_scratch_ptr[dev] = p;
     }
     scratch = g_scratch_ptr[dev];
   }
+  // Every argument check of dig_gla_fwd runs before anything is enqueued.
+  bool empty = false;
+  dig_status st = dig::gla_fwd_check(q, k, v, z, gate_heads, o, r, gamma, y, B, H, L, d_k, d_v, grid_h, grid_w,
+                                     scan_mode, dtype, out_dtype, scratch, ~size_t(0), &empty);
+  if (st != DIG_OK) return st;
   const size_t need = dig_gla_workspace_bytes(B, H, gate_heads, L, d_k, d_v, 0);
   if (need > kScratchBytes) {
     char msg[200];
@@ -61,12 +88,14 @@ extern "C" dig_status dig_gla_fwd_noalloc(const void* q, const void* k, const vo
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the status word must start at zero on every call
-  if (cudaMemsetAsync(scratch, 0, kClearBytes, s) != cudaSuccess) return DIG_ERR_CUDA;
-  const dig_status st = dig_gla_fwd(q, k, v, z, gate_heads, inv_tau, o, r, gamma, eps, y, B, H, L, d_k, d_v, grid_h,
-                                    grid_w, scan_mode, dtype, out_dtype, scratch, kScratchBytes, stream);
-  if (st != DIG_OK) return st;
+  if ((e = cudaMemsetAsync(scratch, 0, kClearBytes, s)) != cudaSuccess) return cuda_fail("status clear", e);
+  if (!empty) {
+    st = dig_gla_fwd(q, k, v, z, gate_heads, inv_tau, o, r, gamma, eps, y, B, H, L, d_k, d_v, grid_h, grid_w,
+                     scan_mode, dtype, out_dtype, scratch, kScratchBytes, stream);
+    if (st != DIG_OK) return st;
+  }
   if (device_status != nullptr &&
-      cudaMemcpyAsync(device_status, scratch, sizeof(unsigned int), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
-    return DIG_ERR_CUDA;
+      (e = cudaMemcpyAsync(device_status, scratch, sizeof(unsigned int), cudaMemcpyDeviceToDevice, s)) != cudaSuccess)
+    return cuda_fail("status copy", e);
   return DIG_OK;
 }

@@ -122,6 +122,10 @@ dig_status dig_gla_fwd(const void *q, const void *k, const void *v, const float 
  *     are rejected with DIG_ERR_WORKSPACE_TOO_SMALL (see dig_last_error).
  *   - The first call on a device looks up the scratch array's device address
  *     (with that device current); make that first call before any stream capture.
+ *     The address is kept for the life of the process: after a cudaDeviceReset
+ *     in the host process it is stale, so do not use this entry point after one.
+ *   - Every argument check of dig_gla_fwd runs first; an invalid call returns
+ *     before anything is enqueued on `stream`.
  *   - Every call clears the scratch's status word (a small memset on `stream`)
  *     and shares the one array: calls that overlap on the GPU (other
  *     streams, other threads) race on it and must not be issued.
