@@ -5,6 +5,7 @@
 // dig_gla_fwd_noalloc (dig_noalloc.cu), held per device until the process exits.
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 
 #include "../../include/dig.h"
@@ -44,6 +45,7 @@ WsLayout ws_layout(int B, int H, int gate_heads, int L, int nchunks, int dk, int
   w.gCH = take(nbz * (size_t)nchunks * 4 * dk * 4);
   w.dsn = take(nseq * (size_t)nchunks * dk * dv * 4);
   w.dhn = take(backward ? nseq * (size_t)nchunks * dk * dv * 4 : 0);
+  w.flist = take(backward ? (1 + nseq * (size_t)nchunks) * 4 : 0);
   w.total = off;
   return w;
 }
@@ -57,6 +59,15 @@ int chunk_len(int dtype, bool backward, int dk, int dv) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Bound of the kernels' device waits: DIG_DEVICE_WAIT_LIMIT_NS in the environment
+// (a test hook that makes a wait run out on purpose), else the two-second default.
+unsigned long long spin_limit_ns() {
+  const char* e = getenv("DIG_DEVICE_WAIT_LIMIT_NS");
+  if (!e || !*e) return 0;
+  const unsigned long long v = strtoull(e, nullptr, 10);
+  return v;
+}
 
 dig_status check_common(int B, int H, int L, int d_k, int d_v, int grid_h, int grid_w, int scan_mode, int dtype,
                         int out_dtype, int gate_heads) {
@@ -150,6 +161,7 @@ dig_status dig_gla_fwd(const void* q, const void* k, const void* v, const float*
   a.gEQ = reinterpret_cast<float*>(ws + lay.gEQ);
   a.gCH = reinterpret_cast<float*>(ws + lay.gCH);
   a.dsn = reinterpret_cast<float*>(ws + lay.dsn);
+  a.spin_ns = spin_limit_ns();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   GlaVariant var{C, dtype == DIG_BF16 ? 2 : 3, d_k, d_v, dtype, out_dtype};
   const cudaError_t e = launch_gla_fwd(var, a, s);
@@ -201,6 +213,8 @@ static dig_status gla_bwd_impl(const void* q, const void* k, const void* v, cons
   a.gCH = reinterpret_cast<float*>((saved ? fws + flay.gCH : ws + lay.gCH));
   a.dsn = reinterpret_cast<float*>((saved ? fws + flay.dsn : ws + lay.dsn));
   a.dhn = reinterpret_cast<float*>(ws + lay.dhn);
+  a.flist = reinterpret_cast<uint32_t*>(ws + lay.flist);
+  a.spin_ns = spin_limit_ns();
   GlaVariant var{C, dtype == DIG_BF16 ? 2 : 3, d_k, d_v, dtype, out_dtype};
   const cudaError_t e = launch_gla_bwd(var, a, saved, s);
   if (e != cudaSuccess) return fail(DIG_ERR_CUDA, "gla_bwd launch: %s", cudaGetErrorString(e));

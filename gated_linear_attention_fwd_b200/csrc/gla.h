@@ -35,6 +35,9 @@ struct GlaArgs {
   float* dsn;        // [nseq][nchunks][DV][DK]  chunk state contribution, then the state entering the chunk
   float* dhn;        // backward: [nseq][nchunks][DV][DK] chunk state-gradient contribution, then the
                      // gradient of the state leaving the chunk
+  uint32_t* flist;   // backward: [0] count, [1..] units the fp16 gradient kernel left to the exact one
+                     // (the exact kernel then processes only those; NULL: every unit)
+  unsigned long long spin_ns;  // bound of a device wait in ns (0: the default of two seconds)
 };
 
 // Kernel-variant selection: chunk length, split count, head dims, types.
@@ -49,7 +52,7 @@ struct GlaVariant {
 // the status word, the gate factors, the per-chunk states and, for the
 // backward, the per-chunk state gradients.
 struct WsLayout {
-  size_t gEQ, gCH, dsn, dhn, total;
+  size_t gEQ, gCH, dsn, dhn, flist, total;
 };
 WsLayout ws_layout(int B, int H, int gate_heads, int L, int nchunks, int dk, int dv, bool backward);
 

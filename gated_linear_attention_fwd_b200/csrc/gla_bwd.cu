@@ -262,7 +262,10 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
     fence_mbar_init();
   }
   if (tid < 128) sh.bnd[tid >> 6][tid & 63] = 0.f;
-  if ((int)blockIdx.x < nunits) fill_rows(a, blockIdx.x, C, sh.rows[0]);
+  // With a unit list (the units the fp16 gradient kernel left), only those units
+  // are processed; the list is written by that kernel, so it is read after the wait.
+  const bool listed = a.flist != nullptr;
+  if (!listed && (int)blockIdx.x < nunits) fill_rows(a, blockIdx.x, C, sh.rows[0]);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -331,21 +334,30 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
   // The kernel before this one is the state scan, which writes only the chunk
   // states and state gradients; everything older has completed.  So the first
   // unit's other rows are requested before the wait for that scan.
-  if ((int)blockIdx.x < nunits) {
-    const int h0 = Unit(a, blockIdx.x).h;
-    if constexpr (PRE) issue_qk(blockIdx.x, sh.rows[0]);
+  auto first_rows = [&](int u0) {
+    const int h0 = Unit(a, u0).h;
+    if constexpr (PRE) issue_qk(u0, sh.rows[0]);
     load_v_rows_t<C, DK, DV, TIN>(a, h0, sh.rows[0], a.v, sbase + BC::OFF_V);
     load_v_rows_t<C, DK, DV, TIN>(a, h0, sh.rows[0], a.dO, sbase + BC::OFF_DO);
-  }
+  };
+  if (!listed && (int)blockIdx.x < nunits) first_rows(blockIdx.x);
   griddep_wait();  // the kernels before this one have completed
   griddep_launch_dependents();
-  if (tid == 0 && (int)blockIdx.x < nunits) issue_states(blockIdx.x);
+  const int count = listed ? (int)__ldcg(a.flist) : nunits;
+  auto unit_at = [&](int kx) { return listed ? (int)__ldcg(a.flist + 1 + kx) : kx; };
+  if (listed && (int)blockIdx.x < count) {
+    fill_rows(a, unit_at(blockIdx.x), C, sh.rows[0]);
+    __syncthreads();
+    first_rows(unit_at(blockIdx.x));
+  }
+  if (tid == 0 && (int)blockIdx.x < count) issue_states(unit_at(blockIdx.x));
 
-  for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
+  for (int kx = blockIdx.x; kx < count; kx += gridDim.x, ++it) {
+    const int u = unit_at(kx);
     const Unit U(a, u);
     const int hz = U.bz - U.b * a.gate_heads;
-    const int un = u + gridDim.x;
-    const bool has_next = un < nunits;
+    const bool has_next = kx + (int)gridDim.x < count;
+    const int un = has_next ? unit_at(kx + gridDim.x) : 0;
     float* bnd = sh.bnd[it & 1];
     const long long* rows = sh.rows[it & 1];  // this unit's grid tokens
     long long* rows_next = sh.rows[(it + 1) & 1];
@@ -729,6 +741,9 @@ __global__ void __launch_bounds__(256, 3) gla_chunk_dh_kernel(const GlaArgs a) {
 }
 
 // ------------------------------------------------------------------ launch
+bool gla_grad_tma_eligible(const GlaArgs& a, int dk, int dv, int tin, int chunk);  // gla_bwd_tma.cu
+cudaError_t launch_grad_tma(const GlaArgs& a, int tout, cudaStream_t s, bool* launched);
+
 namespace {
 
 template <int DK, int DV, typename TIN, typename TOUT>
@@ -738,20 +753,33 @@ cudaError_t launch_typed(const GlaArgs& a, bool saved, cudaStream_t s) {
   const long long units = (long long)a.B * a.H * a.nchunks;
   if (units <= 0) return cudaSuccess;
   cudaError_t e;
+  // bf16 inputs of the shapes the fp16 / TMA gradient kernel covers go through it;
+  // the scan just before it clears the list of units it hands back.
+  const bool tma = std::is_same<TIN, __nv_bfloat16>::value && a.flist != nullptr &&
+                   gla_grad_tma_eligible(a, DK, DV, DIG_BF16, C);
+  uint32_t* zero_word = tma ? a.flist : nullptr;
   if (saved) {  // gate factors and entry states come from the forward: only dH and its reverse scan
     using DC = DhCfg<C, DK, DV, TIN>;
     auto kd = gla_chunk_dh_kernel<C, DK, DV, TIN>;
     if ((e = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, DC::SMEM)) != cudaSuccess)
       return e;
     if ((e = launch_pdl(kd, persistent_grid(DC::PER_SM, units), 256, DC::SMEM, s, a)) != cudaSuccess) return e;
-    if ((e = launch_state_scan(a, a.dhn, true, nullptr, false, DK, DV, s)) != cudaSuccess) return e;
+    if ((e = launch_state_scan(a, a.dhn, true, nullptr, false, DK, DV, s, zero_word)) != cudaSuccess) return e;
   } else {
     if ((e = launch_chunk_state<C, DK, DV, TIN, true>(a, s)) != cudaSuccess) return e;
-    if ((e = launch_state_scan(a, a.dsn, false, a.dhn, true, DK, DV, s)) != cudaSuccess) return e;
+    if ((e = launch_state_scan(a, a.dsn, false, a.dhn, true, DK, DV, s, zero_word)) != cudaSuccess) return e;
+  }
+  GlaArgs b = a;
+  b.flist = nullptr;
+  if (tma) {
+    bool launched = false;
+    if ((e = launch_grad_tma(a, std::is_same<TOUT, float>::value ? DIG_F32 : DIG_BF16, s, &launched)) != cudaSuccess)
+      return e;
+    if (launched) b.flist = a.flist;  // the exact kernel takes only the units handed back
   }
   auto k = gla_chunk_grad_kernel<C, DK, DV, TIN, TOUT>;
   if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, BC::SMEM)) != cudaSuccess) return e;
-  return launch_pdl(k, persistent_grid(BC::PER_SM, units), 256, BC::SMEM, s, a);
+  return launch_pdl(k, persistent_grid(BC::PER_SM, units), 256, BC::SMEM, s, b);
 }
 
 template <int DK, int DV>

@@ -505,6 +505,6 @@ cudaError_t launch_chunk_state(const GlaArgs& a, cudaStream_t s) {
 // (reverse: the same recurrence from the last chunk down, giving the gradient
 // leaving every chunk).  In place in buf0 and, when not null, buf1 (one launch).
 cudaError_t launch_state_scan(const GlaArgs& a, float* buf0, bool rev0, float* buf1, bool rev1, int dk, int dv,
-                              cudaStream_t s);
+                              cudaStream_t s, uint32_t* zero_word = nullptr);
 
 }  // namespace dig

@@ -100,12 +100,14 @@ constexpr int kScanRanges = 16, kScanQuads = 16, kScanWindow = 8;
 struct ScanJob {
   float* buf[2];
   int reverse[2];
+  uint32_t* zero_word;  // set to 0 by the scan (the count of the backward's unit list), or NULL
 };
 __global__ void __launch_bounds__(kScanRanges * kScanQuads, 2) gla_state_scan_kernel(const GlaArgs a, ScanJob job,
                                                                                      int dk, int dv) {
   __shared__ float4 sA[kScanRanges][kScanQuads], sS[kScanRanges][kScanQuads];
   griddep_wait();  // the kernels before this one have completed
   griddep_launch_dependents();
+  if (job.zero_word != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *job.zero_word = 0u;
   float* buf = blockIdx.y ? job.buf[1] : job.buf[0];
   const int reverse = blockIdx.y ? job.reverse[1] : job.reverse[0];
   const int nq = dv * dk / 4;
@@ -503,12 +505,12 @@ int num_sms() {
 }
 
 cudaError_t launch_state_scan(const GlaArgs& a, float* buf0, bool rev0, float* buf1, bool rev1, int dk, int dv,
-                              cudaStream_t s) {
+                              cudaStream_t s, uint32_t* zero_word) {
   const int nq = dv * dk / 4;
   const long long blocks = (long long)a.B * a.H * ((nq + kScanQuads - 1) / kScanQuads);
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 2147483647LL) return cudaErrorInvalidValue;
-  ScanJob job{{buf0, buf1}, {rev0 ? 1 : 0, rev1 ? 1 : 0}};
+  ScanJob job{{buf0, buf1}, {rev0 ? 1 : 0, rev1 ? 1 : 0}, zero_word};
   return launch_pdl(gla_state_scan_kernel, dim3((unsigned)blocks, buf1 ? 2u : 1u), kScanRanges * kScanQuads, 0, s, a,
                     job, dk, dv);
 }
