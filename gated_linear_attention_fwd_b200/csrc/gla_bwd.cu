@@ -252,6 +252,10 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
   __shared__ GradSmem sh;
   const int tid = threadIdx.x, warp = tid >> 5;
   const int nunits = a.B * a.H * a.nchunks;
+  if (a.flist != nullptr) {  // unit-list mode: CTAs beyond the list end before taking any resource
+    griddep_wait();
+    if ((int)blockIdx.x >= (int)__ldcg(a.flist)) return;
+  }
   if (warp == 0) {
     tmem_alloc(&sh.tmem, BC::TM_COLS);
     tmem_relinquish();

@@ -48,7 +48,17 @@ struct TmaGradCfg {
   static constexpr int OFF_SP = 49152, OFF_GT = 53248;  // fp16 [DV][DK], 64-byte swizzle
   static constexpr int OFF_EQ = 57344;                  // fp32 [C][DK], 128-byte swizzle
   static constexpr int OFF_ST = 73728;                  // raw fp32 S_n [DV][DK], then G_n
-  static constexpr int OFF_DLA = 90112;                 // raw S_{n+1} at the unit's start, then d log alpha rows
+  static constexpr int OFF_DLA = 90112;                 // raw S_{n+1} [DV][DK]
+  // bf16 outputs ("decoupled"): once the key gradients are formed, the d log alpha
+  // rows go over the raw states, dq and dk over the gate factors and dv over
+  // S_{n+1}, so the operand tiles are free at once and the next unit's q, k, v,
+  // dO are requested then; the small loads (gate factors, states) follow the
+  // stores.  fp32 outputs (twice the staging) stage over the operand tiles and
+  // request the next unit after the stores have been read.
+  static constexpr bool DEC = !std::is_same<TOUT, float>::value;
+  static constexpr int OFF_X = DEC ? OFF_ST : OFF_DLA;   // d log alpha rows, fp32 [C][DK], 128-byte swizzle
+  static constexpr int OFF_SDQ = DEC ? OFF_EQ : 0, OFF_SDK = DEC ? OFF_EQ + 8192 : 16384;
+  static constexpr int OFF_SDV = DEC ? OFF_DLA : 32768;
   static constexpr int END = 106496;
   static constexpr int SMEM = END + 1024;               // the base is aligned up to 1024 bytes
   static constexpr int TM_R = 0, TM_DQ = 128, TM_DK = 160, TM_DV = 192, TM_COLS = 256;
@@ -120,36 +130,36 @@ __device__ __forceinline__ float h_lo(uint32_t w) { return __half2float(__ushort
 __device__ __forceinline__ float h_hi(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w >> 16))); }
 
 // Masks one C x C product in TMEM (lane = row r; keep column c >= r when
-// `upper`, else c <= r) and rewrites it in place as fp16 pairs: the 16-column
-// block s0 = 64 half + 16 kk becomes the 8 columns at 64 half + 8 kk, the
-// A-operand layout of a K-step of 16 (see acol).  Tracks |value| in `amax`.
+// `upper`, else c <= r) and rewrites it in place as fp16 pairs: the 32-column
+// block s0 = 64 half + 32 kk becomes the 16 columns at 64 half + 16 kk, i.e.
+// K-step j (16 columns) ends up at acol(j), the A-operand layout.  Tracks
+// |value| in `amax`.
 __device__ __forceinline__ void mask_to_f16(uint32_t tmem, uint32_t region, bool upper, uint32_t& amax) {
   const int tid = threadIdx.x, t = tid & 127, wq = t >> 5, half = tid >> 7;
   const uint32_t lane_base = static_cast<uint32_t>(32 * wq) << 16;
 #pragma unroll
-  for (int kk = 0; kk < 4; ++kk) {
-    const int s0 = half * 64 + 16 * kk;
-    const bool zero_block = upper ? (s0 + 15 < 32 * wq) : (s0 > 32 * wq + 31);  // warp-uniform
-    float pv[16];
+  for (int kk = 0; kk < 2; ++kk) {
+    const int s0 = half * 64 + 32 * kk;  // 32-aligned: the block is this warp's diagonal block or off it
+    const bool zero_block = upper ? (s0 < 32 * wq) : (s0 > 32 * wq);  // warp-uniform
+    float pv[32];
     if (!zero_block) {
-      tmem_ld16(tmem + lane_base + region + s0, pv);
+      tmem_ld32(tmem + lane_base + region + s0, pv);
       tmem_ld_wait();
-      const bool full = upper ? (s0 >= 32 * wq + 31) : (s0 + 15 <= 32 * wq);
-      if (!full) {
+      if (s0 == 32 * wq) {  // the diagonal block
 #pragma unroll
-        for (int e = 0; e < 16; ++e) pv[e] = (upper ? (s0 + e >= t) : (s0 + e <= t)) ? pv[e] : 0.f;
+        for (int e = 0; e < 32; ++e) pv[e] = (upper ? (s0 + e >= t) : (s0 + e <= t)) ? pv[e] : 0.f;
       }
     } else {
 #pragma unroll
-      for (int e = 0; e < 16; ++e) pv[e] = 0.f;
+      for (int e = 0; e < 32; ++e) pv[e] = 0.f;
     }
-    uint32_t pk[8];
+    uint32_t pk[16];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
+    for (int e = 0; e < 16; ++e) {
       pk[e] = pack_f16x2(pv[2 * e], pv[2 * e + 1]);
       amax = absmax_f16x2(amax, pk[e]);
     }
-    tmem_st8(tmem + lane_base + region + half * 64 + 8 * kk, pk);
+    tmem_st16(tmem + lane_base + region + half * 64 + 16 * kk, pk);
   }
 }
 // TMEM column of K-step j (16 tokens) of a converted C x C product.
@@ -200,10 +210,16 @@ __global__ void __launch_bounds__(256, 2) gla_grad_tma_kernel(const __grid_const
   bool last_done = true;
 
   // ---- thread 0: TMA issue
-  auto issue_inputs = [&](const TileUnit& T, bool with_eq, uint32_t phase) {  // q, k, v, dO (and the gate factors)
-    ld_state = 2;
+  // The last request of a barrier phase arrives on it (the phase completes once
+  // that arrival and all requested bytes are in); earlier ones only add bytes.
+  auto expect = [&](uint64_t* bar, uint32_t bytes, bool arrive) {
+    if (arrive) mbar_arrive_expect_tx(bar, bytes);
+    else mbar_expect_tx(bar, bytes);
+  };
+  auto issue_tiles = [&](const TileUnit& T, uint32_t phase, bool arrive) {  // q, k, v, dO
+    ld_state = arrive ? 2 : 1;
     ld_ph = phase;
-    mbar_arrive_expect_tx(&sh.bar_ld, TC::IN_BYTES + (with_eq ? TC::EQ_BYTES : 0u));
+    expect(&sh.bar_ld, TC::IN_BYTES, arrive);
     if (!T.col) {
       tma_load_2d(sb + TC::OFF_Q, mp.q, T.h * DK, T.y, &sh.bar_ld);
       tma_load_2d(sb + TC::OFF_K, mp.k, T.h * DK, T.y, &sh.bar_ld);
@@ -219,25 +235,25 @@ __global__ void __launch_bounds__(256, 2) gla_grad_tma_kernel(const __grid_const
         tma_load_4d(sb + TC::OFF_DO + j * 16 * TC::RBV, mp.dO, T.h * DV, row, cl, T.b, &sh.bar_ld);
       }
     }
-    if (with_eq) tma_load_2d(sb + TC::OFF_EQ, mp.eq, 0, T.bz * a.L + T.n * C, &sh.bar_ld);
   };
-  auto issue_eq_early = [&](const TileUnit& T, uint32_t phase) {  // gate factors ahead of the rest (no arrive)
-    ld_state = 1;
+  auto issue_eq = [&](const TileUnit& T, uint32_t phase, bool arrive) {  // gate factors (scan order)
+    ld_state = arrive ? 2 : 1;
     ld_ph = phase;
-    mbar_expect_tx(&sh.bar_ld, TC::EQ_BYTES);
+    expect(&sh.bar_ld, TC::EQ_BYTES, arrive);
     tma_load_2d(sb + TC::OFF_EQ, mp.eq, 0, T.bz * a.L + T.n * C, &sh.bar_ld);
   };
-  auto issue_states = [&](int u, const TileUnit& T, uint32_t phase) {  // S_n, G_n, chunk constants (no arrive)
-    st_state = 1;
+  auto issue_states = [&](int u, const TileUnit& T, uint32_t phase, bool arrive) {  // S_n, G_n, chunk constants
+    st_state = arrive ? 2 : 1;
     st_ph = phase;
-    mbar_expect_tx(&sh.bar_st, 2 * TC::SB + TC::GCH_BYTES);
+    expect(&sh.bar_st, 2 * TC::SB + TC::GCH_BYTES, arrive);
     bulk_copy_g2s(sb + TC::OFF_ST, a.dsn + (size_t)u * DV * DK, TC::SB, &sh.bar_st);
     bulk_copy_g2s(sb + TC::OFF_ST + TC::SB, a.dhn + (size_t)u * DV * DK, TC::SB, &sh.bar_st);
     bulk_copy_g2s(smem_u32(sh.gch), a.gCH + ((size_t)T.bz * a.nchunks + T.n) * 4 * DK, TC::GCH_BYTES, &sh.bar_st);
   };
-  auto issue_next_state = [&](int u, const TileUnit& T) {  // S_{n+1} (completes the phase)
+  auto issue_next_state = [&](int u, const TileUnit& T, uint32_t phase) {  // S_{n+1}; completes the phase
     const bool has_next_chunk = T.n + 1 < a.nchunks;  // G of the last chunk is zero: no boundary term
     st_state = 2;
+    st_ph = phase;
     mbar_arrive_expect_tx(&sh.bar_st, has_next_chunk ? TC::SB : 0u);
     if (has_next_chunk) bulk_copy_g2s(sb + TC::OFF_DLA, a.dsn + (size_t)(u + 1) * DV * DK, TC::SB, &sh.bar_st);
   };
@@ -246,9 +262,10 @@ __global__ void __launch_bounds__(256, 2) gla_grad_tma_kernel(const __grid_const
   griddep_launch_dependents();
   if (tid == 0 && (int)blockIdx.x < nunits) {
     const TileUnit T0(a, blockIdx.x, C);
-    issue_inputs(T0, true, 0);
-    issue_states(blockIdx.x, T0, 0);
-    issue_next_state(blockIdx.x, T0);
+    issue_tiles(T0, 0, false);
+    issue_eq(T0, 0, true);
+    issue_states(blockIdx.x, T0, 0, false);
+    issue_next_state(blockIdx.x, T0, 0);
   }
 
   int it = 0;
@@ -305,7 +322,9 @@ __global__ void __launch_bounds__(256, 2) gla_grad_tma_kernel(const __grid_const
       for (int g = 0; g < 8; ++g) s += sh.red[g][tid];
       sh.bnd[tid] = s;
     }
-    if (tid == 0 && has_next && !timed_out && !sh.abort) issue_states(un, TileUnit(a, un, C), ph ^ 1u);
+    if constexpr (!TC::DEC) {  // the raw-state slot is free: the next unit's S_n, G_n
+      if (tid == 0 && has_next && !timed_out && !sh.abort) issue_states(un, TileUnit(a, un, C), ph ^ 1u, false);
+    }
 
     // ---- 2. inputs, converted in place to fp16 operands: qbar = q EQ, kbar = k / EQ, v, dO
     wait_bar(&sh.bar_ld, ph);
@@ -439,7 +458,7 @@ __global__ void __launch_bounds__(256, 2) gla_grad_tma_kernel(const __grid_const
     wait_group(5);
 
     // ---- 4. key gradients of this thread's token (TMEM lane t) and channel half; d log alpha terms
-    float dq[16], dk[16];
+    float dq[16], dk[16], x[16];
     {
       const int ti = T.rev ? C - 1 - t : t;
       float dqb[16], dkb[16];
@@ -447,47 +466,43 @@ __global__ void __launch_bounds__(256, 2) gla_grad_tma_kernel(const __grid_const
       tmem_ld8(tmem + lane_base + TC::TM_DQ + 16 * half + 8, dqb + 8);
       tmem_ld8(tmem + lane_base + TC::TM_DK + 16 * half, dkb);
       tmem_ld8(tmem + lane_base + TC::TM_DK + 16 * half + 8, dkb + 8);
-      tmem_ld_wait();
-      float e[16], qb[16], kb[16];
+      float4 ef[4];
+      uint4 qv[2], kv[2];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const float4 f = lds128f(sb + TC::OFF_EQ + swz_off<128>(ti, 4 * half + m));
-        e[4 * m] = f.x;
-        e[4 * m + 1] = f.y;
-        e[4 * m + 2] = f.z;
-        e[4 * m + 3] = f.w;
-      }
+      for (int m = 0; m < 4; ++m) ef[m] = lds128f(sb + TC::OFF_EQ + swz_off<128>(ti, 4 * half + m));
 #pragma unroll
       for (int m = 0; m < 2; ++m) {
-        const uint4 qv = lds128(sQ + swz_off<64>(t, 2 * half + m)), kv = lds128(sK + swz_off<64>(t, 2 * half + m));
-        const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w}, kw[4] = {kv.x, kv.y, kv.z, kv.w};
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          qb[8 * m + 2 * w] = h_lo(qw[w]);
-          qb[8 * m + 2 * w + 1] = h_hi(qw[w]);
-          kb[8 * m + 2 * w] = h_lo(kw[w]);
-          kb[8 * m + 2 * w + 1] = h_hi(kw[w]);
-        }
+        qv[m] = lds128(sQ + swz_off<64>(t, 2 * half + m));
+        kv[m] = lds128(sK + swz_off<64>(t, 2 * half + m));
       }
-      float x[16];
+      tmem_ld_wait();
+      const float e[16] = {ef[0].x, ef[0].y, ef[0].z, ef[0].w, ef[1].x, ef[1].y, ef[1].z, ef[1].w,
+                           ef[2].x, ef[2].y, ef[2].z, ef[2].w, ef[3].x, ef[3].y, ef[3].z, ef[3].w};
+      const uint32_t qw[8] = {qv[0].x, qv[0].y, qv[0].z, qv[0].w, qv[1].x, qv[1].y, qv[1].z, qv[1].w};
+      const uint32_t kw[8] = {kv[0].x, kv[0].y, kv[0].z, kv[0].w, kv[1].x, kv[1].y, kv[1].z, kv[1].w};
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
+      for (int w = 0; w < 8; ++w) {
+        const float qa = h_lo(qw[w]), qb2 = h_hi(qw[w]), ka = h_lo(kw[w]), kb2 = h_hi(kw[w]);
+        const int c = 2 * w;
         dq[c] = dqb[c] * e[c];
+        dq[c + 1] = dqb[c + 1] * e[c + 1];
         dk[c] = dkb[c] * __frcp_rn(e[c]);
-        x[c] = qb[c] * dqb[c] - kb[c] * dkb[c];
+        dk[c + 1] = dkb[c + 1] * __frcp_rn(e[c + 1]);
+        x[c] = qa * dqb[c] - ka * dkb[c];
+        x[c + 1] = qb2 * dqb[c + 1] - kb2 * dkb[c + 1];
       }
-#pragma unroll
-      for (int m = 0; m < 4; ++m)
-        sts128(sb + TC::OFF_DLA + swz_off<128>(t, 4 * half + m),
-               make_uint4(__float_as_uint(x[4 * m]), __float_as_uint(x[4 * m + 1]), __float_as_uint(x[4 * m + 2]),
-                          __float_as_uint(x[4 * m + 3])));
     }
-    fence_async_smem();  // the gate-factor reads precede the next unit's copy into the same slot
+    fence_async_smem();  // the gate-factor and operand reads precede the copies into those slots
     tc_fence_before();
     __syncthreads();  // qbar, kbar and gate factors read; every product complete
-    if constexpr (!TC::F32OUT) {
-      if (tid == 0 && has_next && !timed_out && !sh.abort) issue_eq_early(TileUnit(a, un, C), ph ^ 1u);
+    if constexpr (TC::DEC) {  // the operand tiles are free: the next unit's q, k, v, dO
+      if (tid == 0 && has_next && !timed_out && !sh.abort) issue_tiles(TileUnit(a, un, C), ph ^ 1u, false);
     }
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+      sts128(sb + TC::OFF_X + swz_off<128>(t, 4 * half + m),
+             make_uint4(__float_as_uint(x[4 * m]), __float_as_uint(x[4 * m + 1]), __float_as_uint(x[4 * m + 2]),
+                        __float_as_uint(x[4 * m + 3])));
 
     // ---- 5. outputs to staging over the operand tiles (swizzled like the store boxes)
     {
@@ -498,16 +513,16 @@ __global__ void __launch_bounds__(256, 2) gla_grad_tma_kernel(const __grid_const
       if constexpr (!TC::F32OUT) {
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
-          sts128(sQ + swz_off<64>(t, 2 * half + m),
+          sts128(sb + TC::OFF_SDQ + swz_off<64>(t, 2 * half + m),
                  make_uint4(pack_bf16x2(dq[8 * m], dq[8 * m + 1]), pack_bf16x2(dq[8 * m + 2], dq[8 * m + 3]),
                             pack_bf16x2(dq[8 * m + 4], dq[8 * m + 5]), pack_bf16x2(dq[8 * m + 6], dq[8 * m + 7])));
-          sts128(sK + swz_off<64>(t, 2 * half + m),
+          sts128(sb + TC::OFF_SDK + swz_off<64>(t, 2 * half + m),
                  make_uint4(pack_bf16x2(dk[8 * m], dk[8 * m + 1]), pack_bf16x2(dk[8 * m + 2], dk[8 * m + 3]),
                             pack_bf16x2(dk[8 * m + 4], dk[8 * m + 5]), pack_bf16x2(dk[8 * m + 6], dk[8 * m + 7])));
         }
 #pragma unroll
         for (int m = 0; m < 4; ++m)
-          sts128(sV + swz_off<128>(t, 4 * half + m),
+          sts128(sb + TC::OFF_SDV + swz_off<128>(t, 4 * half + m),
                  make_uint4(pack_bf16x2(dv[8 * m], dv[8 * m + 1]), pack_bf16x2(dv[8 * m + 2], dv[8 * m + 3]),
                             pack_bf16x2(dv[8 * m + 4], dv[8 * m + 5]), pack_bf16x2(dv[8 * m + 6], dv[8 * m + 7])));
       } else {
@@ -532,31 +547,32 @@ __global__ void __launch_bounds__(256, 2) gla_grad_tma_kernel(const __grid_const
 
     // ---- 6. d log alpha: cumsum over the chunk in scan order (tile order reversed when `rev`)
     {
-      const int c = tid & 31, sg = tid >> 5;
-      const uint32_t cbase = sb + TC::OFF_DLA + (uint32_t)(c & 3) * 4u;
-      float acc = 0.f;
-#pragma unroll 4
-      for (int e = 0; e < 16; ++e) {
-        const int i = T.rev ? 16 * sg + e : 16 * sg + 15 - e;
-        const uint32_t ad = cbase + swz_off<128>(i, c >> 2);
-        float xv;
-        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(xv) : "r"(ad));
-        acc += xv;
-        asm volatile("st.shared.f32 [%0], %1;" ::"r"(ad), "f"(acc) : "memory");
+      const int c = tid & 31, sg = tid >> 5;  // channel, 16-row segment
+      const uint32_t cbase = sb + TC::OFF_X + (uint32_t)(c & 3) * 4u;
+      float xv[16];
+      __syncthreads();  // every x row written
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(xv[e]) : "r"(cbase + swz_off<128>(16 * sg + e, c >> 2)));
+      // scan order runs down the rows (suffix sums) or, reversed, up them (prefix sums)
+      if (T.rev) {
+#pragma unroll
+        for (int e = 1; e < 16; ++e) xv[e] += xv[e - 1];
+        sh.segtot[sg][c] = xv[15];
+      } else {
+#pragma unroll
+        for (int e = 14; e >= 0; --e) xv[e] += xv[e + 1];
+        sh.segtot[sg][c] = xv[0];
       }
-      sh.segtot[sg][c] = acc;
       __syncthreads();
       float post = sh.bnd[c];
 #pragma unroll
       for (int s2 = 0; s2 < 8; ++s2)
         if (T.rev ? s2 < sg : s2 > sg) post += sh.segtot[s2][c];
-#pragma unroll 4
-      for (int e = 0; e < 16; ++e) {
-        const uint32_t ad = cbase + swz_off<128>(16 * sg + e, c >> 2);
-        float xv;
-        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(xv) : "r"(ad));
-        asm volatile("st.shared.f32 [%0], %1;" ::"r"(ad), "f"(xv + post) : "memory");
-      }
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        asm volatile("st.shared.f32 [%0], %1;" ::"r"(cbase + swz_off<128>(16 * sg + e, c >> 2)), "f"(xv[e] + post)
+                     : "memory");
     }
     fence_async_smem();  // staging writes precede the TMA stores that read them
     const int bad = __syncthreads_or(out_of_range || f16x2_too_large(amax));
@@ -569,42 +585,48 @@ __global__ void __launch_bounds__(256, 2) gla_grad_tma_kernel(const __grid_const
       } else if (!sh.abort) {
         if (!T.col) {
           if constexpr (!TC::F32OUT) {
-            tma_store_2d(mp.dq, T.h * DK, T.y, sQ);
-            tma_store_2d(mp.dk, T.h * DK, T.y, sK);
-            tma_store_2d(mp.dv, T.h * DV, T.y, sV);
+            tma_store_2d(mp.dq, T.h * DK, T.y, sb + TC::OFF_SDQ);
+            tma_store_2d(mp.dk, T.h * DK, T.y, sb + TC::OFF_SDK);
+            tma_store_2d(mp.dv, T.h * DV, T.y, sb + TC::OFF_SDV);
           } else {
             tma_store_2d(mp.dq, T.h * DK, T.y, sb);
             tma_store_2d(mp.dk, T.h * DK, T.y, sb + 16384u);
             tma_store_2d(mp.dv, T.h * DV, T.y, sb + 32768u);
             tma_store_2d(mp.dv, T.h * DV + 32, T.y, sb + TC::OFF_EQ);
           }
-          if (a.gate_heads == 1) tma_reduce_add_2d(mp.dla, T.hz * DK, T.y, sb + TC::OFF_DLA);
-          else tma_store_2d(mp.dla, T.hz * DK, T.y, sb + TC::OFF_DLA);
+          if (a.gate_heads == 1) tma_reduce_add_2d(mp.dla, T.hz * DK, T.y, sb + TC::OFF_X);
+          else tma_store_2d(mp.dla, T.hz * DK, T.y, sb + TC::OFF_X);
         } else {
           for (int j = 0; j < C / 16; ++j) {
             int row, cl;
             T.seg(a, j, row, cl);
             if constexpr (!TC::F32OUT) {
-              tma_store_4d(mp.dq, T.h * DK, row, cl, T.b, sQ + j * 16 * TC::RBK);
-              tma_store_4d(mp.dk, T.h * DK, row, cl, T.b, sK + j * 16 * TC::RBK);
-              tma_store_4d(mp.dv, T.h * DV, row, cl, T.b, sV + j * 16 * TC::RBV);
+              tma_store_4d(mp.dq, T.h * DK, row, cl, T.b, sb + TC::OFF_SDQ + j * 16 * TC::RBK);
+              tma_store_4d(mp.dk, T.h * DK, row, cl, T.b, sb + TC::OFF_SDK + j * 16 * TC::RBK);
+              tma_store_4d(mp.dv, T.h * DV, row, cl, T.b, sb + TC::OFF_SDV + j * 16 * TC::RBV);
             } else {
               tma_store_4d(mp.dq, T.h * DK, row, cl, T.b, sb + j * 2048);
               tma_store_4d(mp.dk, T.h * DK, row, cl, T.b, sb + 16384u + j * 2048);
               tma_store_4d(mp.dv, T.h * DV, row, cl, T.b, sb + 32768u + j * 2048);
               tma_store_4d(mp.dv, T.h * DV + 32, row, cl, T.b, sb + TC::OFF_EQ + j * 2048);
             }
-            if (a.gate_heads == 1) tma_reduce_add_4d(mp.dla, T.hz * DK, row, cl, T.b, sb + TC::OFF_DLA + j * 2048);
-            else tma_store_4d(mp.dla, T.hz * DK, row, cl, T.b, sb + TC::OFF_DLA + j * 2048);
+            if (a.gate_heads == 1) tma_reduce_add_4d(mp.dla, T.hz * DK, row, cl, T.b, sb + TC::OFF_X + j * 2048);
+            else tma_store_4d(mp.dla, T.hz * DK, row, cl, T.b, sb + TC::OFF_X + j * 2048);
           }
         }
         bulk_commit();
       }
       if (has_next && !timed_out && !sh.abort) {
-        bulk_wait_read_all();  // the staging (operand tiles, d log alpha rows) has been read
+        bulk_wait_read_all();  // the staging has been read
         const TileUnit Tn(a, un, C);
-        issue_inputs(Tn, TC::F32OUT, ph ^ 1u);
-        issue_next_state(un, Tn);
+        if constexpr (TC::DEC) {  // the q, k, v, dO tiles are already on their way
+          issue_eq(Tn, ph ^ 1u, true);
+          issue_states(un, Tn, ph ^ 1u, false);
+        } else {
+          issue_tiles(Tn, ph ^ 1u, false);
+          issue_eq(Tn, ph ^ 1u, true);
+        }
+        issue_next_state(un, Tn, ph ^ 1u);
       }
     }
     if (sh.abort) break;  // uniform: read after the barrier above
