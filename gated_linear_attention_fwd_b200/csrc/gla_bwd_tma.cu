@@ -29,6 +29,7 @@
 // take this kernel; everything else runs the exact kernel directly.
 #include "gla_chunk.cuh"
 #include "tma.cuh"
+#include "tma_tiles.cuh"
 #include "tmap.h"
 
 namespace dig {
@@ -80,54 +81,6 @@ struct TmaGradSmem {
   uint32_t tmem;
   int abort;                  // a wait gave up: stop after this unit
 };
-
-// Tile placement of a unit: the chunk's C tokens as a box of consecutive grid
-// tokens (row orders) or as C / 16 column segments (column orders).  `rev`: the
-// tile's rows run against the scan order (tile row i is scan position C-1-i).
-struct TileUnit {
-  int b, h, n, bz, hz;
-  bool rev, col;
-  int y;   // row orders: first grid token of the box, as a row of the [B * L] view
-  int q0;  // column orders: first column-order position of the tile
-  __device__ TileUnit(const GlaArgs& a, int u, int C) {
-    const int bh = u / a.nchunks;
-    n = u - bh * a.nchunks;
-    b = bh / a.H;
-    h = bh - b * a.H;
-    bz = b * a.gate_heads + (a.gate_heads == 1 ? 0 : h);
-    hz = a.gate_heads == 1 ? 0 : h;
-    rev = (a.mode & 1) != 0;
-    col = (a.mode & 2) != 0;
-    const int first = rev ? a.L - (n + 1) * C : n * C;
-    y = b * a.L + first;
-    q0 = first;
-  }
-  // column segment j: grid row and column of its first token
-  __device__ void seg(const GlaArgs& a, int j, int& row, int& cl) const {
-    const int p = q0 + 16 * j;
-    cl = p / a.Hg;
-    row = p - cl * a.Hg;
-  }
-};
-
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ float4 lds128f(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-               : "memory");
-}
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-__device__ __forceinline__ float h_lo(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w & 0xFFFFu))); }
-__device__ __forceinline__ float h_hi(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w >> 16))); }
 
 // Masks one C x C product in TMEM (lane = row r; keep column c >= r when
 // `upper`, else c <= r) and rewrites it in place as fp16 pairs: the 32-column

@@ -515,6 +515,9 @@ cudaError_t launch_state_scan(const GlaArgs& a, float* buf0, bool rev0, float* b
                     job, dk, dv);
 }
 
+bool gla_out_tma_eligible(const GlaArgs& a, int dk, int dv, int tin, int chunk);  // gla_fwd_tma.cu
+cudaError_t launch_out_tma(const GlaArgs& a, int tout, cudaStream_t s, bool* launched);
+
 namespace {
 
 template <int C, int DK, int DV, typename TIN, typename TOUT>
@@ -525,6 +528,12 @@ cudaError_t launch_typed(const GlaArgs& a, cudaStream_t s) {
   cudaError_t e = launch_chunk_state<C, DK, DV, TIN, false>(a, s);
   if (e != cudaSuccess) return e;
   if ((e = launch_state_scan(a, a.dsn, false, nullptr, false, DK, DV, s)) != cudaSuccess) return e;
+  if (std::is_same<TIN, __nv_bfloat16>::value && gla_out_tma_eligible(a, DK, DV, DIG_BF16, C)) {
+    bool launched = false;
+    if ((e = launch_out_tma(a, std::is_same<TOUT, float>::value ? DIG_F32 : DIG_BF16, s, &launched)) != cudaSuccess)
+      return e;
+    if (launched) return cudaGetLastError();
+  }
   auto k3 = gla_chunk_out_kernel<C, DK, DV, TIN, TOUT>;
   if ((e = cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, OC::SMEM)) != cudaSuccess) return e;
   if ((e = launch_pdl(k3, persistent_grid(2, units), 256, OC::SMEM, s, a)) != cudaSuccess) return e;
