@@ -763,11 +763,16 @@ cudaError_t launch_typed(const GlaArgs& a, bool saved, cudaStream_t s) {
                    gla_grad_tma_eligible(a, DK, DV, DIG_BF16, C);
   uint32_t* zero_word = tma ? a.flist : nullptr;
   if (saved) {  // gate factors and entry states come from the forward: only dH and its reverse scan
-    using DC = DhCfg<C, DK, DV, TIN>;
-    auto kd = gla_chunk_dh_kernel<C, DK, DV, TIN>;
-    if ((e = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, DC::SMEM)) != cudaSuccess)
-      return e;
-    if ((e = launch_pdl(kd, persistent_grid(DC::PER_SM, units), 256, DC::SMEM, s, a)) != cudaSuccess) return e;
+    bool reduced = false;
+    if (std::is_same<TIN, __nv_bfloat16>::value && gla_reduce_tma_eligible(a, DK, DV, DIG_BF16, C))
+      if ((e = launch_reduce_tma(a, true, s, &reduced)) != cudaSuccess) return e;
+    if (!reduced) {
+      using DC = DhCfg<C, DK, DV, TIN>;
+      auto kd = gla_chunk_dh_kernel<C, DK, DV, TIN>;
+      if ((e = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize, DC::SMEM)) != cudaSuccess)
+        return e;
+      if ((e = launch_pdl(kd, persistent_grid(DC::PER_SM, units), 256, DC::SMEM, s, a)) != cudaSuccess) return e;
+    }
     if ((e = launch_state_scan(a, a.dhn, true, nullptr, false, DK, DV, s, zero_word)) != cudaSuccess) return e;
   } else {
     if ((e = launch_chunk_state<C, DK, DV, TIN, true>(a, s)) != cudaSuccess) return e;

@@ -486,6 +486,13 @@ inline int persistent_grid(int per_sm, long long units) {
   return (int)(units < slots ? units : slots);
 }
 
+// Per-chunk dS (bwd = false, from k and v into `dsn`) or dH (bwd = true, from q
+// and dO into `dhn`) by the tile-copy kernel (gla_state_tma.cu), for bf16 inputs
+// with d_k = 32, d_v = 64 and 128-token chunks that tile the sequence.
+// `launched` stays false when the tensor maps cannot be encoded.
+bool gla_reduce_tma_eligible(const GlaArgs& a, int dk, int dv, int tin, int chunk);
+cudaError_t launch_reduce_tma(const GlaArgs& a, bool bwd, cudaStream_t s, bool* launched);
+
 // Gate kernel, then chunk-state kernel (which reads the gate factors).
 template <int C, int DK, int DV, typename TIN, bool BWD>
 cudaError_t launch_chunk_state(const GlaArgs& a, cudaStream_t s) {
@@ -495,6 +502,12 @@ cudaError_t launch_chunk_state(const GlaArgs& a, cudaStream_t s) {
   const long long gunits = (long long)a.B * a.gate_heads * a.nchunks;
   cudaError_t e = launch_pdl(gla_gate_kernel<C, DK>, dim3(persistent_grid(4, gunits)), dim3(256), 0, s, a);
   if (e != cudaSuccess) return e;
+  if (std::is_same<TIN, __nv_bfloat16>::value && gla_reduce_tma_eligible(a, DK, DV, DIG_BF16, C)) {
+    bool launched = false;
+    if ((e = launch_reduce_tma(a, false, s, &launched)) != cudaSuccess) return e;
+    if (launched && BWD && (e = launch_reduce_tma(a, true, s, &launched)) != cudaSuccess) return e;
+    if (launched) return cudaSuccess;
+  }
   auto k1 = gla_chunk_state_kernel<C, DK, DV, TIN, BWD>;
   if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, SC::SMEM)) != cudaSuccess) return e;
   return launch_pdl(k1, persistent_grid(SC::PER_SM, units), 256, SC::SMEM, s, a);
