@@ -92,6 +92,11 @@ struct GradSmem {
   uint64_t bar[6];      // completion of the six product groups of a unit
   uint64_t sbar;        // completion of the unit's bulk copies (states and chunk constants)
   uint32_t tmem;
+  // thread 0's record of asynchronous work not yet seen complete, drained before exit
+  int mma_pend;         // the product group whose commit is outstanding (-1: none)
+  uint32_t mma_ph;
+  int st_pend;          // state copies requested and not yet seen landed
+  uint32_t st_ph;
 };
 
 // Masks one C x C product in TMEM (lane = row r; keep column c >= r when
@@ -263,6 +268,8 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
   if (tid == 0) {
     for (int i = 0; i < 6; ++i) mbar_init(&sh.bar[i], 1);
     mbar_init(&sh.sbar, 1);
+    sh.mma_pend = -1;
+    sh.st_pend = 0;
     fence_mbar_init();
   }
   if (tid < 128) sh.bnd[tid >> 6][tid & 63] = 0.f;
@@ -284,15 +291,25 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
   float* EQ = reinterpret_cast<float*>(smem + BC::OFF_EQ);  // EQ rows, then the d log alpha terms
   uint32_t ph = 0;
   int it = 0;
-  bool timed_out = false;
+  bool timed_out = false;  // a wait of this thread gave up: nothing further is issued
+  bool stop = false;       // some wait of the CTA gave up (uniform, from the last barrier)
+  auto commit = [&](int i) {
+    mma_commit(&sh.bar[i]);
+    sh.mma_pend = i;
+    sh.mma_ph = ph;
+  };
+  auto wait_group = [&](int i) {  // one thread: product group i of this unit is complete
+    if (!mbar_wait(&sh.bar[i], ph, spin_limit(a))) timed_out = true;
+    else if (tid == 0 && sh.mma_pend == i) sh.mma_pend = -1;
+  };
   auto wait_all = [&](int i) {  // every thread: product group i of this unit is complete
-    if (!mbar_wait(&sh.bar[i], ph, kSpinLimitNs)) timed_out = true;
+    if (!stop) wait_group(i);
     tc_fence_after();
   };
   auto publish = [&]() {  // this thread's TMEM / shared writes, then a CTA barrier
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();
+    stop = __syncthreads_or(timed_out);
     tc_fence_after();
   };
 
@@ -329,6 +346,8 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
   auto issue_states = [&](int u) {
     const Unit U(a, u);
     const bool has_next_chunk = U.n + 1 < a.nchunks;  // G of the last chunk is zero
+    sh.st_pend = 1;
+    sh.st_ph = ph;
     mbar_arrive_expect_tx(&sh.sbar, 2 * SB + (has_next_chunk ? SB : 0u) + 2 * DK * 4);
     bulk_copy_g2s(sbase + BC::OFF_SP, a.dsn + (size_t)u * DV * DK, SB, &sh.sbar);
     bulk_copy_g2s(sbase + BC::OFF_GT, a.dhn + (size_t)u * DV * DK, SB, &sh.sbar);
@@ -368,7 +387,8 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
     if (has_next) fill_rows(a, un, C, rows_next);  // read after the operand barrier
     // ---- the state blocks, read in place: S' and Gt rows (to registers) and the boundary term
     const bool has_next_chunk = U.n + 1 < a.nchunks;
-    if (!mbar_wait(&sh.sbar, ph, kSpinLimitNs)) timed_out = true;
+    if (!mbar_wait(&sh.sbar, ph, spin_limit(a))) timed_out = true;
+    else if (tid == 0) sh.st_pend = 0;
     float spv[K::NPS][4], gtv[K::NPS][4];
 #pragma unroll
     for (int j = 0; j < K::NPS; ++j) {
@@ -467,7 +487,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
     cp_async_wait_all();
     publish();
     // ---- P^T and the three inter-chunk terms
-    if (tid == 0) {
+    if (tid == 0 && !stop) {
       mma_issue<NTG, NTG, DKP / 16>(tmem + BC::TM_R, dKk, K::AQ_SZ, 256, dQk, K::AQ_SZ, 256, idesc_bf16(128, C),
                                     false);  // P^T[s][t]
       mma_issue<NTV, NTG, DVP / 16>(tmem + BC::TM_DQ, dDOk, K::VR_SZ, 256, dSPm, K::SPT_SZ, 2 * K::SBO_K,
@@ -476,41 +496,45 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
                                     idesc_bf16(128, DKP, false, true), false);  // V Gt^T
       mma_issue<NTG, NTG, DKP / 16>(tmem + BC::TM_DV, dKk, K::AQ_SZ, 256, dGTk, K::SPT_SZ, 256, idesc_bf16(128, DVP),
                                     false);  // kbar Gt
-      mma_commit(&sh.bar[0]);
+      commit(0);
     }
     wait_all(0);
     mask_to_terms<C, BC::PT_STRIDE>(tmem, BC::TM_R, true);
     tmem_st_wait();
     publish();
     // ---- dv += P^T dO; then dP^T into the region once that product has read it
-    if (tid == 0) {
+    if (tid == 0 && !stop) {
       mma_issue_ts<NTP, NTV, C / 16>(tmem + BC::TM_DV, tmem + BC::TM_R, BC::PT_STRIDE, dDOm, K::VR_SZ, 2 * K::SBO_V,
                                      idesc_bf16(128, DVP, false, true), true);
-      mma_commit(&sh.bar[1]);
-      if (!mbar_wait(&sh.bar[1], ph, kSpinLimitNs)) timed_out = true;
+      commit(1);
+      wait_group(1);
       tc_fence_after();
-      mma_issue<NTV, NTV, DVP / 16>(tmem + BC::TM_R, dVk, K::VR_SZ, 256, dDOk, K::VR_SZ, 256, idesc_bf16(128, C),
-                                    false);  // dP^T[s][t]
-      mma_commit(&sh.bar[2]);
+      if (!timed_out) {
+        mma_issue<NTV, NTV, DVP / 16>(tmem + BC::TM_R, dVk, K::VR_SZ, 256, dDOk, K::VR_SZ, 256, idesc_bf16(128, C),
+                                      false);  // dP^T[s][t]
+        commit(2);
+      }
     }
     wait_all(2);
     mask_to_terms<C, BC::PT_STRIDE>(tmem, BC::TM_R, true);
     tmem_st_wait();
     publish();
     // ---- dkbar += dP^T qbar; then dP
-    if (tid == 0) {
+    if (tid == 0 && !stop) {
       mma_issue_ts<NTP, NTG, C / 16>(tmem + BC::TM_DK, tmem + BC::TM_R, BC::PT_STRIDE, dQm, K::AQ_SZ, 2 * K::SBO_K,
                                      idesc_bf16(128, DKP, false, true), true);
-      mma_commit(&sh.bar[3]);
-      if (!mbar_wait(&sh.bar[3], ph, kSpinLimitNs)) timed_out = true;
+      commit(3);
+      wait_group(3);
       tc_fence_after();
-      mma_issue<NTV, NTV, DVP / 16>(tmem + BC::TM_R, dDOk, K::VR_SZ, 256, dVk, K::VR_SZ, 256, idesc_bf16(128, C),
-                                    false);  // dP[t][s]
-      mma_commit(&sh.bar[4]);
+      if (!timed_out) {
+        mma_issue<NTV, NTV, DVP / 16>(tmem + BC::TM_R, dDOk, K::VR_SZ, 256, dVk, K::VR_SZ, 256, idesc_bf16(128, C),
+                                      false);  // dP[t][s]
+        commit(4);
+      }
     }
     wait_all(4);
     // v and dO are no longer read: the next unit's rows start to arrive now
-    if (has_next) {
+    if (has_next && !timed_out && !stop) {
       const int hn = Unit(a, un).h;
       load_v_rows_t<C, DK, DV, TIN>(a, hn, rows_next, a.v, sbase + BC::OFF_V);
       load_v_rows_t<C, DK, DV, TIN>(a, hn, rows_next, a.dO, sbase + BC::OFF_DO);
@@ -519,10 +543,10 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
     tmem_st_wait();
     publish();
     // ---- dqbar += dP kbar
-    if (tid == 0) {
+    if (tid == 0 && !stop) {
       mma_issue_ts<NTP, NTG, C / 16>(tmem + BC::TM_DQ, tmem + BC::TM_R, BC::PT_STRIDE, dKm, K::AQ_SZ, 2 * K::SBO_K,
                                      idesc_bf16(128, DKP, false, true), true);
-      mma_commit(&sh.bar[5]);
+      commit(5);
     }
     wait_all(5);
     ph ^= 1u;
@@ -589,8 +613,8 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
     }
     if (tid < 64) sh.bnd[(it + 1) & 1][tid] = 0.f;  // the next unit's accumulator
     fence_async_smem();  // the staging reads precede the next unit's bulk copies into the same slots
-    __syncthreads();
-    if (tid == 0 && has_next) issue_states(un);  // they land while d log alpha is finished
+    stop = __syncthreads_or(timed_out);
+    if (tid == 0 && has_next && !stop) issue_states(un);  // they land while d log alpha is finished
     if (sg < BC::NSG) {
       float post = bnd[sc];
       for (int s2 = sg + 1; s2 < BC::NSG; ++s2) post += sh.segtot[s2][sc];
@@ -604,9 +628,18 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
         }
       }
     }
-    __syncthreads();  // staging, EQ rows and segment totals are reused by the next unit
+    // staging, EQ rows and segment totals are reused by the next unit; after a
+    // wait gave up anywhere in the CTA, no further unit starts
+    if (__syncthreads_or(timed_out)) break;
   }
+  // ---- drain: this thread's row copies, the state copies and the last products
+  // complete before TMEM is released and the CTA exits
   if (timed_out) set_status(a.status, DIG_ERR_DEVICE_TIMEOUT);
+  cp_async_wait_all();
+  if (tid == 0) {
+    if (sh.st_pend) mbar_wait(&sh.sbar, sh.st_ph, kSpinLimitNs);
+    if (sh.mma_pend >= 0) mbar_wait(&sh.bar[sh.mma_pend], sh.mma_ph, kSpinLimitNs);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -659,7 +692,8 @@ __global__ void __launch_bounds__(256, 3) gla_chunk_dh_kernel(const GlaArgs a) {
   const uint64_t dDOm = sdesc(sbase + DC::OFF_DO, K::SBO_V, 128);
   const uint64_t dQBm = sdesc(sbase + DC::OFF_QB, K::SBO_K, 128);
   uint32_t ph = 0;
-  bool timed_out = false;
+  bool timed_out = false;  // a wait of this thread gave up: the CTA stops after this unit
+  if (tid == 0) sh.mma_pend = 0;
   Piece<TIN, PSK> pq[K::NPK];
   Piece<float, PSK> pe[K::NPK];
   Piece<float, 4> pc[K::NPK * PSK / 4];  // 2^r of the piece's channels
@@ -721,11 +755,15 @@ __global__ void __launch_bounds__(256, 3) gla_chunk_dh_kernel(const GlaArgs a) {
       mma_issue<NTV, NTG, C / 16>(tmem, dDOm, K::VR_SZ, 2 * K::SBO_V, dQBm, K::AQ_SZ, 2 * K::SBO_K,
                                   idesc_bf16(128, DKP, true, true), false);
       mma_commit(&sh.bar);
+      sh.mma_pend = 1;
+      sh.mma_ph = ph;
     }
-    if (!mbar_wait(&sh.bar, ph, kSpinLimitNs)) timed_out = true;
+    if (!mbar_wait(&sh.bar, ph, spin_limit(a))) timed_out = true;
+    else if (tid == 0) sh.mma_pend = 0;
     ph ^= 1u;
     tc_fence_after();
-    if (has_next) load_v_rows_t<C, DK, DV, TIN>(a, Unit(a, un).h, rows_next, a.dO, sbase + DC::OFF_DO);
+    if (has_next && !timed_out)
+      load_v_rows_t<C, DK, DV, TIN>(a, Unit(a, un).h, rows_next, a.dO, sbase + DC::OFF_DO);
     if (tid < 128) stage_rows_dk<C, DK, DV, TIN, 0>(tmem, 0, SD, DC::SDP);
     else stage_rows_dk<C, DK, DV, TIN, 1>(tmem, 0, SD, DC::SDP);
     tc_fence_before();
@@ -735,9 +773,14 @@ __global__ void __launch_bounds__(256, 3) gla_chunk_dh_kernel(const GlaArgs a) {
       const int row = i / (DK / 4), c4 = i - row * (DK / 4);
       __stcg(dst + i, *reinterpret_cast<const float4*>(SD + row * DC::SDP + 4 * c4));
     }
-    __syncthreads();  // staging and operands are reused by the next unit
+    // staging and operands are reused by the next unit; after a wait gave up
+    // anywhere in the CTA, no further unit starts
+    if (__syncthreads_or(timed_out)) break;
   }
+  // ---- drain: this thread's row copies, and the last products, complete before exit
   if (timed_out) set_status(a.status, DIG_ERR_DEVICE_TIMEOUT);
+  cp_async_wait_all();
+  if (tid == 0 && sh.mma_pend) mbar_wait(&sh.bar, sh.mma_ph, kSpinLimitNs);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

@@ -15,6 +15,9 @@
 
 namespace dig {
 
+// Bound of the kernels' waits: the call's test bound when one was set, else the default.
+__device__ __forceinline__ uint64_t spin_limit(const GlaArgs& a) { return a.spin_ns ? a.spin_ns : kSpinLimitNs; }
+
 template <int C_, int DK_, int DV_, typename TIN>
 struct ChunkCfg {
   static constexpr int C = C_, DK = DK_, DV = DV_;
@@ -81,6 +84,8 @@ struct StateSmem {
   long long rows[2][128];  // grid tokens of the units whose loads are in flight (by unit parity)
   uint64_t bar;
   uint32_t tmem;
+  int mma_pend;            // thread 0: products committed and not yet seen complete (drained before exit)
+  uint32_t mma_ph;
 };
 
 // Unit u -> (sequence bh, chunk n); units of one sequence are consecutive.
@@ -320,7 +325,8 @@ __global__ void __launch_bounds__(256, StateCfg<C, DK, DV, TIN, BWD>::MINB) gla_
   const uint64_t dQBm = sdesc(sbase + SC::OFF_QB, Cfg::SBO_K, 128);
   const int nunits = a.B * a.H * a.nchunks;
   uint32_t ph = 0;
-  bool timed_out = false;
+  bool timed_out = false;   // a wait of this thread gave up: the CTA stops after this unit
+  if (tid == 0) sh.mma_pend = 0;
 
   // Row pieces of a unit, loaded one unit ahead: gate factors EQ = 2^(b - r),
   // the chunk constants and k (and q) are issued once the current unit's
@@ -416,11 +422,14 @@ __global__ void __launch_bounds__(256, StateCfg<C, DK, DV, TIN, BWD>::MINB) gla_
         mma_issue<NTV, NTG, C / 16>(tmem + SC::TM_DH, dDOm, Cfg::VR_SZ, 2 * Cfg::SBO_V, dQBm, Cfg::AQ_SZ,
                                     2 * Cfg::SBO_K, idesc_bf16(128, DKP, true, true), false);
       mma_commit(&sh.bar);
+      sh.mma_pend = 1;
+      sh.mma_ph = ph;
     }
-    if (!mbar_wait(&sh.bar, ph, kSpinLimitNs)) timed_out = true;
+    if (!mbar_wait(&sh.bar, ph, spin_limit(a))) timed_out = true;
+    else if (tid == 0) sh.mma_pend = 0;
     ph ^= 1u;
     tc_fence_after();
-    if (has_next) issue_vd(un, rows_next);  // v (and dO) of this unit are consumed
+    if (has_next && !timed_out) issue_vd(un, rows_next);  // v (and dO) of this unit are consumed
     if (tid < 128) stage_rows_dk<C, DK, DV, TIN, 0>(tmem, 0, SD, SC::SDP);
     else stage_rows_dk<C, DK, DV, TIN, 1>(tmem, 0, SD, SC::SDP);
     if constexpr (BWD) {
@@ -444,9 +453,14 @@ __global__ void __launch_bounds__(256, StateCfg<C, DK, DV, TIN, BWD>::MINB) gla_
         }
       }
     }
-    __syncthreads();  // operands, staging and the cumsum buffer are reused by the next unit
+    // operands, staging and the cumsum buffer are reused by the next unit; after a
+    // wait gave up anywhere in the CTA, no further unit starts
+    if (__syncthreads_or(timed_out)) break;
   }
+  // ---- drain: this thread's row copies, and the last products, complete before exit
   if (timed_out) set_status(a.status, DIG_ERR_DEVICE_TIMEOUT);
+  cp_async_wait_all();
+  if (tid == 0 && sh.mma_pend) mbar_wait(&sh.bar, sh.mma_ph, kSpinLimitNs);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

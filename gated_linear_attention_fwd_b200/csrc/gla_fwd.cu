@@ -83,6 +83,8 @@ struct OutSmem {
   uint64_t bar_a;  // P, qbar S'
   uint64_t bar_b;  // P V
   uint32_t tmem;
+  int mma_pend;    // thread 0: product group (0: P / qbar S', 1: P V) not yet seen complete, -1: none
+  uint32_t mma_ph;
 };
 
 // ============================================================== 2. state scan
@@ -244,7 +246,8 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
   const int nunits = a.B * a.H * a.nchunks;
   const bool with_y = a.y != nullptr && a.r != nullptr;
   uint32_t ph = 0;
-  bool timed_out = false;
+  bool timed_out = false;  // a wait of this thread gave up: the CTA stops after this unit
+  if (tid == 0) sh.mma_pend = -1;
 
   // Row pieces of a unit, loaded one unit ahead: q, k, gate factors, entry-state
   // rows and 2^r are issued as soon as the current unit's operands are written,
@@ -383,12 +386,15 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
       mma_issue<NTG, NTG, DKP / 16>(tmem + OC::TM_P, dAQ, Cfg::AQ_SZ, 256, dBS, OC::BS_SZ, 256,
                                     idesc_bf16(128, OC::NB), false);  // [P | O] = qbar [kbar | S'^T]^T
       mma_commit(&sh.bar_a);
+      sh.mma_pend = 0;
+      sh.mma_ph = ph;
     }
     if (has_next) {  // this unit's row pieces are consumed
       issue_rows(un, rows_next);
       issue_s(un);
     }
-    if (!mbar_wait(&sh.bar_a, ph, kSpinLimitNs)) timed_out = true;
+    if (!mbar_wait(&sh.bar_a, ph, spin_limit(a))) timed_out = true;
+    else if (tid == 0) sh.mma_pend = -1;
     tc_fence_after();
     // ---- mask P (s <= t) and store it as bf16 terms in TMEM, one K-step of 16 at a time
     if (32 * wq < C) {  // warp-uniform: lanes that are token rows
@@ -423,18 +429,23 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
       tmem_st_wait();
     }
     tc_fence_before();
-    __syncthreads();
+    const bool stop = __syncthreads_or(timed_out);  // a wait gave up: no further products
     tc_fence_after();
-    if (tid == 0) {
+    if (tid == 0 && !stop) {
       mma_issue_ts<NTG, NTV, C / 16>(tmem + OC::TM_O, tmem + OC::TM_PT, OC::PT_STRIDE, dVRm, Cfg::VR_SZ,
                                      2 * Cfg::SBO_V, idesc_bf16(128, DVP, false, true), true);
       mma_commit(&sh.bar_b);
+      sh.mma_pend = 1;
+      sh.mma_ph = ph;
     }
-    if (!mbar_wait(&sh.bar_b, ph, kSpinLimitNs)) timed_out = true;
+    if (!stop) {
+      if (!mbar_wait(&sh.bar_b, ph, spin_limit(a))) timed_out = true;
+      else if (tid == 0) sh.mma_pend = -1;
+    }
     ph ^= 1u;
     tc_fence_after();
     const int hn = has_next ? Unit(a, un).h : 0;
-    if (has_next) load_v_rows_t<C, DK, DV, TIN>(a, hn, rows_next, a.v, sbase + OC::OFF_VR);  // v of this unit is consumed
+    if (has_next && !stop) load_v_rows_t<C, DK, DV, TIN>(a, hn, rows_next, a.v, sbase + OC::OFF_VR);  // v of this unit is consumed
     if (!kAhead) issue_r(U.h, rows);
     if (tid < 128) stage_o<C, DK, DV, TIN, 0>(tmem, stage, sh.red);
     else stage_o<C, DK, DV, TIN, 1>(tmem, stage, sh.red);
@@ -478,9 +489,14 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
       }
     }
     if (has_next) issue_r(hn, rows_next);
-    __syncthreads();  // staging and row sums are rewritten by the next unit
+    // staging and row sums are rewritten by the next unit; after a wait gave up
+    // anywhere in the CTA, no further unit starts
+    if (__syncthreads_or(timed_out)) break;
   }
+  // ---- drain: this thread's row copies, and the last products, complete before exit
   if (timed_out) set_status(a.status, DIG_ERR_DEVICE_TIMEOUT);
+  cp_async_wait_all();
+  if (tid == 0 && sh.mma_pend >= 0) mbar_wait(sh.mma_pend ? &sh.bar_b : &sh.bar_a, sh.mma_ph, kSpinLimitNs);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
