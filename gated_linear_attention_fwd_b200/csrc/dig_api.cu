@@ -60,6 +60,8 @@ int chunk_len(int dtype, bool backward, int dk, int dv) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+}  // namespace
+
 // Bound of the kernels' device waits: DIG_DEVICE_WAIT_LIMIT_NS in the environment
 // (a test hook that makes a wait run out on purpose), else the two-second default.
 unsigned long long spin_limit_ns() {
@@ -89,7 +91,6 @@ dig_status check_common(int B, int H, int L, int d_k, int d_v, int grid_h, int g
   return DIG_OK;
 }
 
-}  // namespace
 }  // namespace dig
 
 using namespace dig;

@@ -38,6 +38,11 @@ struct GlaArgs {
   uint32_t* flist;   // backward: [0] count, [1..] units the fp16 gradient kernel left to the exact one
                      // (the exact kernel then processes only those; NULL: every unit)
   unsigned long long spin_ns;  // bound of a device wait in ns (0: the default of two seconds)
+  // value gate and state input / output (the extended entry points; all NULL otherwise)
+  const float* zb;   // value-gate logits [B, L, gate_heads, DV] (grid order)
+  float* gEQb;       // [B * gate_heads][L (scan order)][DV]   2^(e - rho), e the value-gate cumsum
+  float* gCHb;       // [B * gate_heads][nchunks][4][DV]       2^rho, 2^(Gb - rho), 2^Gb, Gb
+  float* sfin;       // [nseq][DV][DK] the state after the last chunk (written by the forward scan)
 };
 
 // Kernel-variant selection: chunk length, split count, head dims, types.

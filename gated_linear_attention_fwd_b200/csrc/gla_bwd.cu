@@ -229,9 +229,11 @@ __device__ __forceinline__ void stage_key_grads(uint8_t* smem, const float* dq, 
   }
 }
 
-// dv of this thread's token (TMEM lane t) and channel half -> staging row.
+// dv of this thread's token (TMEM lane t) and channel half -> staging row.  With
+// a value gate (`eqb`: the unit's rows of 2^(e - rho)) the product is the
+// gradient of vbar = v / EQb and is rescaled to dv = dvbar / EQb.
 template <int C, int DK, int DV, typename TIN, typename TOUT, int H>
-__device__ __forceinline__ void stage_dv(uint32_t tmem, uint8_t* smem) {
+__device__ __forceinline__ void stage_dv(uint32_t tmem, uint8_t* smem, const float* eqb = nullptr, int nvalid = 0) {
   using K = ChunkCfg<C, DK, DV, TIN>;
   using BC = BwdCfg<C, DK, DV, TIN, TOUT>;
   constexpr int VO = H ? K::DV0 : 0, VN = H ? K::DV1 : K::DV0;
@@ -242,12 +244,21 @@ __device__ __forceinline__ void stage_dv(uint32_t tmem, uint8_t* smem) {
 #pragma unroll
   for (int c = 0; c < VN; c += 8) tmem_ld8(lt + c, v + c);
   tmem_ld_wait();
+  if (eqb != nullptr && t < nvalid) {
+#pragma unroll
+    for (int i = 0; i < VN; ++i) v[i] = __fdiv_rn(v[i], __ldg(eqb + (size_t)t * DV + VO + i));
+  }
   TOUT* sv = reinterpret_cast<TOUT*>(smem + BC::OFF_SV + t * BC::VSB) + VO;
 #pragma unroll
   for (int c = 0; c < VN; c += 4) st_out4(sv + c, v + c);
 }
 
-template <int C, int DK, int DV, typename TIN, typename TOUT>
+// With EXT (value gate and state input / output, fp32 inputs): v and dO are
+// loaded as vbar = v / EQb and dObar = dO EQb, S' and Gt carry the value-side
+// references 2^rho and 2^(Gb - rho) of their rows, dv is rescaled by 1 / EQb, and
+// the last chunk's boundary term uses the final state (its G is the gradient of
+// the final state, zero when none is given).
+template <int C, int DK, int DV, typename TIN, typename TOUT, bool EXT = false>
 __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a) {
   using K = ChunkCfg<C, DK, DV, TIN>;
   using BC = BwdCfg<C, DK, DV, TIN, TOUT>;
@@ -345,23 +356,26 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
   constexpr uint32_t SB = DV * DK * 4;
   auto issue_states = [&](int u) {
     const Unit U(a, u);
-    const bool has_next_chunk = U.n + 1 < a.nchunks;  // G of the last chunk is zero
+    const bool has_next_chunk = U.n + 1 < a.nchunks;  // G of the last chunk is zero without EXT
+    const bool has_bnd = has_next_chunk || EXT;
+    const float* s_next = has_next_chunk ? a.dsn + (size_t)(u + 1) * DV * DK : a.sfin + (size_t)U.bh * DV * DK;
     sh.st_pend = 1;
     sh.st_ph = ph;
-    mbar_arrive_expect_tx(&sh.sbar, 2 * SB + (has_next_chunk ? SB : 0u) + 2 * DK * 4);
+    mbar_arrive_expect_tx(&sh.sbar, 2 * SB + (has_bnd ? SB : 0u) + 2 * DK * 4);
     bulk_copy_g2s(sbase + BC::OFF_SP, a.dsn + (size_t)u * DV * DK, SB, &sh.sbar);
     bulk_copy_g2s(sbase + BC::OFF_GT, a.dhn + (size_t)u * DV * DK, SB, &sh.sbar);
-    if (has_next_chunk) bulk_copy_g2s(sbase + BC::OFF_Q, a.dsn + (size_t)(u + 1) * DV * DK, SB, &sh.sbar);
+    if (has_bnd) bulk_copy_g2s(sbase + BC::OFF_Q, s_next, SB, &sh.sbar);
     bulk_copy_g2s(smem_u32(sh.gch), a.gCH + ((size_t)U.bz * a.nchunks + U.n) * 4 * DK, 2 * DK * 4, &sh.sbar);
   };
   // The kernel before this one is the state scan, which writes only the chunk
   // states and state gradients; everything older has completed.  So the first
   // unit's other rows are requested before the wait for that scan.
+  constexpr int VSV = EXT ? VS_VBAR : VS_NONE, VSD = EXT ? VS_DOBAR : VS_NONE;
   auto first_rows = [&](int u0) {
-    const int h0 = Unit(a, u0).h;
+    const Unit U0(a, u0);
     if constexpr (PRE) issue_qk(u0, sh.rows[0]);
-    load_v_rows_t<C, DK, DV, TIN>(a, h0, sh.rows[0], a.v, sbase + BC::OFF_V);
-    load_v_rows_t<C, DK, DV, TIN>(a, h0, sh.rows[0], a.dO, sbase + BC::OFF_DO);
+    load_v_rows_t<C, DK, DV, TIN, 256, VSV>(a, U0.h, sh.rows[0], a.v, sbase + BC::OFF_V, U0.bz, U0.n);
+    load_v_rows_t<C, DK, DV, TIN, 256, VSD>(a, U0.h, sh.rows[0], a.dO, sbase + BC::OFF_DO, U0.bz, U0.n);
   };
   if (!listed && (int)blockIdx.x < nunits) first_rows(blockIdx.x);
   griddep_wait();  // the kernels before this one have completed
@@ -387,6 +401,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
     if (has_next) fill_rows(a, un, C, rows_next);  // read after the operand barrier
     // ---- the state blocks, read in place: S' and Gt rows (to registers) and the boundary term
     const bool has_next_chunk = U.n + 1 < a.nchunks;
+    const bool has_bnd = has_next_chunk || EXT;
     if (!mbar_wait(&sh.sbar, ph, spin_limit(a))) timed_out = true;
     else if (tid == 0) sh.st_pend = 0;
     float spv[K::NPS][4], gtv[K::NPS][4];
@@ -399,15 +414,21 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
       const int off = (in ? jr * DK : 0) + 4 * g;
       const float4 sv = *reinterpret_cast<const float4*>(smem + BC::OFF_SP + 4 * off);
       const float4 gv = *reinterpret_cast<const float4*>(smem + BC::OFF_GT + 4 * off);
-      const float4 nv = has_next_chunk ? *reinterpret_cast<const float4*>(smem + BC::OFF_Q + 4 * off)
+      const float4 nv = has_bnd ? *reinterpret_cast<const float4*>(smem + BC::OFF_Q + 4 * off)
                                        : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float4 c0 = *reinterpret_cast<const float4*>(&sh.gch[4 * g]);
-      const float4 c1 = *reinterpret_cast<const float4*>(&sh.gch[DK + 4 * g]);
-      spv[j][0] = sv.x * c0.x;  // S' = 2^r S_n
+      float4 c0 = *reinterpret_cast<const float4*>(&sh.gch[4 * g]);
+      float4 c1 = *reinterpret_cast<const float4*>(&sh.gch[DK + 4 * g]);
+      if constexpr (EXT) {  // the row's value-side references: 2^rho (S'), 2^(Gb - rho) (Gt)
+        const float* chb = a.gCHb + ((size_t)U.bz * a.nchunks + U.n) * 4 * DV + (in ? jr : 0);
+        const float rb = __ldg(chb), gb = __ldg(chb + DV);
+        c0 = make_float4(c0.x * rb, c0.y * rb, c0.z * rb, c0.w * rb);
+        c1 = make_float4(c1.x * gb, c1.y * gb, c1.z * gb, c1.w * gb);
+      }
+      spv[j][0] = sv.x * c0.x;  // S' = 2^r S_n (2^rho with a value gate)
       spv[j][1] = sv.y * c0.y;
       spv[j][2] = sv.z * c0.z;
       spv[j][3] = sv.w * c0.w;
-      gtv[j][0] = gv.x * c1.x;  // Gt = 2^(Gamma - r) G_n
+      gtv[j][0] = gv.x * c1.x;  // Gt = 2^(Gamma - r) G_n (2^(Gb - rho))
       gtv[j][1] = gv.y * c1.y;
       gtv[j][2] = gv.z * c1.z;
       gtv[j][3] = gv.w * c1.w;
@@ -535,9 +556,9 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
     wait_all(4);
     // v and dO are no longer read: the next unit's rows start to arrive now
     if (has_next && !timed_out && !stop) {
-      const int hn = Unit(a, un).h;
-      load_v_rows_t<C, DK, DV, TIN>(a, hn, rows_next, a.v, sbase + BC::OFF_V);
-      load_v_rows_t<C, DK, DV, TIN>(a, hn, rows_next, a.dO, sbase + BC::OFF_DO);
+      const Unit Un(a, un);
+      load_v_rows_t<C, DK, DV, TIN, 256, VSV>(a, Un.h, rows_next, a.v, sbase + BC::OFF_V, Un.bz, Un.n);
+      load_v_rows_t<C, DK, DV, TIN, 256, VSD>(a, Un.h, rows_next, a.dO, sbase + BC::OFF_DO, Un.bz, Un.n);
     }
     mask_to_terms<C, BC::PT_STRIDE>(tmem, BC::TM_R, false);
     tmem_st_wait();
@@ -551,6 +572,8 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
     wait_all(5);
     ph ^= 1u;
     // ---- dq, dk and the tokens' d log alpha terms from TMEM, the operands and EQ
+    const float* eqb = EXT ? a.gEQb + ((size_t)U.bz * a.L + (size_t)U.n * C) * DV : nullptr;
+    const int nvalid = min(C, a.L - U.n * C);
     float dq[KL], dk[KL];
     if (tid < 128) key_grads<C, DK, DV, TIN, TOUT, 0>(tmem, sbase, EQ, dq, dk);
     else key_grads<C, DK, DV, TIN, TOUT, 1>(tmem, sbase, EQ, dq, dk);
@@ -559,8 +582,8 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
     if (tid < 128) stage_key_grads<C, DK, DV, TIN, TOUT, 0>(smem, dq, dk);
     else stage_key_grads<C, DK, DV, TIN, TOUT, 1>(smem, dq, dk);
     if constexpr (BC::ONE_PASS) {
-      if (tid < 128) stage_dv<C, DK, DV, TIN, TOUT, 0>(tmem, smem);
-      else stage_dv<C, DK, DV, TIN, TOUT, 1>(tmem, smem);
+      if (tid < 128) stage_dv<C, DK, DV, TIN, TOUT, 0>(tmem, smem, eqb, nvalid);
+      else stage_dv<C, DK, DV, TIN, TOUT, 1>(tmem, smem, eqb, nvalid);
     }
     tc_fence_before();
     __syncthreads();
@@ -595,8 +618,8 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
       store_dv();
     } else {
       __syncthreads();  // dq / dk staging read: dv takes its place
-      if (tid < 128) stage_dv<C, DK, DV, TIN, TOUT, 0>(tmem, smem);
-      else stage_dv<C, DK, DV, TIN, TOUT, 1>(tmem, smem);
+      if (tid < 128) stage_dv<C, DK, DV, TIN, TOUT, 0>(tmem, smem, eqb, nvalid);
+      else stage_dv<C, DK, DV, TIN, TOUT, 1>(tmem, smem, eqb, nvalid);
       __syncthreads();
       store_dv();
     }
@@ -834,6 +857,26 @@ cudaError_t launch_typed(const GlaArgs& a, bool saved, cudaStream_t s) {
   return launch_pdl(k, persistent_grid(BC::PER_SM, units), 256, BC::SMEM, s, b);
 }
 
+// Value gate and state input / output (fp32 inputs, exact kernels): gates, dS and
+// dH, the forward scan seeded with S_0 (its final carry, the final state, kept
+// for the last chunk's boundary term) and the reverse scan seeded with the final
+// state's gradient (its final carry is the gradient of S_0), then the gradients.
+template <int DK, int DV, typename TOUT>
+cudaError_t launch_typed_ext(const GlaArgs& a, const ScanEnds& ends, cudaStream_t s) {
+  constexpr int C = bwd_chunk_len(DK, DV, true);
+  using BC = BwdCfg<C, DK, DV, float, TOUT>;
+  const long long units = (long long)a.B * a.H * a.nchunks;
+  if (units <= 0) return cudaSuccess;
+  cudaError_t e;
+  if ((e = launch_chunk_state<C, DK, DV, float, true, true>(a, s)) != cudaSuccess) return e;
+  if ((e = launch_state_scan(a, a.dsn, false, a.dhn, true, DK, DV, s, nullptr, &ends)) != cudaSuccess) return e;
+  GlaArgs b = a;
+  b.flist = nullptr;
+  auto k = gla_chunk_grad_kernel<C, DK, DV, float, TOUT, true>;
+  if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, BC::SMEM)) != cudaSuccess) return e;
+  return launch_pdl(k, persistent_grid(BC::PER_SM, units), 256, BC::SMEM, s, b);
+}
+
 template <int DK, int DV>
 cudaError_t dispatch_types(const GlaVariant& v, const GlaArgs& a, bool saved, cudaStream_t s) {
   using bf = __nv_bfloat16;
@@ -853,6 +896,18 @@ cudaError_t launch_gla_bwd(const GlaVariant& v, const GlaArgs& a, bool saved, cu
   if (v.dk == 32 && v.dv == 64) return dispatch_types<32, 64>(v, a, saved, s);
   if (v.dk == 36 && v.dv == 72) return dispatch_types<36, 72>(v, a, saved, s);
   if (v.dk == 64 && v.dv == 64) return dispatch_types<64, 64>(v, a, saved, s);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_gla_bwd_ext(const GlaVariant& v, const GlaArgs& a, const ScanEnds& ends, cudaStream_t s) {
+  if (v.tin != DIG_F32 || v.chunk != bwd_chunk_len(v.dk, v.dv, true)) return cudaErrorInvalidValue;
+  const bool bf = v.tout == DIG_BF16;
+  if (v.dk == 32 && v.dv == 64)
+    return bf ? launch_typed_ext<32, 64, __nv_bfloat16>(a, ends, s) : launch_typed_ext<32, 64, float>(a, ends, s);
+  if (v.dk == 36 && v.dv == 72)
+    return bf ? launch_typed_ext<36, 72, __nv_bfloat16>(a, ends, s) : launch_typed_ext<36, 72, float>(a, ends, s);
+  if (v.dk == 64 && v.dv == 64)
+    return bf ? launch_typed_ext<64, 64, __nv_bfloat16>(a, ends, s) : launch_typed_ext<64, 64, float>(a, ends, s);
   return cudaErrorInvalidValue;
 }
 

@@ -124,12 +124,18 @@ __device__ __forceinline__ size_t tok_row(long long grow, const GlaArgs& a, int 
 // cp_async_wait_all); fp32 values are split into three bf16 terms.  Channels
 // DV..DVP are zeroed (they are a contracted dimension in some products).
 // NTH threads of the CTA share the pieces.
-template <int C, int DK, int DV, typename TIN, int NTH = 256>
+// With a value gate (VS != VS_NONE, fp32 inputs only) each row is scaled on the
+// way by its token's value-gate factor EQb = 2^(e - rho) of the unit's chunk
+// (gate row bz, chunk n): v / EQb (VS_VBAR), v 2^(Gb - rho) / EQb = v 2^(Gb - e)
+// (VS_VHAT), dO EQb (VS_DOBAR) or dO EQb 2^rho = dO 2^e (VS_DOE).
+enum { VS_NONE = 0, VS_VBAR = 1, VS_VHAT = 2, VS_DOBAR = 3, VS_DOE = 4 };
+template <int C, int DK, int DV, typename TIN, int NTH = 256, int VS = VS_NONE>
 __device__ __forceinline__ void load_v_rows_t(const GlaArgs& a, int h, const long long* rows, const void* src,
-                                              uint32_t vr) {
+                                              uint32_t vr, int bz = 0, int n = 0) {
   using Cfg = ChunkCfg<C, DK, DV, TIN>;
   constexpr int NPV = cdiv(C * Cfg::NGV, NTH);
   const int tid = threadIdx.x;
+  static_assert(VS == VS_NONE || std::is_same<TIN, float>::value, "value-gate scaling on the fp32 path only");
   if constexpr (std::is_same<TIN, __nv_bfloat16>::value) {
 #pragma unroll
     for (int j = 0; j < NPV; ++j) {
@@ -160,6 +166,20 @@ __device__ __forceinline__ void load_v_rows_t(const GlaArgs& a, int h, const lon
       if (i < C * Cfg::NGV) {
         float x[8];
         pv[j].unpack(x);
+        if constexpr (VS != VS_NONE) {
+          if (rows[t] >= 0) {
+            const float* eq = a.gEQb + ((size_t)bz * a.L + (size_t)n * C + t) * DV + 8 * g;
+            const float* ch = a.gCHb + ((size_t)bz * a.nchunks + n) * 4 * DV + 8 * g;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float f = __ldg(eq + e);
+              if constexpr (VS == VS_VBAR) x[e] = __fdiv_rn(x[e], f);
+              if constexpr (VS == VS_VHAT) x[e] = __fdiv_rn(x[e] * __ldg(ch + DV + e), f);
+              if constexpr (VS == VS_DOBAR) x[e] *= f;
+              if constexpr (VS == VS_DOE) x[e] *= f * __ldg(ch + e);
+            }
+          }
+        }
         st_piece<Cfg::NTV, 8>(vr, t, Cfg::SBO_V, 8 * g, Cfg::VR_SZ, x);
       }
     }
@@ -206,10 +226,10 @@ __global__ void __launch_bounds__(256) gla_gate_kernel(const GlaArgs a) {
   constexpr int NSG = 256 / DK;  // token segments of the cumsum
   constexpr int SEGL = cdiv(C, NSG);
   constexpr int NG = DK / 4;     // 4-channel groups of a token row
-  static_assert(NSG <= 8 && DK <= 64, "cumsum segments");
+  static_assert(NSG >= 1 && NSG <= 8 && DK % 4 == 0, "cumsum segments");
   __shared__ __align__(16) float G[C * GP];
-  __shared__ float segtot[8][64];
-  __shared__ float gam[64];
+  __shared__ float segtot[8][DK];
+  __shared__ float gam[DK];
   __shared__ long long grows[C];
   griddep_wait();  // the kernels before this one have completed
   griddep_launch_dependents();
@@ -228,8 +248,8 @@ __global__ void __launch_bounds__(256) gla_gate_kernel(const GlaArgs a) {
     for (int i = tid; i < C * NG; i += 256) {
       const int t = i / NG, g = i - t * NG;
       const long long gr = grows[t];
-      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);  // padding tokens do not decay
-      if (gr >= 0) {
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);  // padding tokens (and an absent gate) do not decay
+      if (gr >= 0 && a.z != nullptr) {
         const float4 zz = __ldg(reinterpret_cast<const float4*>(a.z + ((size_t)gr * a.gate_heads + hz) * DK) + g);
         x = make_float4(log2_decay(zz.x, a.inv_tau), log2_decay(zz.y, a.inv_tau), log2_decay(zz.z, a.inv_tau),
                         log2_decay(zz.w, a.inv_tau));
@@ -294,7 +314,9 @@ __global__ void __launch_bounds__(256) gla_gate_kernel(const GlaArgs a) {
 // gate kernel's factors.  With BWD it also forms the chunk's state-gradient
 // contribution dH = (q 2^b)^T dO, q 2^b = q EQ 2^r (to `dhn`), which the reverse
 // scan turns into the gradient of every chunk's exit state.
-template <int C, int DK, int DV, typename TIN, bool BWD>
+// With EXT (value gate, fp32 inputs) v is scaled to v 2^(Gb - e) and dO to dO 2^e
+// on load, so that dS and dH carry the value-side decays too.
+template <int C, int DK, int DV, typename TIN, bool BWD, bool EXT = false>
 __global__ void __launch_bounds__(256, StateCfg<C, DK, DV, TIN, BWD>::MINB) gla_chunk_state_kernel(const GlaArgs a) {
   using Cfg = ChunkCfg<C, DK, DV, TIN>;
   using SC = StateCfg<C, DK, DV, TIN, BWD>;
@@ -357,9 +379,10 @@ __global__ void __launch_bounds__(256, StateCfg<C, DK, DV, TIN, BWD>::MINB) gla_
     }
   };
   auto issue_vd = [&](int u, const long long* rows) {
-    const int h = Unit(a, u).h;
-    load_v_rows_t<C, DK, DV, TIN>(a, h, rows, a.v, sbase + SC::OFF_VR);
-    if constexpr (BWD) load_v_rows_t<C, DK, DV, TIN>(a, h, rows, a.dO, sbase + SC::OFF_DO);
+    const Unit U(a, u);
+    load_v_rows_t<C, DK, DV, TIN, 256, EXT ? VS_VHAT : VS_NONE>(a, U.h, rows, a.v, sbase + SC::OFF_VR, U.bz, U.n);
+    if constexpr (BWD)
+      load_v_rows_t<C, DK, DV, TIN, 256, EXT ? VS_DOE : VS_NONE>(a, U.h, rows, a.dO, sbase + SC::OFF_DO, U.bz, U.n);
   };
   if ((int)blockIdx.x < nunits) {
     issue_rows(blockIdx.x, sh.rows[0]);
@@ -507,8 +530,20 @@ inline int persistent_grid(int per_sm, long long units) {
 bool gla_reduce_tma_eligible(const GlaArgs& a, int dk, int dv, int tin, int chunk);
 cudaError_t launch_reduce_tma(const GlaArgs& a, bool bwd, cudaStream_t s, bool* launched);
 
-// Gate kernel, then chunk-state kernel (which reads the gate factors).
-template <int C, int DK, int DV, typename TIN, bool BWD>
+// The value gate's factors: the gate kernel over the value channels, from zb
+// into gEQb / gCHb.
+template <int C, int DV>
+cudaError_t launch_value_gate(const GlaArgs& a, cudaStream_t s) {
+  GlaArgs g = a;
+  g.z = a.zb;
+  g.gEQ = a.gEQb;
+  g.gCH = a.gCHb;
+  const long long gunits = (long long)a.B * a.gate_heads * a.nchunks;
+  return launch_pdl(gla_gate_kernel<C, DV>, dim3(persistent_grid(4, gunits)), dim3(256), 0, s, g);
+}
+
+// Gate kernel(s), then chunk-state kernel (which reads the gate factors).
+template <int C, int DK, int DV, typename TIN, bool BWD, bool EXT = false>
 cudaError_t launch_chunk_state(const GlaArgs& a, cudaStream_t s) {
   using SC = StateCfg<C, DK, DV, TIN, BWD>;
   const long long units = (long long)a.B * a.H * a.nchunks;
@@ -516,22 +551,34 @@ cudaError_t launch_chunk_state(const GlaArgs& a, cudaStream_t s) {
   const long long gunits = (long long)a.B * a.gate_heads * a.nchunks;
   cudaError_t e = launch_pdl(gla_gate_kernel<C, DK>, dim3(persistent_grid(4, gunits)), dim3(256), 0, s, a);
   if (e != cudaSuccess) return e;
-  if (std::is_same<TIN, __nv_bfloat16>::value && gla_reduce_tma_eligible(a, DK, DV, DIG_BF16, C)) {
+  if constexpr (EXT) {
+    if ((e = launch_value_gate<C, DV>(a, s)) != cudaSuccess) return e;
+  }
+  if (!EXT && std::is_same<TIN, __nv_bfloat16>::value && gla_reduce_tma_eligible(a, DK, DV, DIG_BF16, C)) {
     bool launched = false;
     if ((e = launch_reduce_tma(a, false, s, &launched)) != cudaSuccess) return e;
     if (launched && BWD && (e = launch_reduce_tma(a, true, s, &launched)) != cudaSuccess) return e;
     if (launched) return cudaSuccess;
   }
-  auto k1 = gla_chunk_state_kernel<C, DK, DV, TIN, BWD>;
+  auto k1 = gla_chunk_state_kernel<C, DK, DV, TIN, BWD, EXT>;
   if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, SC::SMEM)) != cudaSuccess) return e;
   return launch_pdl(k1, persistent_grid(SC::PER_SM, units), 256, SC::SMEM, s, a);
 }
 
+// Optional ends of the scans (per buffer): the carry entering the first step
+// (NULL: zero) and the carry after the last step, written in the caller's
+// [B*H][DK][DV] layout (fin) and in the state layout [B*H][DV][DK] (fin_rows).
+struct ScanEnds {
+  const float* seed[2];
+  float* fin[2];
+  float* fin_rows[2];
+};
 // Scan of per-chunk contributions X_n (DV x DK fp32 each, per sequence) into
-// the state entering every chunk: Y_0 = 0, Y_{n+1} = diag(2^Gamma_n) Y_n + X_n
-// (reverse: the same recurrence from the last chunk down, giving the gradient
-// leaving every chunk).  In place in buf0 and, when not null, buf1 (one launch).
+// the state entering every chunk: Y_0 = 0 (or the seed), Y_{n+1} =
+// diag(2^Gamma_n) Y_n diag(2^Gb_n) + X_n (Gb = 0 without a value gate; reverse:
+// the same recurrence from the last chunk down, giving the gradient leaving
+// every chunk).  In place in buf0 and, when not null, buf1 (one launch).
 cudaError_t launch_state_scan(const GlaArgs& a, float* buf0, bool rev0, float* buf1, bool rev1, int dk, int dv,
-                              cudaStream_t s, uint32_t* zero_word = nullptr);
+                              cudaStream_t s, uint32_t* zero_word = nullptr, const ScanEnds* ends = nullptr);
 
 }  // namespace dig

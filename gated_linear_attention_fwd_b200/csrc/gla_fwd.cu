@@ -97,12 +97,16 @@ struct OutSmem {
 // the passes (two memory round trips in all); longer ones stream in windows.
 // blockIdx.y selects one of two buffers (the backward scans its states forward
 // and its state gradients in reverse in one launch); `reverse` runs the chunks
-// from the last to the first.
+// from the last to the first.  With a value gate the decay of element (j, c) is
+// 2^Gamma[c] 2^Gb[j].  The carry entering the first step is zero or a given
+// seed (S_0, or the gradient of the final state), and the carry after the last
+// step (the final state, or the gradient of S_0) can be written out.
 constexpr int kScanRanges = 16, kScanQuads = 16, kScanWindow = 8;
 struct ScanJob {
   float* buf[2];
   int reverse[2];
   uint32_t* zero_word;  // set to 0 by the scan (the count of the backward's unit list), or NULL
+  ScanEnds ends;
 };
 __global__ void __launch_bounds__(kScanRanges * kScanQuads, 2) gla_state_scan_kernel(const GlaArgs a, ScanJob job,
                                                                                      int dk, int dv) {
@@ -127,11 +131,28 @@ __global__ void __launch_bounds__(kScanRanges * kScanQuads, 2) gla_state_scan_ke
   float4* st = reinterpret_cast<float4*>(buf + (size_t)bh * nch * dv * dk) + quad;
   const size_t st_stride = (size_t)nq;
   const float* dec = a.gCH + ((size_t)bz * nch * 4 + 2) * dk + c0;  // 2^Gamma of chunk n at dec + n * 4 * dk
+  const int jrow = (quad * 4) / dk;                                   // the quad's value channel
+  const float* decb = a.gCHb ? a.gCHb + ((size_t)bz * nch * 4 + 2) * dv + jrow : nullptr;  // 2^Gb[j]
   auto at = [&](int n) { return reverse ? nch - 1 - n : n; };         // physical chunk of scan step n
   auto fma4 = [](float4 g, float4 s, float4 d) {
     return make_float4(fmaf(g.x, s.x, d.x), fmaf(g.y, s.y, d.y), fmaf(g.z, s.z, d.z), fmaf(g.w, s.w, d.w));
   };
   auto mul4 = [](float4 g, float4 x) { return make_float4(g.x * x.x, g.y * x.y, g.z * x.z, g.w * x.w); };
+  auto decay = [&](int n) {  // the element decay of physical chunk n
+    float4 g = __ldg(reinterpret_cast<const float4*>(dec + (size_t)n * 4 * dk));
+    if (decb != nullptr) {
+      const float gb = __ldg(decb + (size_t)n * 4 * dv);
+      g = make_float4(g.x * gb, g.y * gb, g.z * gb, g.w * gb);
+    }
+    return g;
+  };
+  const int side = blockIdx.y;
+  const float* seed = job.ends.seed[side];
+  float4 seed4 = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (seed != nullptr && act) {  // [B*H][DK][DV]: element (j, c) at c * dv + j
+    const float* sp = seed + (size_t)bh * dk * dv + (size_t)c0 * dv + jrow;
+    seed4 = make_float4(__ldg(sp), __ldg(sp + dv), __ldg(sp + 2 * dv), __ldg(sp + 3 * dv));
+  }
   float4 A = make_float4(1.f, 1.f, 1.f, 1.f), s = make_float4(0.f, 0.f, 0.f, 0.f);
   float4 d[kScanWindow];
   const bool resident = per <= kScanWindow;  // uniform: one window holds the whole range
@@ -141,7 +162,7 @@ __global__ void __launch_bounds__(kScanRanges * kScanQuads, 2) gla_state_scan_ke
 #pragma unroll
       for (int e = 0; e < kScanWindow; ++e) {
         if (w0 + e < n1) {
-          g[e] = __ldg(reinterpret_cast<const float4*>(dec + (size_t)at(w0 + e) * 4 * dk));
+          g[e] = decay(at(w0 + e));
           d[e] = __ldcg(st + at(w0 + e) * st_stride);
         }
       }
@@ -158,14 +179,27 @@ __global__ void __launch_bounds__(kScanRanges * kScanQuads, 2) gla_state_scan_ke
   sS[rg][lq] = s;
   __syncthreads();
   if (!act) return;
-  float4 S = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (rg == 0 && (job.ends.fin[side] != nullptr || job.ends.fin_rows[side] != nullptr)) {
+    float4 F = seed4;  // the carry after the last step: every range folded onto the seed
+    for (int m = 0; m < kScanRanges; ++m) F = fma4(sA[m][lq], F, sS[m][lq]);
+    if (job.ends.fin_rows[side] != nullptr)
+      reinterpret_cast<float4*>(job.ends.fin_rows[side] + (size_t)bh * dk * dv)[quad] = F;
+    if (job.ends.fin[side] != nullptr) {
+      float* fp = job.ends.fin[side] + (size_t)bh * dk * dv + (size_t)c0 * dv + jrow;
+      fp[0] = F.x;
+      fp[dv] = F.y;
+      fp[2 * dv] = F.z;
+      fp[3 * dv] = F.w;
+    }
+  }
+  float4 S = seed4;
   for (int m = 0; m < rg; ++m) S = fma4(sA[m][lq], S, sS[m][lq]);
   if (resident) {  // the range's contributions are still in registers; its decays are reread (L1)
 #pragma unroll
     for (int e = 0; e < kScanWindow; ++e) {
       if (n0 + e < n1) {
         __stcg(st + at(n0 + e) * st_stride, S);
-        S = fma4(__ldg(reinterpret_cast<const float4*>(dec + (size_t)at(n0 + e) * 4 * dk)), S, d[e]);
+        S = fma4(decay(at(n0 + e)), S, d[e]);
       }
     }
     return;
@@ -175,7 +209,7 @@ __global__ void __launch_bounds__(kScanRanges * kScanQuads, 2) gla_state_scan_ke
 #pragma unroll
     for (int e = 0; e < kScanWindow; ++e) {
       if (w0 + e < n1) {
-        g[e] = __ldg(reinterpret_cast<const float4*>(dec + (size_t)at(w0 + e) * 4 * dk));
+        g[e] = decay(at(w0 + e));
         d[e] = __ldcg(st + at(w0 + e) * st_stride);
       }
     }
@@ -190,8 +224,13 @@ __global__ void __launch_bounds__(kScanRanges * kScanQuads, 2) gla_state_scan_ke
 }
 
 // ============================================================== 3. outputs
+// O rows (TMEM lane t = token t) of this thread's channel half -> staging and
+// the row's partial sum of squares.  With a value gate (`eqb`: the unit's rows
+// of 2^(e - rho), NULL otherwise) the product P vbar + qbar S'^T is rescaled to
+// o = EQb (P vbar + qbar S'^T) first; `nvalid` tokens of the chunk are real.
 template <int C, int DK, int DV, typename TIN, int H>
-__device__ __forceinline__ void stage_o(uint32_t tmem, float* stage, float* red) {
+__device__ __forceinline__ void stage_o(uint32_t tmem, float* stage, float* red, const float* eqb = nullptr,
+                                        int nvalid = 0) {
   using Cfg = ChunkCfg<C, DK, DV, TIN>;
   using OC = OutCfg<C, DK, DV, TIN>;
   constexpr int VO = H ? Cfg::DV0 : 0, VN = H ? Cfg::DV1 : Cfg::DV0;
@@ -201,6 +240,10 @@ __device__ __forceinline__ void stage_o(uint32_t tmem, float* stage, float* red)
   for (int c = 0; c < cround(VN, 8); c += 8)
     tmem_ld8(tmem + (static_cast<uint32_t>(32 * wq) << 16) + OC::TM_O + VO + c, ov + c);
   tmem_ld_wait();
+  if (eqb != nullptr && t < nvalid) {
+#pragma unroll
+    for (int i = 0; i < VN; ++i) ov[i] *= __ldg(eqb + (size_t)t * DV + VO + i);
+  }
   float ss = 0.f;
 #pragma unroll
   for (int i = 0; i < VN; ++i) ss += ov[i] * ov[i];
@@ -213,7 +256,9 @@ __device__ __forceinline__ void stage_o(uint32_t tmem, float* stage, float* red)
   }
 }
 
-template <int C, int DK, int DV, typename TIN, typename TOUT>
+// With EXT (value gate, fp32 inputs): v is loaded as vbar = v / EQb, the S'^T
+// rows carry 2^rho of their value channel, and the output is rescaled by EQb.
+template <int C, int DK, int DV, typename TIN, typename TOUT, bool EXT = false>
 __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) {
   using Cfg = ChunkCfg<C, DK, DV, TIN>;
   using OC = OutCfg<C, DK, DV, TIN>;
@@ -305,11 +350,12 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
   // The kernel before this one is the state scan, which writes only the chunk
   // states; everything older has completed.  So the first unit's other rows are
   // requested before the wait for that scan.
+  constexpr int VSV = EXT ? VS_VBAR : VS_NONE;
   if (kAhead && (int)blockIdx.x < nunits) {
-    const int h0 = Unit(a, blockIdx.x).h;
+    const Unit U0(a, blockIdx.x);
     issue_rows(blockIdx.x, sh.rows[0]);
-    load_v_rows_t<C, DK, DV, TIN>(a, h0, sh.rows[0], a.v, sbase + OC::OFF_VR);
-    issue_r(h0, sh.rows[0]);
+    load_v_rows_t<C, DK, DV, TIN, 256, VSV>(a, U0.h, sh.rows[0], a.v, sbase + OC::OFF_VR, U0.bz, U0.n);
+    issue_r(U0.h, sh.rows[0]);
   }
   griddep_wait();  // the kernels before this one have completed
   griddep_launch_dependents();
@@ -329,7 +375,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
       }
       issue_rows(u, rows);
       issue_s(u);
-      load_v_rows_t<C, DK, DV, TIN>(a, U.h, rows, a.v, sbase + OC::OFF_VR);
+      load_v_rows_t<C, DK, DV, TIN, 256, VSV>(a, U.h, rows, a.v, sbase + OC::OFF_VR, U.bz, U.n);
     }
     if (has_next) fill_rows(a, un, C, rows_next);  // visible after the next barrier
     // ---- operands: qbar = q 2^(b-r), kbar = k 2^(r-b); S'^T rows = (2^r S_n)[:, j]
@@ -363,17 +409,23 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
         float sv[4], cv[4];
         ps[j].unpack(sv);
         pc[j].unpack(cv);
+        // value-gate reference of the row's value channel (1 without a value gate)
+        const float rb = EXT ? __ldg(a.gCHb + ((size_t)U.bz * a.nchunks + U.n) * 4 * DV + jr) : 1.f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) sv[e] *= cv[e];
+        for (int e = 0; e < 4; ++e) sv[e] *= cv[e] * rb;
         st_piece<NTG, 4>(sSPT, jr, Cfg::SBO_K, 4 * g, OC::BS_SZ, sv);
       }
     }
     if constexpr (Cfg::NPAD > 0) {  // zero K padding (the output staging of the previous unit overwrote it)
+      // of the C token rows of qbar and kbar and of the DV rows of S'^T (more than C when d_v > C)
       const float zz[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int i = tid; i < C * Cfg::NPAD; i += 256) {
+      constexpr int NR = C > DV ? C : DV;
+      for (int i = tid; i < NR * Cfg::NPAD; i += 256) {
         const int row = i / Cfg::NPAD, c = DK + 4 * (i % Cfg::NPAD);
-        st_piece<NTG, 4>(sbase + OC::OFF_AQ, row, Cfg::SBO_K, c, Cfg::AQ_SZ, zz);
-        st_piece<NTG, 4>(sbase + OC::OFF_BS, row, Cfg::SBO_K, c, OC::BS_SZ, zz);
+        if (row < C) {
+          st_piece<NTG, 4>(sbase + OC::OFF_AQ, row, Cfg::SBO_K, c, Cfg::AQ_SZ, zz);
+          st_piece<NTG, 4>(sbase + OC::OFF_BS, row, Cfg::SBO_K, c, OC::BS_SZ, zz);
+        }
         if (row < DV) st_piece<NTG, 4>(sSPT, row, Cfg::SBO_K, c, OC::BS_SZ, zz);
       }
     }
@@ -444,11 +496,15 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
     }
     ph ^= 1u;
     tc_fence_after();
-    const int hn = has_next ? Unit(a, un).h : 0;
-    if (has_next && !stop) load_v_rows_t<C, DK, DV, TIN>(a, hn, rows_next, a.v, sbase + OC::OFF_VR);  // v of this unit is consumed
+    const Unit Un(a, has_next ? un : u);
+    const int hn = Un.h;
+    if (has_next && !stop)  // v of this unit is consumed
+      load_v_rows_t<C, DK, DV, TIN, 256, VSV>(a, hn, rows_next, a.v, sbase + OC::OFF_VR, Un.bz, Un.n);
     if (!kAhead) issue_r(U.h, rows);
-    if (tid < 128) stage_o<C, DK, DV, TIN, 0>(tmem, stage, sh.red);
-    else stage_o<C, DK, DV, TIN, 1>(tmem, stage, sh.red);
+    const float* eqb = EXT ? a.gEQb + ((size_t)U.bz * a.L + (size_t)U.n * C) * DV : nullptr;
+    const int nvalid = min(C, a.L - U.n * C);
+    if (tid < 128) stage_o<C, DK, DV, TIN, 0>(tmem, stage, sh.red, eqb, nvalid);
+    else stage_o<C, DK, DV, TIN, 1>(tmem, stage, sh.red, eqb, nvalid);
     tc_fence_before();
     __syncthreads();
     // ---- o and y rows, 8 channels per piece
@@ -521,12 +577,12 @@ int num_sms() {
 }
 
 cudaError_t launch_state_scan(const GlaArgs& a, float* buf0, bool rev0, float* buf1, bool rev1, int dk, int dv,
-                              cudaStream_t s, uint32_t* zero_word) {
+                              cudaStream_t s, uint32_t* zero_word, const ScanEnds* ends) {
   const int nq = dv * dk / 4;
   const long long blocks = (long long)a.B * a.H * ((nq + kScanQuads - 1) / kScanQuads);
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 2147483647LL) return cudaErrorInvalidValue;
-  ScanJob job{{buf0, buf1}, {rev0 ? 1 : 0, rev1 ? 1 : 0}, zero_word};
+  ScanJob job{{buf0, buf1}, {rev0 ? 1 : 0, rev1 ? 1 : 0}, zero_word, ends ? *ends : ScanEnds{}};
   return launch_pdl(gla_state_scan_kernel, dim3((unsigned)blocks, buf1 ? 2u : 1u), kScanRanges * kScanQuads, 0, s, a,
                     job, dk, dv);
 }
@@ -536,21 +592,21 @@ cudaError_t launch_out_tma(const GlaArgs& a, int tout, cudaStream_t s, bool* lau
 
 namespace {
 
-template <int C, int DK, int DV, typename TIN, typename TOUT>
-cudaError_t launch_typed(const GlaArgs& a, cudaStream_t s) {
+template <int C, int DK, int DV, typename TIN, typename TOUT, bool EXT = false>
+cudaError_t launch_typed(const GlaArgs& a, cudaStream_t s, const ScanEnds* ends = nullptr) {
   using OC = OutCfg<C, DK, DV, TIN>;
   const long long units = (long long)a.B * a.H * a.nchunks;
   if (units <= 0) return cudaSuccess;
-  cudaError_t e = launch_chunk_state<C, DK, DV, TIN, false>(a, s);
+  cudaError_t e = launch_chunk_state<C, DK, DV, TIN, false, EXT>(a, s);
   if (e != cudaSuccess) return e;
-  if ((e = launch_state_scan(a, a.dsn, false, nullptr, false, DK, DV, s)) != cudaSuccess) return e;
-  if (std::is_same<TIN, __nv_bfloat16>::value && gla_out_tma_eligible(a, DK, DV, DIG_BF16, C)) {
+  if ((e = launch_state_scan(a, a.dsn, false, nullptr, false, DK, DV, s, nullptr, ends)) != cudaSuccess) return e;
+  if (!EXT && std::is_same<TIN, __nv_bfloat16>::value && gla_out_tma_eligible(a, DK, DV, DIG_BF16, C)) {
     bool launched = false;
     if ((e = launch_out_tma(a, std::is_same<TOUT, float>::value ? DIG_F32 : DIG_BF16, s, &launched)) != cudaSuccess)
       return e;
     if (launched) return cudaGetLastError();
   }
-  auto k3 = gla_chunk_out_kernel<C, DK, DV, TIN, TOUT>;
+  auto k3 = gla_chunk_out_kernel<C, DK, DV, TIN, TOUT, EXT>;
   if ((e = cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, OC::SMEM)) != cudaSuccess) return e;
   if ((e = launch_pdl(k3, persistent_grid(2, units), 256, OC::SMEM, s, a)) != cudaSuccess) return e;
   return cudaGetLastError();
@@ -567,6 +623,12 @@ cudaError_t dispatch_types(const GlaVariant& v, const GlaArgs& a, cudaStream_t s
   return launch_typed<64, DK, DV, float, float>(a, s);
 }
 
+template <int DK, int DV>
+cudaError_t dispatch_ext(const GlaVariant& v, const GlaArgs& a, const ScanEnds& ends, cudaStream_t s) {
+  if (v.tout == DIG_BF16) return launch_typed<64, DK, DV, float, __nv_bfloat16, true>(a, s, &ends);
+  return launch_typed<64, DK, DV, float, float, true>(a, s, &ends);
+}
+
 }  // namespace
 
 bool gla_variant_built(int dk, int dv) {
@@ -577,6 +639,14 @@ cudaError_t launch_gla_fwd(const GlaVariant& v, const GlaArgs& a, cudaStream_t s
   if (v.dk == 32 && v.dv == 64) return dispatch_types<32, 64>(v, a, s);
   if (v.dk == 36 && v.dv == 72) return dispatch_types<36, 72>(v, a, s);
   if (v.dk == 64 && v.dv == 64) return dispatch_types<64, 64>(v, a, s);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_gla_fwd_ext(const GlaVariant& v, const GlaArgs& a, const ScanEnds& ends, cudaStream_t s) {
+  if (v.tin != DIG_F32 || v.chunk != 64) return cudaErrorInvalidValue;
+  if (v.dk == 32 && v.dv == 64) return dispatch_ext<32, 64>(v, a, ends, s);
+  if (v.dk == 36 && v.dv == 72) return dispatch_ext<36, 72>(v, a, ends, s);
+  if (v.dk == 64 && v.dv == 64) return dispatch_ext<64, 64>(v, a, ends, s);
   return cudaErrorInvalidValue;
 }
 

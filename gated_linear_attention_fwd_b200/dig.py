@@ -58,6 +58,14 @@ lib.dig_gla_bwd.argtypes = [_vp, _vp, _vp, _vp, _i, _f, _vp, _vp, _vp, _vp, _vp,
 lib.dig_gla_bwd_saved.restype = _i
 lib.dig_gla_bwd_saved.argtypes = [_vp, _vp, _vp, _vp, _i, _f, _vp, _vp, _vp, _vp, _vp,
                                   _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp, _sz, _vp]
+lib.dig_gla_ext_workspace_bytes.restype = _sz
+lib.dig_gla_ext_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i]
+lib.dig_gla_fwd_ext.restype = _i
+lib.dig_gla_fwd_ext.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _f, _vp, _vp, _vp, _vp, _f, _vp, _vp,
+                                _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]
+lib.dig_gla_bwd_ext.restype = _i
+lib.dig_gla_bwd_ext.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _f, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]
 lib.dig_srem_reorient_dwconv.restype = _i
 lib.dig_srem_reorient_dwconv.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
 lib.dig_srem_reorient_dwconv_bwd.restype = _i
@@ -177,6 +185,42 @@ def dig_gla_bwd_saved(q, k, v, z, inv_tau, dO, dq, dk, dv, dlog_alpha, grid_h, g
                                _ptr(fwd_workspace), fwd_workspace.numel() * fwd_workspace.element_size(),
                                _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "dig_gla_bwd_saved")
+
+
+def new_ext_workspace(B, H, L, d_k, d_v, dtype=torch.bfloat16, backward=False, device="cuda",
+                      gate_heads=1) -> torch.Tensor:
+    """A zero-filled workspace (uint8) sized for dig_gla_fwd_ext / dig_gla_bwd_ext."""
+    n = int(lib.dig_gla_ext_workspace_bytes(B, H, gate_heads, L, d_k, d_v, _code(dtype), 1 if backward else 0))
+    if n == 0:
+        raise ValueError("unsupported shape for the extended GLA entry points")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def dig_gla_fwd_ext(q, k, v, z, inv_tau, o, grid_h, grid_w, scan_mode, workspace, zb=None, S0=None,
+                    S_final=None, r=None, gamma=None, eps=1e-5, y=None, stream=None):
+    """GLA with a value gate (zb [B,L,gate_heads,dv] fp32 logits) and state input /
+    output (S0, S_final [B,H,dk,dv] fp32); see include/dig.h."""
+    B, L, H, dk = q.shape
+    dv = v.shape[3]
+    st = lib.dig_gla_fwd_ext(_ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(zb), z.shape[2], float(inv_tau), _ptr(S0),
+                             _ptr(o), _ptr(r), _ptr(gamma), float(eps), _ptr(y), _ptr(S_final),
+                             B, H, L, dk, dv, grid_h, grid_w, scan_mode, _code(q.dtype), _code(o.dtype),
+                             _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "dig_gla_fwd_ext")
+
+
+def dig_gla_bwd_ext(q, k, v, z, inv_tau, dO, dq, dk, dv, dlog_alpha, grid_h, grid_w, scan_mode, workspace,
+                    zb=None, S0=None, o=None, dS_final=None, dlog_beta=None, dS0=None, stream=None):
+    """Gradients for dig_gla_fwd_ext (see include/dig.h); o is the forward's output,
+    needed for dlog_beta."""
+    B, L, H, d_k = q.shape
+    d_v = v.shape[3]
+    st = lib.dig_gla_bwd_ext(_ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(zb), z.shape[2], float(inv_tau), _ptr(S0),
+                             _ptr(o), _ptr(dO), _ptr(dS_final), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dlog_alpha),
+                             _ptr(dlog_beta), _ptr(dS0),
+                             B, H, L, d_k, d_v, grid_h, grid_w, scan_mode, _code(q.dtype), _code(dq.dtype),
+                             _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "dig_gla_bwd_ext")
 
 
 def dig_srem_reorient_dwconv(x, w, bias, y, scan_mode, stream=None):

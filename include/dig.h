@@ -139,6 +139,52 @@ dig_status dig_gla_fwd_noalloc(const void *q, const void *k, const void *v, cons
                                int scan_mode, int dtype, int out_dtype,
                                unsigned int *device_status, void *stream);
 
+/* GLA forward with a value gate and state input / output (slide "Gated Linear
+ * Attention Transformer (GLA) の導入", eq. (5): G_t = alpha_t^T beta_t (outer
+ * product), S_t = G_t (*) S_{t-1} + k_t^T v_t, o_t = q_t S_t, the recurrence
+ * started from S_0 instead of zero).  Arguments as dig_gla_fwd, plus:
+ *   zb       [B, L, gate_heads, d_v] fp32  value-gate logits, beta = exp(inv_tau *
+ *                                          logsigmoid(zb)); NULL: beta = 1
+ *   S0       [B, H, d_k, d_v] fp32         initial state (S0[b][h][c][j] = S_0[c][j]);
+ *                                          NULL: zero
+ *   S_final  [B, H, d_k, d_v] fp32         written: the state after the last scan
+ *                                          position (the S0 of a following segment);
+ *                                          may be NULL
+ * A sequence cut into segments and run segment by segment, each from the last
+ * one's S_final, gives the same o as one call over the whole sequence (in the
+ * scan order of each call).  d_v must be 64 or 72.  The call runs the fp32
+ * kernels (64-token chunks); bf16 inputs are widened into the workspace, whose
+ * size dig_gla_ext_workspace_bytes(..., dtype, 0) gives (zero-filled before the
+ * first use).  Errors as dig_gla_fwd. */
+dig_status dig_gla_fwd_ext(const void *q, const void *k, const void *v, const float *z, const float *zb,
+                           int gate_heads, float inv_tau, const float *S0, void *o,
+                           const void *r, const float *gamma, float eps, void *y, float *S_final,
+                           int B, int H, int L, int d_k, int d_v, int grid_h, int grid_w,
+                           int scan_mode, int dtype, int out_dtype,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/* Gradients for dig_gla_fwd_ext of sum(o * dO) + sum(S_final * dS_final).
+ *   o          [B, L, H, d_v] out_dtype  the forward's output (read only for
+ *                                        dlog_beta; may be NULL without it)
+ *   dS_final   [B, H, d_k, d_v] fp32     gradient of S_final; NULL: zero
+ *   dlog_beta  [B, L, gate_heads, d_v] fp32  dLoss/dlog(beta), summed over heads
+ *                                        when gate_heads == 1; NULL: not formed
+ *                                        (then zb may be NULL)
+ *   dS0        [B, H, d_k, d_v] fp32     written: gradient of S0; may be NULL
+ * Other arguments and results as dig_gla_bwd; the workspace size is
+ * dig_gla_ext_workspace_bytes(..., dtype, 1). */
+dig_status dig_gla_bwd_ext(const void *q, const void *k, const void *v, const float *z, const float *zb,
+                           int gate_heads, float inv_tau, const float *S0, const void *o, const void *dO,
+                           const float *dS_final, void *dq, void *dk, void *dv, float *dlog_alpha,
+                           float *dlog_beta, float *dS0,
+                           int B, int H, int L, int d_k, int d_v, int grid_h, int grid_w,
+                           int scan_mode, int dtype, int out_dtype,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/* Bytes of workspace dig_gla_fwd_ext (pass = 0) or dig_gla_bwd_ext (pass = 1)
+ * needs; 0 for invalid or unsupported shapes. */
+size_t dig_gla_ext_workspace_bytes(int B, int H, int gate_heads, int L, int d_k, int d_v, int dtype, int pass);
+
 /* GLA backward: gradients of sum(o * dO) for the forward above.
  *   dO          [B, L, H, d_v]  dtype
  *   dq, dk      [B, L, H, d_k]  out_dtype

@@ -114,6 +114,7 @@ EDGE = [
     (1, 1, 64, 64, 32, 64, "bf16", 1, 1 / 16, 0.0),     # one sequence of 32 chunks over the 16 scan ranges
     (1, 1, 128, 160, 32, 64, "bf16", 1, 1 / 16, 0.0),   # 160 chunks: two load windows per scan range
     (1, 1, 2, 2, 32, 64, "f32", 1, 1 / 16, 0.0),        # 4 tokens
+    (1, 2, 16, 24, 36, 72, "f32", 1, 1 / 16, 0.0),     # fp32 d_v = 72 > the 64-token chunk
 ]
 
 
