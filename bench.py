@@ -325,6 +325,39 @@ def time_gla_config(dig, index, dev, stream, flush, warmup, iters, seed_offset=0
     return t_f, t_b
 
 
+def time_dig_block(dev, flush, warmup, iters):
+    """Event-timed mean microseconds of one synthetic DiG-S/2 block forward at the
+    bench workload's shape (dense projections by cuBLAS, the rest by libdig.so) and
+    of the GLA mixer call inside it, averaged over the four layers' scan orders,
+    L2 flushed before every block."""
+    from gated_linear_attention_fwd_b200 import dig_block
+    w = inputs.WORKLOADS[WORKLOAD_INDEX]
+    B, L = w.B, w.L
+    blk_us, mix_us = [], []
+    for layer in range(4):
+        blk = dig_block.dig_s2(w.grid_h, w.grid_w, layer=layer, seed=layer, device=dev)
+        g = torch.Generator(device="cpu").manual_seed(100 + layer)
+        x0 = torch.randn(B, L, blk.D, generator=g).to(dev, torch.bfloat16)
+        cond = torch.randn(B, blk.D, generator=g).to(dev, torch.bfloat16)
+        buf = blk.buffers(B, L, dev)
+        x = x0.clone()
+        for i in range(warmup):
+            blk.forward(x, cond, buf)
+        timing, evs = {}, []
+        for i in range(iters):
+            x.copy_(x0)
+            flush.fill_(float(i))
+            e = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            e[0].record()
+            blk.forward(x, cond, buf, timing=timing)
+            e[1].record()
+            evs.append(e)
+        torch.cuda.synchronize()
+        blk_us.append(float(np.mean([a.elapsed_time(b) for a, b in evs])) * 1e3)
+        mix_us.append(float(np.mean([a.elapsed_time(b) for a, b in timing["mixer_events"]])) * 1e3)
+    return float(np.mean(blk_us)), float(np.mean(mix_us))
+
+
 def per_config_record(index, t_f, t_b, world, hbm, tflops):
     """tokens/s of fwd+bwd and the fraction of roofline of each, with the metric's bytes."""
     w = inputs.WORKLOADS[index]
@@ -501,6 +534,11 @@ def run_ours(args, rank, world, local_rank):
         if cfg_err is None:
             cfg_t = {i: (max_over_ranks(a, world, dev), max_over_ranks(b, world, dev)) for i, (a, b) in cfg_t.items()}
 
+    # the mixer in its block: a synthetic DiG-S/2 block forward at the same shape
+    blk_t, blk_err = run_guarded(lambda: time_dig_block(dev, flush, args.warmup, max(args.steps, 10)), world, dev)
+    if blk_err is None:
+        blk_t = tuple(max_over_ranks(tv, world, dev) for tv in blk_t)
+
     if rank != 0:
         return None
     hbm, tflops, peak_kind = _peaks()
@@ -550,6 +588,16 @@ def run_ours(args, rank, world, local_rank):
         line["per_config_note"] = ("fwd+bwd (dig_gla_fwd + dig_gla_bwd_saved, bf16 outputs) per metric shape; "
                                    "bytes count d log(alpha) once per head; fractions of the measured HBM copy "
                                    "bandwidth")
+    if blk_err is None:
+        b_us, m_us = blk_t
+        line["dig_block"] = {"block_us": b_us, "mixer_us": m_us, "mixer_share": m_us / b_us,
+                             "config": "DiG-S/2 block forward at %s (B=%d, L=%d, D=384), scan orders cycling"
+                                       % (w.name, B, L),
+                             "note": "adaLN + GLA layer (q/k/v/r/out projections by cuBLAS, gate projection, "
+                                     "dig_gla_fwd with the Swish*RMSNorm epilogue) + FFN + SREM conv; mixer = the "
+                                     "dig_gla_fwd call; random weights, synthetic tokens and conditioning"}
+    else:
+        line["dig_block"] = {"error": blk_err}
     if world == 1 and not args.no_cpu_baseline:
         tps, dt, cores, n = cpu_sample(w, x, steps=1, min_seconds=10.0)
         import oracle

@@ -77,6 +77,12 @@ lib.dig_gate_proj_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_longlon
 lib.dig_gate_proj_bwd.restype = _i
 lib.dig_gate_proj_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp, _vp, ctypes.c_longlong,
                                   _i, _i, _i, _i, _i, _vp]
+lib.dig_block_rmsnorm_modulate.restype = _i
+lib.dig_block_rmsnorm_modulate.argtypes = [_vp, _vp, _vp, ctypes.c_longlong, _f, _vp, _i, ctypes.c_longlong, _i, _vp]
+lib.dig_block_gated_add.restype = _i
+lib.dig_block_gated_add.argtypes = [_vp, _vp, ctypes.c_longlong, _vp, _i, ctypes.c_longlong, _i, _vp]
+lib.dig_block_activation.restype = _i
+lib.dig_block_activation.argtypes = [_vp, ctypes.c_longlong, _i, _vp]
 lib.dig_read_status.restype = _i
 lib.dig_read_status.argtypes = [_vp, _vp]
 lib.dig_status_string.restype = ctypes.c_char_p
@@ -267,6 +273,38 @@ def dig_gate_proj_bwd(x, W1, W2, u, z, dlog_alpha, inv_tau, dx, dW1, dW2, db=Non
                                _ptr(dx), _ptr(dW1), _ptr(dW2), _ptr(db), rows, D, R, d_k, _code(x.dtype),
                                _code(dx.dtype), _stream(stream))
     _check(st, "dig_gate_proj_bwd")
+
+
+def _mod_stride(t):
+    """Row stride (in values) of a [B, D] modulation slice."""
+    return t.stride(0)
+
+
+def dig_block_rmsnorm_modulate(x, shift, scale, y, eps=1e-6, stream=None):
+    """y = RMSNorm(x) * (1 + scale[b]) + shift[b]; x, y [B, rows, D] bf16; shift, scale
+    [B, D] fp32 (rows of one [B, 6 D] tensor may be passed as slices)."""
+    B, rows, D = x.shape
+    if shift.stride(1) != 1 or scale.stride(1) != 1 or shift.stride(0) != scale.stride(0):
+        raise ValueError("shift and scale must be row slices of one tensor")
+    st = lib.dig_block_rmsnorm_modulate(_ptr(x), ctypes.c_void_p(shift.data_ptr()), ctypes.c_void_p(scale.data_ptr()),
+                                        _mod_stride(shift), float(eps), _ptr(y), B, rows, D, _stream(stream))
+    _check(st, "dig_block_rmsnorm_modulate")
+
+
+def dig_block_gated_add(x, gate, y, stream=None):
+    """x += gate[b] * y; x, y [B, rows, D] bf16; gate [B, D] fp32 (a row slice)."""
+    B, rows, D = x.shape
+    if gate.stride(1) != 1:
+        raise ValueError("gate must have unit stride along D")
+    st = lib.dig_block_gated_add(_ptr(x), ctypes.c_void_p(gate.data_ptr()), _mod_stride(gate), _ptr(y), B, rows, D,
+                                 _stream(stream))
+    _check(st, "dig_block_gated_add")
+
+
+def dig_block_activation(x, kind, stream=None):
+    """In place on bf16 x: kind 0 SiLU, kind 1 GELU (tanh form)."""
+    st = lib.dig_block_activation(_ptr(x), x.numel(), int(kind), _stream(stream))
+    _check(st, "dig_block_activation")
 
 
 def dig_read_status(workspace, stream=None) -> int:

@@ -298,6 +298,26 @@ dig_status dig_gate_proj_bwd(const void *x, const float *W1, const float *W2, co
                              long long rows, int D, int R, int d_k, int dtype, int out_dtype,
                              void *stream);
 
+/* Element-wise steps of a DiG block around its token mixer (slide "DiG" Fig. 4,
+ * the DiG block: adaLN scale / shift / gate regressed from the conditioning,
+ * RMS normalisation, gated residuals, SiLU in the conditioning MLP, GELU in the
+ * feed-forward network).  The paper gives the block's structure, not these
+ * interfaces; they serve the library's synthetic block.  Tensors are bf16 rows
+ * of D values, B batches of rows_per_batch rows each; the modulation vectors are
+ * fp32, D values per batch at stride mod_stride (so that slices of one [B, 6 D]
+ * projection can be passed).  Pointers 16-byte aligned; D a multiple of 8.
+ *   rmsnorm_modulate:  y = x / sqrt(mean(x^2) + eps) * (1 + scale[b]) + shift[b]
+ *                      (D up to 2048)
+ *   gated_add:         x += gate[b] * y
+ *   activation:        x in place, n values: kind 0 SiLU a sigmoid(a), kind 1 GELU
+ *                      (tanh form) */
+dig_status dig_block_rmsnorm_modulate(const void *x, const float *shift, const float *scale,
+                                      long long mod_stride, float eps, void *y, int B,
+                                      long long rows_per_batch, int D, void *stream);
+dig_status dig_block_gated_add(void *x, const float *gate, long long mod_stride, const void *y, int B,
+                               long long rows_per_batch, int D, void *stream);
+dig_status dig_block_activation(void *x, long long n, int kind, void *stream);
+
 /* Synchronises `stream`, returns the device status word kept in `workspace`
  * (DIG_OK, DIG_ERR_DEVICE_TIMEOUT or DIG_ERR_GATE_RANGE) and clears it. */
 dig_status dig_read_status(void *workspace, void *stream);
