@@ -88,24 +88,30 @@ def metric_bytes(w):
 
 
 # This library's kernels per op, in launch order, and the sources they are built from.
-OP_KERNELS = {
-    "fwd": ["gla_gate_kernel", "gla_chunk_state_kernel", "gla_state_scan_kernel", "gla_chunk_out_kernel"],
-    "bwd": ["gla_chunk_dh_kernel", "gla_state_scan_kernel", "gla_chunk_grad_kernel"],
+OP_KERNELS = {  # this library's kernels per op on the bench workload (bf16, d_k = 32, d_v = 64)
+    # row scan orders: tile-copy dS and output kernels; column orders: the row-piece ones
+    "fwd": ["gla_gate_kernel", "gla_reduce_tma_kernel | gla_chunk_state_kernel", "gla_state_scan_kernel",
+            "gla_out_tma_kernel | gla_chunk_out_kernel"],
+    # the exact gradient kernel is launched on the list of units the fp16 kernel hands back (empty here)
+    "bwd": ["gla_reduce_tma_kernel | gla_chunk_dh_kernel", "gla_state_scan_kernel", "gla_grad_tma_kernel",
+            "gla_chunk_grad_kernel"],
     "conv": ["srem_dwconv_kernel"],
     "epi_bwd": ["epilogue_bwd_kernel"],
     "conv_bwd": ["srem_dwconv_bwd_kernel"],
-    "gate_fwd": ["gate_proj_fwd_kernel"],
+    "gate_fwd": ["gate_proj_tc_kernel"],
     "gate_bwd": ["gate_proj_bwd_kernel"],
 }
 STEP_OPS = ("fwd", "bwd", "conv")  # the ops of one timed step
 _CHUNK_SRC = ["gla_chunk.cuh", "gla_common.cuh", "sm100.cuh", "dig_common.cuh", "gla.h"]
+_TMA_SRC = ["tma.cuh", "tma_tiles.cuh", "tmap.cu", "tmap.h"]
 OP_SOURCES = {
-    "fwd": ["gla_fwd.cu"] + _CHUNK_SRC,
-    "bwd": ["gla_bwd.cu", "gla_fwd.cu"] + _CHUNK_SRC,
+    "fwd": ["gla_fwd.cu", "gla_state_tma.cu", "gla_fwd_tma.cu"] + _TMA_SRC + _CHUNK_SRC,
+    "bwd": ["gla_bwd.cu", "gla_bwd_tma.cu", "gla_state_tma.cu", "gla_fwd.cu"] + _TMA_SRC + _CHUNK_SRC,
     "conv": ["srem.cu", "srem.cuh", "dig_common.cuh", "gla.h"],
     "epi_bwd": ["epilogue_bwd.cu", "gla_common.cuh", "sm100.cuh", "dig_common.cuh", "bwd_ops.h"],
     "conv_bwd": ["srem_bwd.cu", "srem.cuh", "gla_common.cuh", "sm100.cuh", "dig_common.cuh", "bwd_ops.h"],
-    "gate_fwd": ["gate_proj.cu", "gate_proj.h", "gla_common.cuh", "sm100.cuh", "dig_common.cuh"],
+    "gate_fwd": ["gate_proj_tc.cu", "gate_proj.cu", "gate_proj.h", "tma.cuh", "tma_tiles.cuh", "tmap.cu",
+                 "gla_common.cuh", "sm100.cuh", "dig_common.cuh"],
     "gate_bwd": ["gate_proj.cu", "gate_proj.h", "gla_common.cuh", "sm100.cuh", "dig_common.cuh"],
 }
 OP_NAMES = {"fwd": "dig_gla_fwd", "bwd": "dig_gla_bwd_saved", "conv": "dig_srem_reorient_dwconv",

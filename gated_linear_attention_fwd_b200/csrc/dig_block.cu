@@ -69,11 +69,14 @@ __global__ void __launch_bounds__(256) rmsnorm_mod_kernel(const __nv_bfloat16* _
       const int piece = lane + 32 * p;
       if (piece < np) {
         float out[8];
+        const float4 s0 = __ldg(reinterpret_cast<const float4*>(sc + 8 * piece));
+        const float4 s1 = __ldg(reinterpret_cast<const float4*>(sc + 8 * piece) + 1);
+        const float4 h0 = __ldg(reinterpret_cast<const float4*>(sh + 8 * piece));
+        const float4 h1 = __ldg(reinterpret_cast<const float4*>(sh + 8 * piece) + 1);
+        const float scv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+        const float shv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int c = 8 * piece + e;
-          out[e] = fmaf(v[p][e] * inv, 1.f + __ldg(sc + c), __ldg(sh + c));
-        }
+        for (int e = 0; e < 8; ++e) out[e] = fmaf(v[p][e] * inv, 1.f + scv[e], shv[e]);
         st8(y + row * D + 8 * piece, out);
       }
     }
@@ -92,9 +95,11 @@ __global__ void __launch_bounds__(256) gated_add_kernel(__nv_bfloat16* __restric
     float xv[8], yv[8];
     ld8(x + 8 * i, xv);
     ld8(y + 8 * i, yv);
-    const float* g = gate + b * mod_stride + c0;
+    const float4 ga = __ldg(reinterpret_cast<const float4*>(gate + b * mod_stride + c0));
+    const float4 gb = __ldg(reinterpret_cast<const float4*>(gate + b * mod_stride + c0) + 1);
+    const float gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
 #pragma unroll
-    for (int e = 0; e < 8; ++e) xv[e] = fmaf(__ldg(g + e), yv[e], xv[e]);
+    for (int e = 0; e < 8; ++e) xv[e] = fmaf(gv[e], yv[e], xv[e]);
     st8(x + 8 * i, xv);
   }
 }
@@ -151,7 +156,8 @@ dig_status dig_block_rmsnorm_modulate(const void* x, const float* shift, const f
     return block_fail(DIG_ERR_INVALID_ARGUMENT, "rmsnorm_modulate: D must be a multiple of 8 up to 2048");
   if (B == 0 || rows_per_batch == 0) return DIG_OK;
   if (!x || !shift || !scale || !y) return block_fail(DIG_ERR_INVALID_ARGUMENT, "rmsnorm_modulate: NULL tensor");
-  if (!al16(x) || !al16(y)) return block_fail(DIG_ERR_MISALIGNED, "rmsnorm_modulate: misaligned tensor");
+  if (!al16(x) || !al16(y) || !al16(shift) || !al16(scale) || mod_stride % 4 != 0)
+    return block_fail(DIG_ERR_MISALIGNED, "rmsnorm_modulate: misaligned tensor or modulation row");
   const long long rows = (long long)B * rows_per_batch;
   return launched(launch_pdl(rmsnorm_mod_kernel, dim3(grid_for(rows * 32)), dim3(256), 0,
                              static_cast<cudaStream_t>(stream), static_cast<const __nv_bfloat16*>(x), shift, scale,
@@ -164,7 +170,8 @@ dig_status dig_block_gated_add(void* x, const float* gate, long long mod_stride,
     return block_fail(DIG_ERR_INVALID_ARGUMENT, "gated_add: D must be a positive multiple of 8");
   if (B == 0 || rows_per_batch == 0) return DIG_OK;
   if (!x || !gate || !y) return block_fail(DIG_ERR_INVALID_ARGUMENT, "gated_add: NULL tensor");
-  if (!al16(x) || !al16(y)) return block_fail(DIG_ERR_MISALIGNED, "gated_add: misaligned tensor");
+  if (!al16(x) || !al16(y) || !al16(gate) || mod_stride % 4 != 0)
+    return block_fail(DIG_ERR_MISALIGNED, "gated_add: misaligned tensor or gate row");
   const long long n8 = (long long)B * rows_per_batch * D / 8;
   return launched(launch_pdl(gated_add_kernel, dim3(grid_for(n8)), dim3(256), 0, static_cast<cudaStream_t>(stream),
                              static_cast<__nv_bfloat16*>(x), gate, mod_stride, static_cast<const __nv_bfloat16*>(y),

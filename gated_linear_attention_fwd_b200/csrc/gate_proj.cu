@@ -349,10 +349,20 @@ size_t gate_proj_smem_bytes(int D, int R, int dk, bool backward) {
   return backward ? gate_bwd_smem(D, RT, dk) : gate_fwd_smem(D, RT, dk);
 }
 
+bool gate_proj_tc_eligible(long long rows, int D, int R, int dk, int tin);  // gate_proj_tc.cu
+cudaError_t launch_gate_proj_tc(const void* x, const float* W1, const float* W2, const float* b, float* z, float* u,
+                                long long rows, int D, int R, int dk, uint32_t* status, cudaStream_t s,
+                                bool* launched);
+
 cudaError_t launch_gate_proj_fwd(const void* x, const float* W1, const float* W2, const float* b, float* z, float* u,
                                  long long rows, int D, int R, int dk, int tin, cudaStream_t s) {
   using bf = __nv_bfloat16;
   if (rows == 0) return cudaSuccess;
+  if (gate_proj_tc_eligible(rows, D, R, dk, tin)) {  // bf16 x: x W1 on the tensor cores
+    bool launched = false;
+    const cudaError_t e = launch_gate_proj_tc(x, W1, W2, b, z, u, rows, D, R, dk, nullptr, s, &launched);
+    if (e != cudaSuccess || launched) return e;
+  }
   if (R <= 16)
     return tin == DIG_BF16 ? fwd_typed<bf, 16>(x, W1, W2, b, z, u, rows, D, R, dk, s)
                            : fwd_typed<float, 16>(x, W1, W2, b, z, u, rows, D, R, dk, s);

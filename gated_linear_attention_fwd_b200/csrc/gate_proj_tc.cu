@@ -1,0 +1,242 @@
+// gate_proj_tc.cu -- the gate logits' low-rank projection on the tensor cores
+// (DiG slides, "Gated Linear Attention Transformer (GLA) の導入", eq. (5): the
+// key gate is sigmoid of a low-rank projection D -> R -> d_k of the block input):
+//
+//   u = x W1   [rows, R],   z = u W2 + b   [rows, d_k]
+//
+// About 2 D R multiply-adds per token against 2 D bytes of x: 16 per byte at
+// R = 16, beyond what the FP32 pipes deliver at HBM speed, so x W1 is a tcgen05
+// product: per tile of 128 token rows, A = the x tile (bf16, K-major, tiles of
+// 64 channels by TMA with the 128-byte swizzle), B = W1^T as two bf16 terms
+// (hi + lo, so the product keeps fp32-level accuracy), M = 128, N = 16, into one
+// of two TMEM accumulators.  One thread streams the x blocks through a ring of
+// eight stages and issues the products; four warps read u back (lane = row),
+// form z = u W2 + b from W2 in shared memory and store u and z.  bf16 x, R <= 16,
+// D a multiple of 64 (up to 1152) and d_k <= 64 take this kernel.
+#include "tma.cuh"
+#include "tma_tiles.cuh"
+#include "tmap.h"
+
+namespace dig {
+
+namespace {
+
+constexpr int kBM = 128, kKB = 64, kNS = 8;  // rows per tile, channels per x block, ring stages
+constexpr uint32_t kXB = kBM * kKB * 2;       // bytes of one x block (16 KB)
+constexpr int kMaxD = 1152;
+
+struct GpSmem {
+  uint64_t full[kNS], empty[kNS], acc_full[2], acc_empty[2];
+  uint32_t tmem;
+  int abort;
+};
+
+// Dynamic shared memory: the x ring, W1^T terms (D / 64 blocks of 16 rows x 128
+// bytes per term), W2 [16][d_k] and b [d_k] (fp32).
+struct GpLayout {
+  uint32_t ring, w1, w2, bias, total;
+  __host__ __device__ GpLayout(int D, int dk) {
+    ring = 0;
+    w1 = kNS * kXB;
+    w2 = w1 + 2u * (uint32_t)(D / kKB) * 2048u;
+    bias = w2 + 16u * dk * 4u;
+    total = bias + (uint32_t)dk * 4u;
+  }
+};
+
+template <int DK>
+__global__ void __launch_bounds__(256, 1) gate_proj_tc_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                              const float* __restrict__ W1,
+                                                              const float* __restrict__ W2,
+                                                              const float* __restrict__ b, float* __restrict__ z,
+                                                              float* __restrict__ u, long long rows, int D, int R,
+                                                              uint32_t* status) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ GpSmem sh;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const uint32_t sb = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sb - smem_u32(smem_raw));
+  const GpLayout lay(D, DK);
+  const int nkb = D / kKB;
+  const long long ntiles = (rows + kBM - 1) / kBM;
+  const int mytiles = blockIdx.x < ntiles ? (int)((ntiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
+  const int total = mytiles * nkb;  // x blocks this CTA consumes
+  if (warp == 0) {
+    tmem_alloc(&sh.tmem, 32);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int i = 0; i < kNS; ++i) {
+      mbar_init(&sh.full[i], 1);
+      mbar_init(&sh.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sh.acc_full[i], 1);
+      mbar_init(&sh.acc_empty[i], 128);
+    }
+    sh.abort = 0;
+    fence_mbar_init();
+  }
+  griddep_wait();  // the kernels before this one have completed
+  griddep_launch_dependents();
+  // ---- W1^T as two bf16 terms (row n = output r, K-major, 128-byte swizzle), W2 and b
+  // element (k, n) for i = 16 k + n: consecutive threads read consecutive W1 values
+  // (when R = 16); eight loads in flight per thread before their stores
+  for (int i0 = tid; i0 < 16 * D; i0 += 8 * 256) {
+    float wv[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int i = i0 + e * 256, k = i >> 4, n = i & 15;
+      wv[e] = (i < 16 * D && n < R) ? __ldg(W1 + (size_t)k * R + n) : 0.f;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int i = i0 + e * 256, k = i >> 4, n = i & 15;
+      if (i < 16 * D) {
+        const __nv_bfloat16 hi = __float2bfloat16_rn(wv[e]);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(wv[e] - __bfloat162float(hi));
+        const uint32_t off = (uint32_t)(k / kKB) * 2048u + swz_off<128>(n, (k % kKB) / 8) + (k % 8) * 2;
+        *reinterpret_cast<__nv_bfloat16*>(sgen + lay.w1 + off) = hi;
+        *reinterpret_cast<__nv_bfloat16*>(sgen + lay.w1 + (uint32_t)nkb * 2048u + off) = lo;
+      }
+    }
+  }
+  float* sW2 = reinterpret_cast<float*>(sgen + lay.w2);
+  float* sB = reinterpret_cast<float*>(sgen + lay.bias);
+  for (int i = tid; i < 16 * DK; i += 256) sW2[i] = (i / DK) < R ? __ldg(W2 + (size_t)(i / DK) * DK + i % DK) : 0.f;
+  for (int i = tid; i < DK; i += 256) sB[i] = b ? __ldg(b + i) : 0.f;
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem;
+  const uint64_t spin = kSpinLimitNs;
+
+  if (warp == 0) {
+    // ---------------- one thread: x blocks through the ring, products into the accumulators
+    if (tid == 0) {
+      auto tile_row = [&](int g) { return (int)((blockIdx.x + (long long)(g / nkb) * gridDim.x) * kBM); };
+      auto load = [&](int g) {
+        const int s = g % kNS;
+        mbar_arrive_expect_tx(&sh.full[s], kXB);
+        tma_load_2d(sb + lay.ring + s * kXB, xmap, (g % nkb) * kKB, tile_row(g), &sh.full[s]);
+      };
+      int issued = 0, committed = -1;  // blocks requested; last block whose products were committed
+      bool stop = false;
+      for (; issued < total && issued < kNS; ++issued) load(issued);
+      for (int g = 0; g < total && !stop; ++g) {
+        const int s = g % kNS, i = g / nkb, kb = g % nkb, ac = i & 1;
+        if (!mbar_wait(&sh.full[s], (g / kNS) & 1, spin)) { stop = true; break; }
+        if (kb == 0 && i >= 2 && !mbar_wait(&sh.acc_empty[ac], ((i >> 1) - 1) & 1, spin)) { stop = true; break; }
+        tc_fence_after();
+        const uint32_t xs = sb + lay.ring + s * kXB;
+#pragma unroll
+        for (int ks = 0; ks < kKB / 16; ++ks)
+#pragma unroll
+          for (int tt = 0; tt < 2; ++tt)
+            mma_bf16(tmem + 16u * ac, sdesc_sw<128>(xs + 32 * ks),
+                     sdesc_sw<128>(sb + lay.w1 + (uint32_t)(tt * nkb + kb) * 2048u + 32 * ks),
+                     idesc_bf16(kBM, 16), (kb | ks | tt) ? 1u : 0u);
+        mma_commit(&sh.empty[s]);
+        if (kb == nkb - 1) mma_commit(&sh.acc_full[ac]);
+        committed = g;
+        // the block before this one has been read: its stage takes the block kNS - 1 ahead
+        if (g >= 1 && issued < total) {
+          const int gp = g - 1;
+          if (!mbar_wait(&sh.empty[gp % kNS], (gp / kNS) & 1, spin)) { stop = true; break; }
+          load(issued++);
+        }
+      }
+      if (stop) sh.abort = 1;
+      // drain: every requested block has landed and the last products completed
+      for (int g = (committed < 0 ? 0 : committed + 1); g < issued; ++g)
+        mbar_wait(&sh.full[g % kNS], (g / kNS) & 1, kSpinLimitNs);
+      if (committed >= 0) mbar_wait(&sh.empty[committed % kNS], (committed / kNS) & 1, kSpinLimitNs);
+      if (stop && status != nullptr) set_status(status, DIG_ERR_DEVICE_TIMEOUT);
+    }
+  } else if (warp >= 4) {
+    // ---------------- four warps: u from TMEM (lane = tile row), z = u W2 + b, stores
+    const int lr = tid - 128;  // TMEM lane = row within the tile
+    const uint32_t lane_base = static_cast<uint32_t>(32 * (warp - 4)) << 16;
+    for (int i = 0; i < mytiles; ++i) {
+      const int ac = i & 1;
+      const bool ok = mbar_wait(&sh.acc_full[ac], (i >> 1) & 1, spin);
+      if (!ok || sh.abort) {
+        sh.abort = 1;
+        if (status != nullptr) set_status(status, DIG_ERR_DEVICE_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      float uv[16];
+      tmem_ld16(tmem + lane_base + 16u * ac, uv);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&sh.acc_empty[ac]);
+      const long long row = (blockIdx.x + (long long)i * gridDim.x) * kBM + lr;
+      if (row < rows) {
+        if (u != nullptr) {
+#pragma unroll
+          for (int r = 0; r < 16; ++r)
+            if (r < R) u[row * R + r] = uv[r];
+        }
+        float* zr = z + row * DK;
+#pragma unroll
+        for (int c0 = 0; c0 < DK; c0 += 4) {
+          float acc[4] = {sB[c0], sB[c0 + 1], sB[c0 + 2], sB[c0 + 3]};
+#pragma unroll
+          for (int r = 0; r < 16; ++r) {
+            const float4 w4 = *reinterpret_cast<const float4*>(sW2 + r * DK + c0);
+            acc[0] = fmaf(uv[r], w4.x, acc[0]);
+            acc[1] = fmaf(uv[r], w4.y, acc[1]);
+            acc[2] = fmaf(uv[r], w4.z, acc[2]);
+            acc[3] = fmaf(uv[r], w4.w, acc[3]);
+          }
+          *reinterpret_cast<float4*>(zr + c0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 32);
+}
+
+template <int DK>
+cudaError_t launch_dk(const CUtensorMap& m, const float* W1, const float* W2, const float* b, float* z, float* u,
+                      long long rows, int D, int R, uint32_t* status, cudaStream_t s) {
+  auto k = gate_proj_tc_kernel<DK>;
+  const uint32_t smem = GpLayout(D, DK).total + 1024;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const long long ntiles = (rows + kBM - 1) / kBM;
+  const int grid = (int)(ntiles < num_sms() ? ntiles : num_sms());
+  return launch_pdl(k, dim3(grid), dim3(256), smem, s, m, W1, W2, b, z, u, rows, D, R, status);
+}
+
+}  // namespace
+
+bool gate_proj_tc_eligible(long long rows, int D, int R, int dk, int tin) {
+  return tin == DIG_BF16 && rows > 0 && rows <= 0x7FFFFFFFLL && R >= 1 && R <= 16 && D % kKB == 0 && D <= kMaxD &&
+         (dk == 32 || dk == 36 || dk == 64) && tmap_available();
+}
+
+// `launched` stays false when the tensor map cannot be encoded (the caller runs
+// the CUDA-core kernel).  `status`: a device word that receives
+// DIG_ERR_DEVICE_TIMEOUT if a wait gives up, or NULL.
+cudaError_t launch_gate_proj_tc(const void* x, const float* W1, const float* W2, const float* b, float* z, float* u,
+                                long long rows, int D, int R, int dk, uint32_t* status, cudaStream_t s,
+                                bool* launched) {
+  *launched = false;
+  CUtensorMap m;
+  memset(&m, 0, sizeof(m));
+  if (!tmap_rows(&m, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, (uint64_t)rows, kKB, kBM, 128)) return cudaSuccess;
+  cudaError_t e;
+  if (dk == 32) e = launch_dk<32>(m, W1, W2, b, z, u, rows, D, R, status, s);
+  else if (dk == 36) e = launch_dk<36>(m, W1, W2, b, z, u, rows, D, R, status, s);
+  else e = launch_dk<64>(m, W1, W2, b, z, u, rows, D, R, status, s);
+  if (e == cudaSuccess) *launched = true;
+  return e;
+}
+
+}  // namespace dig

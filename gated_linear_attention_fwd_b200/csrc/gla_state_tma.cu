@@ -12,9 +12,9 @@
 // one); what differs is the data path: k (or q), v (or dO) and the gate factors
 // arrive as whole tiles by TMA into one of two stages, so the next unit's tiles
 // land while this unit is converted and multiplied, and the block leaves by a
-// TMA tile store.  Only bf16 inputs with d_k = 32, d_v = 64 and 128-token chunks
-// that tile the sequence (and, for the column orders, 16-row column segments)
-// take this kernel.
+// TMA tile store.  Only bf16 inputs with d_k = 32, d_v = 64, 128-token chunks
+// that tile the sequence and the row scan orders take this kernel (the kernel
+// itself also reads the column orders' tiles as 16-row segments).
 #include "tma_tiles.cuh"
 
 namespace dig {
@@ -34,7 +34,7 @@ struct TmaReduceCfg {
   static constexpr int OFF_OUT = 2 * STAGE;         // [d_v][d_k] fp32, 128-byte swizzle
   static constexpr int END = OFF_OUT + DV * DK * 4;  // 106496
   static constexpr int SMEM = END + 1024;
-  static constexpr int TM_COLS = 64;                 // one 32-column accumulator per stage
+  static constexpr int TM_COLS = 128;                // per stage: the hi and lo terms' products, 32 columns each
   static constexpr uint32_t IN_BYTES = C * RBX + C * RBY + C * DK * 4, GCH_BYTES = 2 * DK * 4;
 };
 
@@ -156,17 +156,20 @@ __global__ void __launch_bounds__(256, 2) gla_reduce_tma_kernel(const __grid_con
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    // ---- D[j][c] = sum_t Y[t][j] X[t][c]: A = the y tile read MN-major (M = value
-    //      channels, 64 of 128 rows used), B = the x terms read MN-major, K = tokens
+    // ---- D[j][c'] = sum_t Y[t][j] X'[t][c']: A = the y tile read MN-major (M = value
+    //      channels, 64 of 128 rows used), B = the hi and lo terms side by side (N = 2 d_k:
+    //      two 32-channel MN atoms 8 KB apart), K = tokens; the two halves are added on
+    //      the way out.  One N = 64 product per K-step instead of two N = 32 ones: the
+    //      tensor core takes about as long per instruction at either width.
     if (tid == 0 && !timed_out && !sh.abort) {
-      const uint32_t dtm = tmem + 32u * s;
+      const uint32_t dtm = tmem + 64u * s;
+      uint64_t bdesc = sdesc_sw<64>(st + TC::S_XH);
+      bdesc &= ~(static_cast<uint64_t>(0x3FFF) << 16);  // leading byte offset: the lo term's atom
+      bdesc |= static_cast<uint64_t>(((TC::S_XL - TC::S_XH) >> 4) & 0x3FFF) << 16;
 #pragma unroll
       for (int ks = 0; ks < C / 16; ++ks)
-#pragma unroll
-        for (int tt = 0; tt < 2; ++tt)
-          mma_bf16(dtm, sdesc_sw<128>(st + TC::S_Y + 2048 * ks),
-                   sdesc_sw<64>(st + (tt ? TC::S_XL : TC::S_XH) + 1024 * ks), idesc_bf16(128, DK, true, true),
-                   (ks | tt) ? 1u : 0u);
+        mma_bf16(dtm, sdesc_sw<128>(st + TC::S_Y + 2048 * ks), bdesc + (uint64_t)((1024 * ks) >> 4),
+                 idesc_bf16(128, 2 * DK, true, true), ks ? 1u : 0u);
       mma_commit(&sh.mma[s]);
       mark(2 + s, ph);
     }
@@ -179,9 +182,12 @@ __global__ void __launch_bounds__(256, 2) gla_reduce_tma_kernel(const __grid_con
     if (tid == 0 && stored) bulk_wait_read_all();  // the previous block has left the staging
     __syncthreads();
     if (warp < 2) {  // lanes 0 .. 63
-      float d[32];
-      tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 32u * s, d);
+      float d[32], dl[32];
+      tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 64u * s, d);
+      tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 64u * s + 32u, dl);
       tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) d[i] += dl[i];
       const int j = tid;
 #pragma unroll
       for (int m = 0; m < 8; ++m)
@@ -216,9 +222,13 @@ __global__ void __launch_bounds__(256, 2) gla_reduce_tma_kernel(const __grid_con
 }
 
 // ------------------------------------------------------------------ launch
+// The row scan orders only: in the column orders the tile arrives as eight 16-row
+// segment copies per tensor, and the row-piece kernels were faster there (same box,
+// DiG-S/2 1792^2: forward 82 vs 85 us, backward 111.6 vs 112.6 us), while this kernel
+// wins in the row orders (forward 73.5 vs 76.7 us, backward 98.3 vs 100.3 us).
 bool gla_reduce_tma_eligible(const GlaArgs& a, int dk, int dv, int tin, int chunk) {
   if (tin != DIG_BF16 || dk != 32 || dv != 64 || chunk != 128 || a.L % 128 != 0) return false;
-  if ((a.mode & 2) && a.Hg % 16 != 0) return false;
+  if (a.mode & 2) return false;
   return tmap_available();
 }
 

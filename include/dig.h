@@ -305,7 +305,8 @@ dig_status dig_gate_proj_bwd(const void *x, const float *W1, const float *W2, co
  * interfaces; they serve the library's synthetic block.  Tensors are bf16 rows
  * of D values, B batches of rows_per_batch rows each; the modulation vectors are
  * fp32, D values per batch at stride mod_stride (so that slices of one [B, 6 D]
- * projection can be passed).  Pointers 16-byte aligned; D a multiple of 8.
+ * projection can be passed; mod_stride a multiple of 4).  Pointers, including the
+ * modulation slices, 16-byte aligned; D a multiple of 8.
  *   rmsnorm_modulate:  y = x / sqrt(mean(x^2) + eps) * (1 + scale[b]) + shift[b]
  *                      (D up to 2048)
  *   gated_add:         x += gate[b] * y
