@@ -26,23 +26,40 @@ constexpr uint32_t kXB = kBM * kKB * 2;       // bytes of one x block (16 KB)
 constexpr int kMaxD = 1152;
 
 struct GpSmem {
-  uint64_t full[kNS], empty[kNS], acc_full[2], acc_empty[2];
+  uint64_t full[kNS], empty[kNS], acc_full[2], acc_empty[2], wbar;
   uint32_t tmem;
   int abort;
 };
 
-// Dynamic shared memory: the x ring, W1^T terms (D / 64 blocks of 16 rows x 128
-// bytes per term), W2 [16][d_k] and b [d_k] (fp32).
+// Stages of the x ring: eight, six when D > 768 (the W1 terms then need the room).
+__host__ __device__ inline int ring_stages(int D) { return D > 768 ? 6 : kNS; }
+
+// Dynamic shared memory: the x ring (which first receives W1 and W2 as fp32 by bulk
+// copy), W1^T terms (D / 64 blocks of 16 rows x 128 bytes per term), W2 [16][d_k]
+// and b [d_k] (fp32), and the output staging (z [128][d_k], u [128][R] fp32).
 struct GpLayout {
-  uint32_t ring, w1, w2, bias, total;
+  uint32_t ring, w1, w2, bias, zst, ust, total;
   __host__ __device__ GpLayout(int D, int dk) {
     ring = 0;
-    w1 = kNS * kXB;
+    w1 = (uint32_t)ring_stages(D) * kXB;
     w2 = w1 + 2u * (uint32_t)(D / kKB) * 2048u;
     bias = w2 + 16u * dk * 4u;
-    total = bias + (uint32_t)dk * 4u;
+    zst = (bias + (uint32_t)dk * 4u + 15u) & ~15u;
+    ust = zst + (uint32_t)kBM * dk * 4u;
+    total = ust + (uint32_t)kBM * 16u * 4u;
   }
 };
+
+// OR of a predicate over the 128 threads of the four epilogue warps (named barrier 1).
+__device__ __forceinline__ bool epi_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
 
 template <int DK>
 __global__ void __launch_bounds__(256, 1) gate_proj_tc_kernel(const __grid_constant__ CUtensorMap xmap,
@@ -74,37 +91,59 @@ __global__ void __launch_bounds__(256, 1) gate_proj_tc_kernel(const __grid_const
       mbar_init(&sh.acc_full[i], 1);
       mbar_init(&sh.acc_empty[i], 128);
     }
+    mbar_init(&sh.wbar, 1);
     sh.abort = 0;
     fence_mbar_init();
   }
+  // every thread waits on these barriers (the weights' one first): they must be
+  // initialised before any thread reaches a wait
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
   griddep_wait();  // the kernels before this one have completed
   griddep_launch_dependents();
-  // ---- W1^T as two bf16 terms (row n = output r, K-major, 128-byte swizzle), W2 and b
-  // element (k, n) for i = 16 k + n: consecutive threads read consecutive W1 values
-  // (when R = 16); eight loads in flight per thread before their stores
-  for (int i0 = tid; i0 < 16 * D; i0 += 8 * 256) {
-    float wv[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int i = i0 + e * 256, k = i >> 4, n = i & 15;
-      wv[e] = (i < 16 * D && n < R) ? __ldg(W1 + (size_t)k * R + n) : 0.f;
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int i = i0 + e * 256, k = i >> 4, n = i & 15;
-      if (i < 16 * D) {
-        const __nv_bfloat16 hi = __float2bfloat16_rn(wv[e]);
-        const __nv_bfloat16 lo = __float2bfloat16_rn(wv[e] - __bfloat162float(hi));
-        const uint32_t off = (uint32_t)(k / kKB) * 2048u + swz_off<128>(n, (k % kKB) / 8) + (k % 8) * 2;
-        *reinterpret_cast<__nv_bfloat16*>(sgen + lay.w1 + off) = hi;
-        *reinterpret_cast<__nv_bfloat16*>(sgen + lay.w1 + (uint32_t)nkb * 2048u + off) = lo;
-      }
-    }
+  const int ns = ring_stages(D);
+  // ---- W1 and W2 (fp32) into the still empty ring by two bulk copies, then W1^T as two
+  // bf16 terms (row n = output r, K-major, 128-byte swizzle), W2 and b into their places
+  const uint32_t w1_bytes = (uint32_t)D * R * 4u, w2_off = (w1_bytes + 15u) & ~15u;
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&sh.wbar, w1_bytes + (uint32_t)R * DK * 4u);
+    bulk_copy_g2s(sb + lay.ring, W1, w1_bytes, &sh.wbar);
+    bulk_copy_g2s(sb + lay.ring + w2_off, W2, (uint32_t)R * DK * 4u, &sh.wbar);
   }
   float* sW2 = reinterpret_cast<float*>(sgen + lay.w2);
   float* sB = reinterpret_cast<float*>(sgen + lay.bias);
-  for (int i = tid; i < 16 * DK; i += 256) sW2[i] = (i / DK) < R ? __ldg(W2 + (size_t)(i / DK) * DK + i % DK) : 0.f;
-  for (int i = tid; i < DK; i += 256) sB[i] = b ? __ldg(b + i) : 0.f;
+  const float bv = (tid < DK && b != nullptr) ? __ldg(b + tid) : 0.f;
+  const bool w_ok = mbar_wait(&sh.wbar, 0, kSpinLimitNs);
+  const float* rawW1 = reinterpret_cast<const float*>(sgen + lay.ring);
+  const float* rawW2 = reinterpret_cast<const float*>(sgen + lay.ring + w2_off);
+  for (int i = tid; i < 16 * D; i += 256) {  // element (k, n), i = 16 k + n
+    const int k = i >> 4, n = i & 15;
+    const float w = (n < R && w_ok) ? rawW1[k * R + n] : 0.f;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(w - __bfloat162float(hi));
+    const uint32_t off = (uint32_t)(k / kKB) * 2048u + swz_off<128>(n, (k % kKB) / 8) + (k % 8) * 2;
+    *reinterpret_cast<__nv_bfloat16*>(sgen + lay.w1 + off) = hi;
+    *reinterpret_cast<__nv_bfloat16*>(sgen + lay.w1 + (uint32_t)nkb * 2048u + off) = lo;
+  }
+  for (int i = tid; i < 16 * DK; i += 256) sW2[i] = (i / DK < R && w_ok) ? rawW2[i] : 0.f;
+  if (tid < DK) sB[tid] = bv;
+  if (!w_ok) {
+    sh.abort = 1;
+    if (status != nullptr) set_status(status, DIG_ERR_DEVICE_TIMEOUT);
+  }
+  // every thread's reads of the raw weights precede the x copies into the ring
+  fence_async_smem();
+  __syncthreads();
+  auto tile_row = [&](int g) { return (int)((blockIdx.x + (long long)(g / nkb) * gridDim.x) * kBM); };
+  auto load = [&](int g) {
+    const int s = g % ns;
+    mbar_arrive_expect_tx(&sh.full[s], kXB);
+    tma_load_2d(sb + lay.ring + s * kXB, xmap, (g % nkb) * kKB, tile_row(g), &sh.full[s]);
+  };
+  int issued = 0;  // thread 0: blocks requested
+  if (tid == 0 && !sh.abort)
+    for (; issued < total && issued < ns; ++issued) load(issued);
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -115,18 +154,11 @@ __global__ void __launch_bounds__(256, 1) gate_proj_tc_kernel(const __grid_const
   if (warp == 0) {
     // ---------------- one thread: x blocks through the ring, products into the accumulators
     if (tid == 0) {
-      auto tile_row = [&](int g) { return (int)((blockIdx.x + (long long)(g / nkb) * gridDim.x) * kBM); };
-      auto load = [&](int g) {
-        const int s = g % kNS;
-        mbar_arrive_expect_tx(&sh.full[s], kXB);
-        tma_load_2d(sb + lay.ring + s * kXB, xmap, (g % nkb) * kKB, tile_row(g), &sh.full[s]);
-      };
-      int issued = 0, committed = -1;  // blocks requested; last block whose products were committed
+      int committed = -1;  // the last block whose products were committed
       bool stop = false;
-      for (; issued < total && issued < kNS; ++issued) load(issued);
-      for (int g = 0; g < total && !stop; ++g) {
-        const int s = g % kNS, i = g / nkb, kb = g % nkb, ac = i & 1;
-        if (!mbar_wait(&sh.full[s], (g / kNS) & 1, spin)) { stop = true; break; }
+      for (int g = 0; g < total && !stop && !sh.abort; ++g) {
+        const int s = g % ns, i = g / nkb, kb = g % nkb, ac = i & 1;
+        if (!mbar_wait(&sh.full[s], (g / ns) & 1, spin)) { stop = true; break; }
         if (kb == 0 && i >= 2 && !mbar_wait(&sh.acc_empty[ac], ((i >> 1) - 1) & 1, spin)) { stop = true; break; }
         tc_fence_after();
         const uint32_t xs = sb + lay.ring + s * kXB;
@@ -140,18 +172,18 @@ __global__ void __launch_bounds__(256, 1) gate_proj_tc_kernel(const __grid_const
         mma_commit(&sh.empty[s]);
         if (kb == nkb - 1) mma_commit(&sh.acc_full[ac]);
         committed = g;
-        // the block before this one has been read: its stage takes the block kNS - 1 ahead
+        // the block before this one has been read: its stage takes the block ns - 1 ahead
         if (g >= 1 && issued < total) {
           const int gp = g - 1;
-          if (!mbar_wait(&sh.empty[gp % kNS], (gp / kNS) & 1, spin)) { stop = true; break; }
+          if (!mbar_wait(&sh.empty[gp % ns], (gp / ns) & 1, spin)) { stop = true; break; }
           load(issued++);
         }
       }
       if (stop) sh.abort = 1;
       // drain: every requested block has landed and the last products completed
       for (int g = (committed < 0 ? 0 : committed + 1); g < issued; ++g)
-        mbar_wait(&sh.full[g % kNS], (g / kNS) & 1, kSpinLimitNs);
-      if (committed >= 0) mbar_wait(&sh.empty[committed % kNS], (committed / kNS) & 1, kSpinLimitNs);
+        mbar_wait(&sh.full[g % ns], (g / ns) & 1, kSpinLimitNs);
+      if (committed >= 0) mbar_wait(&sh.empty[committed % ns], (committed / ns) & 1, kSpinLimitNs);
       if (stop && status != nullptr) set_status(status, DIG_ERR_DEVICE_TIMEOUT);
     }
   } else if (warp >= 4) {
@@ -161,7 +193,7 @@ __global__ void __launch_bounds__(256, 1) gate_proj_tc_kernel(const __grid_const
     for (int i = 0; i < mytiles; ++i) {
       const int ac = i & 1;
       const bool ok = mbar_wait(&sh.acc_full[ac], (i >> 1) & 1, spin);
-      if (!ok || sh.abort) {
+      if (epi_any(!ok || sh.abort)) {  // uniform over the four warps (they share barrier 1)
         sh.abort = 1;
         if (status != nullptr) set_status(status, DIG_ERR_DEVICE_TIMEOUT);
         break;
@@ -172,30 +204,40 @@ __global__ void __launch_bounds__(256, 1) gate_proj_tc_kernel(const __grid_const
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&sh.acc_empty[ac]);
-      const long long row = (blockIdx.x + (long long)i * gridDim.x) * kBM + lr;
-      if (row < rows) {
-        if (u != nullptr) {
+      // z = u W2 + b of this row, then the tile's u and z rows (contiguous in global
+      // memory) leave through shared memory as coalesced 16-byte stores
+      float* zs = reinterpret_cast<float*>(sgen + lay.zst);
+      float* us = reinterpret_cast<float*>(sgen + lay.ust);
+      named_bar(1, 128);  // the previous tile's staged rows have been stored
 #pragma unroll
-          for (int r = 0; r < 16; ++r)
-            if (r < R) u[row * R + r] = uv[r];
+      for (int r = 0; r < 16; ++r)
+        if (r < R) us[lr * R + r] = uv[r];
+#pragma unroll
+      for (int c0 = 0; c0 < DK; c0 += 4) {
+        float acc[4] = {sB[c0], sB[c0 + 1], sB[c0 + 2], sB[c0 + 3]};
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          const float4 w4 = *reinterpret_cast<const float4*>(sW2 + r * DK + c0);
+          acc[0] = fmaf(uv[r], w4.x, acc[0]);
+          acc[1] = fmaf(uv[r], w4.y, acc[1]);
+          acc[2] = fmaf(uv[r], w4.z, acc[2]);
+          acc[3] = fmaf(uv[r], w4.w, acc[3]);
         }
-        float* zr = z + row * DK;
-#pragma unroll
-        for (int c0 = 0; c0 < DK; c0 += 4) {
-          float acc[4] = {sB[c0], sB[c0 + 1], sB[c0 + 2], sB[c0 + 3]};
-#pragma unroll
-          for (int r = 0; r < 16; ++r) {
-            const float4 w4 = *reinterpret_cast<const float4*>(sW2 + r * DK + c0);
-            acc[0] = fmaf(uv[r], w4.x, acc[0]);
-            acc[1] = fmaf(uv[r], w4.y, acc[1]);
-            acc[2] = fmaf(uv[r], w4.z, acc[2]);
-            acc[3] = fmaf(uv[r], w4.w, acc[3]);
-          }
-          *reinterpret_cast<float4*>(zr + c0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        }
+        *reinterpret_cast<float4*>(zs + lr * DK + c0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      }
+      named_bar(1, 128);
+      const long long row0 = (blockIdx.x + (long long)i * gridDim.x) * kBM;
+      const int nrow = (int)(rows - row0 < kBM ? rows - row0 : kBM);
+      const int zq = nrow * DK / 4, uq = nrow * R;  // float4s of z; floats of u
+      float4* zg = reinterpret_cast<float4*>(z + row0 * DK);
+      for (int q = lr; q < zq; q += 128) zg[q] = reinterpret_cast<const float4*>(zs)[q];
+      if (u != nullptr) {
+        float* ug = u + row0 * R;
+        for (int q = lr; q < uq; q += 128) ug[q] = us[q];
       }
     }
   }
+  if (tid == 0 && !w_ok) mbar_wait(&sh.wbar, 0, kSpinLimitNs);  // the weights' copies have landed
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
