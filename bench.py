@@ -105,8 +105,9 @@ STEP_OPS = ("fwd", "bwd", "conv")  # the ops of one timed step
 _CHUNK_SRC = ["gla_chunk.cuh", "gla_common.cuh", "sm100.cuh", "dig_common.cuh", "gla.h"]
 _TMA_SRC = ["tma.cuh", "tma_tiles.cuh", "tmap.cu", "tmap.h"]
 OP_SOURCES = {
-    "fwd": ["gla_fwd.cu", "gla_state_tma.cu", "gla_fwd_tma.cu"] + _TMA_SRC + _CHUNK_SRC,
-    "bwd": ["gla_bwd.cu", "gla_bwd_tma.cu", "gla_state_tma.cu", "gla_fwd.cu"] + _TMA_SRC + _CHUNK_SRC,
+    "fwd": ["gla_fwd.cu", "gla_state_tma.cu", "gla_fwd_tma.cu", "gla_strong.cuh"] + _TMA_SRC + _CHUNK_SRC,
+    "bwd": ["gla_bwd.cu", "gla_bwd_tma.cu", "gla_state_tma.cu", "gla_fwd.cu", "gla_strong.cuh"] + _TMA_SRC +
+           _CHUNK_SRC,
     "conv": ["srem.cu", "srem.cuh", "dig_common.cuh", "gla.h"],
     "epi_bwd": ["epilogue_bwd.cu", "gla_common.cuh", "sm100.cuh", "dig_common.cuh", "bwd_ops.h"],
     "conv_bwd": ["srem_bwd.cu", "srem.cuh", "gla_common.cuh", "sm100.cuh", "dig_common.cuh", "bwd_ops.h"],

@@ -46,6 +46,7 @@ WsLayout ws_layout(int B, int H, int gate_heads, int L, int nchunks, int dk, int
   w.dsn = take(nseq * (size_t)nchunks * dk * dv * 4);
   w.dhn = take(backward ? nseq * (size_t)nchunks * dk * dv * 4 : 0);
   w.flist = take(backward ? (1 + nseq * (size_t)nchunks) * 4 : 0);
+  w.sflag = take(nbz * (size_t)nchunks * 4);
   w.total = off;
   return w;
 }
@@ -162,6 +163,9 @@ dig_status dig_gla_fwd(const void* q, const void* k, const void* v, const float*
   a.gEQ = reinterpret_cast<float*>(ws + lay.gEQ);
   a.gCH = reinterpret_cast<float*>(ws + lay.gCH);
   a.dsn = reinterpret_cast<float*>(ws + lay.dsn);
+  a.sflag = reinterpret_cast<int*>(ws + lay.sflag);
+  a.chunk = C;
+  a.in_bf16 = dtype == DIG_BF16;
   a.spin_ns = spin_limit_ns();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   GlaVariant var{C, dtype == DIG_BF16 ? 2 : 3, d_k, d_v, dtype, out_dtype};
@@ -215,6 +219,9 @@ static dig_status gla_bwd_impl(const void* q, const void* k, const void* v, cons
   a.dsn = reinterpret_cast<float*>((saved ? fws + flay.dsn : ws + lay.dsn));
   a.dhn = reinterpret_cast<float*>(ws + lay.dhn);
   a.flist = reinterpret_cast<uint32_t*>(ws + lay.flist);
+  a.sflag = reinterpret_cast<int*>((saved ? fws + flay.sflag : ws + lay.sflag));
+  a.chunk = C;
+  a.in_bf16 = dtype == DIG_BF16;
   a.spin_ns = spin_limit_ns();
   GlaVariant var{C, dtype == DIG_BF16 ? 2 : 3, d_k, d_v, dtype, out_dtype};
   const cudaError_t e = launch_gla_bwd(var, a, saved, s);

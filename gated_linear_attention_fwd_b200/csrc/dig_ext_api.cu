@@ -99,6 +99,8 @@ dig_status ext_setup(const void* q, const void* k, const void* v, const float* z
   a->B = B; a->H = H; a->L = L; a->Hg = grid_h; a->Wg = grid_w; a->mode = scan_mode; a->gate_heads = gate_heads;
   a->inv_tau = inv_tau;
   a->nchunks = (L + kExtChunk - 1) / kExtChunk;
+  a->chunk = kExtChunk;
+  a->in_bf16 = 0;  // the kernels read fp32 copies of bf16 inputs
   a->status = reinterpret_cast<uint32_t*>(ws);
   a->gEQ = reinterpret_cast<float*>(ws + lay.base.gEQ);
   a->gCH = reinterpret_cast<float*>(ws + lay.base.gCH);

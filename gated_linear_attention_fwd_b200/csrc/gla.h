@@ -43,6 +43,12 @@ struct GlaArgs {
   float* gEQb;       // [B * gate_heads][L (scan order)][DV]   2^(e - rho), e the value-gate cumsum
   float* gCHb;       // [B * gate_heads][nchunks][4][DV]       2^rho, 2^(Gb - rho), 2^Gb, Gb
   float* sfin;       // [nseq][DV][DK] the state after the last chunk (written by the forward scan)
+  // chunks whose key gate decays too fast for the chunk factorisation
+  int* sflag;        // [B * gate_heads][nchunks] 1 where such a chunk was found (written by the gate
+                     // kernel; those chunks are recomputed exactly, gla_strong.cuh); NULL: such a
+                     // chunk sets DIG_ERR_GATE_RANGE instead
+  int chunk;         // tokens per chunk of this call
+  int in_bf16;       // q, k, v, dO are bf16 (else fp32)
 };
 
 // Kernel-variant selection: chunk length, split count, head dims, types.
@@ -57,7 +63,7 @@ struct GlaVariant {
 // the status word, the gate factors, the per-chunk states and, for the
 // backward, the per-chunk state gradients.
 struct WsLayout {
-  size_t gEQ, gCH, dsn, dhn, flist, total;
+  size_t gEQ, gCH, dsn, dhn, flist, sflag, total;
 };
 WsLayout ws_layout(int B, int H, int gate_heads, int L, int nchunks, int dk, int dv, bool backward);
 

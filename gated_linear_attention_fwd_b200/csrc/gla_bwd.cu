@@ -24,6 +24,7 @@
 // of its gradient product before the next one overwrites the region.  With the
 // three gradient accumulators this is 256 TMEM columns, so two CTAs share an SM.
 #include "gla_chunk.cuh"
+#include "gla_strong.cuh"
 
 namespace dig {
 
@@ -389,10 +390,13 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
   }
   if (tid == 0 && (int)blockIdx.x < count) issue_states(unit_at(blockIdx.x));
 
+  bool any_strong = false;  // uniform: a unit of this CTA has a flagged chunk
   for (int kx = blockIdx.x; kx < count; kx += gridDim.x, ++it) {
     const int u = unit_at(kx);
     const Unit U(a, u);
     const int hz = U.bz - U.b * a.gate_heads;
+    const bool skip = !EXT && strong::flagged(a, U.bz, U.n);  // strong gate: its gradients come after the loop
+    any_strong |= skip;
     const bool has_next = kx + (int)gridDim.x < count;
     const int un = has_next ? unit_at(kx + gridDim.x) : 0;
     float* bnd = sh.bnd[it & 1];
@@ -596,7 +600,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
       int tt, g;
       piece_of<K::NGK>(i, tt, g);
       const long long gr = i < C * K::NGK ? rows[tt] : -1;
-      if (gr >= 0) {
+      if (gr >= 0 && !skip) {
         const size_t off = tok_row(gr, a, U.h) * DK + g * PSK;
         copy_piece<KPB>(reinterpret_cast<TOUT*>(a.dq) + off, smem + BC::OFF_SQ + tt * BC::KSB + g * KPB);
         copy_piece<KPB>(reinterpret_cast<TOUT*>(a.dk) + off, smem + BC::OFF_SK + tt * BC::KSB + g * KPB);
@@ -609,7 +613,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
         int tt, g;
         piece_of<K::NGV>(i, tt, g);
         const long long gr = i < C * K::NGV ? rows[tt] : -1;
-        if (gr >= 0)
+        if (gr >= 0 && !skip)
           copy_piece<VPB>(reinterpret_cast<TOUT*>(a.dv) + tok_row(gr, a, U.h) * DV + 8 * g,
                           smem + BC::OFF_SV + tt * BC::VSB + g * VPB);
       }
@@ -643,7 +647,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
       for (int s2 = sg + 1; s2 < BC::NSG; ++s2) post += sh.segtot[s2][sc];
       for (int t = t0; t < t1; ++t) {
         const long long gr = rows[t];
-        if (gr >= 0) {
+        if (gr >= 0 && !skip) {
           float* dst = a.dla + ((size_t)gr * a.gate_heads + hz) * DK + sc;
           const float val = EQ[t * BC::EP + sc] + post;
           if (a.gate_heads == 1) atomicAdd(dst, val);
@@ -667,6 +671,15 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_grad_kernel(const GlaArgs a)
   __syncthreads();
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tmem, BC::TM_COLS);
+  if constexpr (!EXT) {  // this CTA's units of chunks flagged by the gate kernel (strong gates), exactly in fp32
+    static_assert(BC::SMEM >= strong::Cfg<C, DK, DV>::SMEM_GRAD, "shared memory of the strong-gate phase");
+    if (any_strong && !__syncthreads_or(timed_out))
+      for (int kx = blockIdx.x; kx < count; kx += gridDim.x) {
+        const int u = unit_at(kx);
+        const Unit U(a, u);
+        if (strong::flagged(a, U.bz, U.n)) strong::grad_unit<C, DK, DV, TIN, TOUT>(a, u, smem);
+      }
+  }
 }
 
 // ============================================================== dH from saved records

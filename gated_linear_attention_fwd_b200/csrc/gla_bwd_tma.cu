@@ -29,6 +29,7 @@
 // take this kernel; everything else runs the exact kernel directly.
 #include "gla_chunk.cuh"
 #include "tma.cuh"
+#include "gla_strong.cuh"
 #include "tma_tiles.cuh"
 #include "tmap.h"
 
@@ -230,6 +231,7 @@ __global__ void __launch_bounds__(256, 2) gla_grad_tma_kernel(const __grid_const
     const bool has_next_chunk = T.n + 1 < a.nchunks;
     uint32_t amax = 0;  // running |value| of this thread's fp16 operands and products
     bool out_of_range = false;
+    const bool strong_unit = strong::flagged(a, T.bz, T.n);
 
     // ---- 1. states: the boundary term and the S', Gt operands
     wait_bar(&sh.bar_st, ph);
@@ -528,7 +530,8 @@ __global__ void __launch_bounds__(256, 2) gla_grad_tma_kernel(const __grid_const
                      : "memory");
     }
     fence_async_smem();  // staging writes precede the TMA stores that read them
-    const int bad = __syncthreads_or(out_of_range || f16x2_too_large(amax));
+    // a chunk flagged by the gate kernel (strong gate) goes to the exact kernel too
+    const int bad = __syncthreads_or(out_of_range || f16x2_too_large(amax) || strong_unit);
 
     // ---- 7. stores (thread 0), then the next unit's tiles into the freed slots
     if (tid == 0) {

@@ -218,8 +218,11 @@ __device__ __forceinline__ void stage_rows_dk(uint32_t tmem, int col0, float* sd
 // the chunk's tokens, per key channel, stored as the factors EQ = 2^(b - r)
 // (r = b at the chunk's middle token) and the chunk constants {2^r,
 // 2^(Gamma - r), 2^Gamma, Gamma}.  Computed once; every head that shares the
-// gate reads them.  Tokens past the sequence end do not decay.  A factor
-// outside 2^+-115 sets DIG_ERR_GATE_RANGE.
+// gate reads them.  Tokens past the sequence end do not decay.  A chunk with a
+// factor outside 2^+-115 is flagged in a.sflag and gets neutral factors (EQ = 1,
+// constants {1, 0, 2^Gamma, Gamma}: the chunk kernels then form finite values
+// there, the scans the right decay), and gla_strong.cu recomputes it exactly;
+// without a flag array it sets DIG_ERR_GATE_RANGE.
 template <int C, int DK>
 __global__ void __launch_bounds__(256) gla_gate_kernel(const GlaArgs a) {
   constexpr int GP = DK + 4;     // row pitch (floats) of the cumsum buffer
@@ -283,6 +286,7 @@ __global__ void __launch_bounds__(256) gla_gate_kernel(const GlaArgs a) {
     __syncthreads();
     // ---- gate factors and chunk constants
     const float* Gr = G + (C / 2 - 1) * GP;  // b at the reference token
+    bool out_of_range = false;
     for (int i = tid; i < C * NG; i += 256) {
       const int t = i / NG, g = i - t * NG;
       const int p = n * C + t;
@@ -290,20 +294,33 @@ __global__ void __launch_bounds__(256) gla_gate_kernel(const GlaArgs a) {
         const float4 bt = *reinterpret_cast<const float4*>(G + t * GP + 4 * g);
         const float4 rr = *reinterpret_cast<const float4*>(Gr + 4 * g);
         const float d0 = bt.x - rr.x, d1 = bt.y - rr.y, d2 = bt.z - rr.z, d3 = bt.w - rr.w;
-        bad |= fmaxf(fmaxf(fabsf(d0), fabsf(d1)), fmaxf(fabsf(d2), fabsf(d3))) > 115.f;
+        out_of_range |= !(fmaxf(fmaxf(fabsf(d0), fabsf(d1)), fmaxf(fabsf(d2), fabsf(d3))) <= 115.f);
         *reinterpret_cast<float4*>(a.gEQ + ((size_t)bz * a.L + p) * DK + 4 * g) =
             make_float4(ex2(d0), ex2(d1), ex2(d2), ex2(d3));
       }
     }
+    const float r = tid < DK ? Gr[tid] : 0.f, gm = tid < DK ? gam[tid] : 0.f;
+    // uniform: the chunk leaves the range; after this barrier the cumsum buffer,
+    // token table and segment totals may be rewritten by the next unit
+    const bool strong = __syncthreads_or(out_of_range) != 0;
+    if (strong && a.sflag == nullptr) bad = true;
+    if (strong && a.sflag != nullptr) {  // this thread's factors of the chunk become neutral
+      for (int i = tid; i < C * NG; i += 256) {
+        const int t = i / NG, g = i - t * NG;
+        const int p = n * C + t;
+        if (p < a.L)
+          *reinterpret_cast<float4*>(a.gEQ + ((size_t)bz * a.L + p) * DK + 4 * g) = make_float4(1.f, 1.f, 1.f, 1.f);
+      }
+    }
     if (tid < DK) {
       float* ch = a.gCH + ((size_t)bz * a.nchunks + n) * 4 * DK + tid;
-      const float r = Gr[tid], gm = gam[tid];
-      ch[0 * DK] = exp2f(r);
-      ch[1 * DK] = exp2f(gm - r);
+      const bool neutral = strong && a.sflag != nullptr;
+      ch[0 * DK] = neutral ? 1.f : exp2f(r);
+      ch[1 * DK] = neutral ? 0.f : exp2f(gm - r);
       ch[2 * DK] = exp2f(gm);
       ch[3 * DK] = gm;
     }
-    __syncthreads();  // the cumsum buffer, token table and segment totals are reused by the next unit
+    if (tid == 0 && a.sflag != nullptr) a.sflag[u] = strong ? 1 : 0;
   }
   if (bad) set_status(a.status, DIG_ERR_GATE_RANGE);
 }
@@ -538,6 +555,7 @@ cudaError_t launch_value_gate(const GlaArgs& a, cudaStream_t s) {
   g.z = a.zb;
   g.gEQ = a.gEQb;
   g.gCH = a.gCHb;
+  g.sflag = nullptr;  // a value-gate chunk out of range is reported, not recomputed
   const long long gunits = (long long)a.B * a.gate_heads * a.nchunks;
   return launch_pdl(gla_gate_kernel<C, DV>, dim3(persistent_grid(4, gunits)), dim3(256), 0, s, g);
 }

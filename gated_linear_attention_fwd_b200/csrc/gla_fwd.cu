@@ -46,6 +46,7 @@
 // inputs (v) are exact in one term.  The masked P is converted to its terms in
 // place in TMEM and read from there as the A operand of P V.
 #include "gla_chunk.cuh"
+#include "gla_strong.cuh"
 
 namespace dig {
 
@@ -108,6 +109,54 @@ struct ScanJob {
   uint32_t* zero_word;  // set to 0 by the scan (the count of the backward's unit list), or NULL
   ScanEnds ends;
 };
+// One thread's share of the scan of a sequence with a chunk flagged by the gate
+// kernel (strong gate): both passes again, each flagged chunk contributing the
+// block formed from its tokens (strong::state_quad) instead of the stored one.
+// Every thread of the CTA calls it (it holds a barrier).  The value-gated entry
+// points never flag a chunk, so it writes no scan ends and applies no value decay.
+struct ScanRange {
+  float4* st;
+  size_t st_stride;
+  int reverse, bh, bz, c0, jrow, n0, n1, rg, lq;
+  bool act;
+  float4 seed4;
+  int dk, dv;
+};
+__device__ __noinline__ void scan_exact(const GlaArgs a, const ScanRange r, float4 (*sA)[kScanQuads],
+                                        float4 (*sS)[kScanQuads]) {
+  const int nch = a.nchunks;
+  const int* flags = a.sflag + (size_t)r.bz * nch;
+  const float* dec = a.gCH + ((size_t)r.bz * nch * 4 + 2) * r.dk + r.c0;  // 2^Gamma of chunk n at dec + n * 4 * dk
+  auto at = [&](int m) { return r.reverse ? nch - 1 - m : m; };
+  auto decay = [&](int n) { return __ldg(reinterpret_cast<const float4*>(dec + (size_t)n * 4 * r.dk)); };
+  auto contrib = [&](int n) {
+    return __ldcg(flags + n) != 0 ? strong::state_quad(a, r.reverse != 0, r.bh, n, r.c0, r.jrow, r.dk, r.dv)
+                                  : __ldcg(r.st + n * r.st_stride);
+  };
+  auto fma4 = [](float4 g, float4 s, float4 d) {
+    return make_float4(fmaf(g.x, s.x, d.x), fmaf(g.y, s.y, d.y), fmaf(g.z, s.z, d.z), fmaf(g.w, s.w, d.w));
+  };
+  float4 A = make_float4(1.f, 1.f, 1.f, 1.f), s = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (r.act) {
+    for (int m = r.n0; m < r.n1; ++m) {
+      const float4 g = decay(at(m));
+      s = fma4(g, s, contrib(at(m)));
+      A = make_float4(g.x * A.x, g.y * A.y, g.z * A.z, g.w * A.w);
+    }
+  }
+  sA[r.rg][r.lq] = A;  // only this thread wrote or read its entry since the last barrier
+  sS[r.rg][r.lq] = s;
+  __syncthreads();
+  if (!r.act) return;
+  float4 S = r.seed4;
+  for (int m = 0; m < r.rg; ++m) S = fma4(sA[m][r.lq], S, sS[m][r.lq]);
+  for (int m = r.n0; m < r.n1; ++m) {
+    const float4 dd = contrib(at(m));  // read before the entering state takes its place
+    __stcg(r.st + at(m) * r.st_stride, S);
+    S = fma4(decay(at(m)), S, dd);
+  }
+}
+
 __global__ void __launch_bounds__(kScanRanges * kScanQuads, 2) gla_state_scan_kernel(const GlaArgs a, ScanJob job,
                                                                                      int dk, int dv) {
   __shared__ float4 sA[kScanRanges][kScanQuads], sS[kScanRanges][kScanQuads];
@@ -153,17 +202,25 @@ __global__ void __launch_bounds__(kScanRanges * kScanQuads, 2) gla_state_scan_ke
     const float* sp = seed + (size_t)bh * dk * dv + (size_t)c0 * dv + jrow;
     seed4 = make_float4(__ldg(sp), __ldg(sp + dv), __ldg(sp + 2 * dv), __ldg(sp + 3 * dv));
   }
+  // Chunks of this sequence flagged by the gate kernel (strong gates) send the
+  // whole CTA down the exact path below; each thread reads the flags of its range
+  // with its first pass's loads, and the CTA looks at them at the barrier after it.
+  const int* flags = a.sflag != nullptr ? a.sflag + (size_t)bz * nch : nullptr;
+  int flagged_seq = 0;
   float4 A = make_float4(1.f, 1.f, 1.f, 1.f), s = make_float4(0.f, 0.f, 0.f, 0.f);
   float4 d[kScanWindow];
   const bool resident = per <= kScanWindow;  // uniform: one window holds the whole range
   if (act) {
     for (int w0 = n0; w0 < n1; w0 += kScanWindow) {
       float4 g[kScanWindow];
+      int fl[kScanWindow];
 #pragma unroll
       for (int e = 0; e < kScanWindow; ++e) {
+        fl[e] = 0;
         if (w0 + e < n1) {
           g[e] = decay(at(w0 + e));
           d[e] = __ldcg(st + at(w0 + e) * st_stride);
+          if (flags != nullptr) fl[e] = __ldcg(flags + at(w0 + e));
         }
       }
 #pragma unroll
@@ -171,13 +228,18 @@ __global__ void __launch_bounds__(kScanRanges * kScanQuads, 2) gla_state_scan_ke
         if (w0 + e < n1) {
           s = fma4(g[e], s, d[e]);
           A = mul4(g[e], A);
+          flagged_seq |= fl[e];  // next to the block's use: the loads have landed by now
         }
       }
     }
   }
   sA[rg][lq] = A;
   sS[rg][lq] = s;
-  __syncthreads();
+  if (__syncthreads_or(flagged_seq != 0)) {  // rare: both passes again, exactly (strong gates)
+    const ScanRange r{st, st_stride, reverse, bh, bz, c0, jrow, n0, n1, rg, lq, act, seed4, dk, dv};
+    scan_exact(a, r, sA, sS);
+    return;
+  }
   if (!act) return;
   if (rg == 0 && (job.ends.fin[side] != nullptr || job.ends.fin_rows[side] != nullptr)) {
     float4 F = seed4;  // the carry after the last step: every range folded onto the seed
@@ -362,8 +424,11 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
   if (kAhead && (int)blockIdx.x < nunits) issue_s(blockIdx.x);
 
   int it = 0;
+  bool any_strong = false;  // uniform: a unit of this CTA has a flagged chunk
   for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
     const Unit U(a, u);
+    const bool skip = !EXT && strong::flagged(a, U.bz, U.n);  // strong gate: o and y come after the loop
+    any_strong |= skip;
     const int un = u + gridDim.x;
     const bool has_next = kAhead && un < nunits;
     const long long* rows = sh.rows[it & 1];
@@ -514,7 +579,7 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
       int tt, g;
       piece_of<Cfg::NGV>(i, tt, g);
       const long long gr = i < C * Cfg::NGV ? rows[tt] : -1;
-      if (gr >= 0) {
+      if (gr >= 0 && !skip) {
         const size_t off = tok_row(gr, a, U.h) * DV + 8 * g;
         float ov[8];
         const float4 o0 = *reinterpret_cast<const float4*>(stage + tt * OC::OP + 8 * g);
@@ -557,6 +622,14 @@ __global__ void __launch_bounds__(256, 2) gla_chunk_out_kernel(const GlaArgs a) 
   __syncthreads();
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tmem, OC::TM_COLS);
+  if constexpr (!EXT) {  // this CTA's units of chunks flagged by the gate kernel (strong gates), exactly in fp32
+    static_assert(OC::SMEM >= strong::Cfg<C, DK, DV>::SMEM_OUT, "shared memory of the strong-gate phase");
+    if (any_strong && !__syncthreads_or(timed_out))
+      for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+        const Unit U(a, u);
+        if (strong::flagged(a, U.bz, U.n)) strong::out_unit<C, DK, DV, TIN, TOUT>(a, u, smem);
+      }
+  }
 }
 
 // ------------------------------------------------------------------ launch

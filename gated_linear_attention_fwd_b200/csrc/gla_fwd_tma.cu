@@ -18,6 +18,7 @@
 // are formed), so those loads run under this unit's work.  Only bf16 inputs with
 // d_k = 32, d_v = 64 and 128-token chunks that tile the sequence (and, for the
 // column orders, 16-row column segments) take this kernel.
+#include "gla_strong.cuh"
 #include "tma_tiles.cuh"
 
 namespace dig {
@@ -202,9 +203,11 @@ __global__ void __launch_bounds__(256, 2) gla_out_tma_kernel(const __grid_consta
   __syncthreads();  // gamma
 
   int it = 0;
+  bool any_strong = false;  // uniform: a unit of this CTA has a chunk flagged by the gate kernel (strong gate)
   for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
     const uint32_t ph = it & 1;
     const TileUnit T(a, u, C);
+    const bool skip = strong::flagged(a, T.bz, T.n);  // its o and y come after the loop
     const int un = u + gridDim.x;
     const bool has_next = un < nunits;
     auto can_issue = [&]() { return tid == 0 && !timed_out && !sh.abort; };
@@ -376,7 +379,7 @@ __global__ void __launch_bounds__(256, 2) gla_out_tma_kernel(const __grid_consta
 
     // ---- 6. stores (thread 0), then the slots the stores read are refilled
     if (tid == 0) {
-      if (!timed_out && !sh.abort) {
+      if (!timed_out && !sh.abort && !skip) {
         if constexpr (!TC::F32OUT) {
           tile_store<C>(mp.o, T.h * DV, T, a, sb + TC::OFF_EQ, TC::RBV);
           if (with_y) tile_store<C>(mp.y, T.h * DV, T, a, sb + TC::OFF_R, TC::RBV);
@@ -401,6 +404,7 @@ __global__ void __launch_bounds__(256, 2) gla_out_tma_kernel(const __grid_consta
         }
       }
     }
+    any_strong |= skip;
     if (sh.abort) break;  // uniform: read after the barrier above
   }
 
@@ -416,6 +420,14 @@ __global__ void __launch_bounds__(256, 2) gla_out_tma_kernel(const __grid_consta
   __syncthreads();
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tmem, TC::TM_COLS);
+  // this CTA's units of flagged chunks, exactly in fp32, over the drained operand slots
+  static_assert(TC::SMEM - 1024 >= strong::Cfg<C, DK, DV>::SMEM_OUT, "shared memory of the strong-gate phase");
+  if (any_strong && !__syncthreads_or(timed_out || sh.abort))
+    for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+      const TileUnit T(a, u, C);
+      if (strong::flagged(a, T.bz, T.n))
+        strong::out_unit<C, DK, DV, __nv_bfloat16, TOUT>(a, u, smem_raw + (sb - smem_u32(smem_raw)));
+    }
 }
 
 // ------------------------------------------------------------------ launch

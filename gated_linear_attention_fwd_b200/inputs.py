@@ -147,3 +147,30 @@ def custom(B, H, grid_h, grid_w, dk, dv, dtype="bf16", gate="direct", inv_tau=1.
     """A workload of arbitrary shape with the same generators (parity edge cases)."""
     return Workload("custom", B, H, grid_h, grid_w, dk, dv, dtype, gate, D=D, inv_tau=inv_tau,
                     conv_C=conv_C)
+
+
+def strong_gate(w: Workload, kind: str, seed: int, gate_heads: int = 1) -> np.ndarray:
+    """Gate logits z [B, L, gate_heads, dk] (float32) whose decay within a chunk
+    leaves the range of the chunk factorisation (more than 115 halvings over half
+    a chunk in some key channel), for the strong-gate parity cases:
+      "alpha0": z = -1e4 everywhere, so alpha = 0 to fp32 precision and the state
+                keeps only the current token (o_t = (q_t . k_t) v_t);
+      "tau1":   z ~ N(-3, 1), meant with inv_tau = 1 (alpha ~ 0.05, ~4.4 halvings per token);
+      "mixed":  z ~ N(0, 1), except z = -1e4 on the grid tokens of the top-left
+                quadrant (rows < grid_h / 2, columns < grid_w / 2), so that every scan
+                order has both flagged and ordinary chunks, and flagged chunks hold
+                ordinary tokens too."""
+    rng = np.random.default_rng(seed)
+    B, L, dk = w.B, w.L, w.dk
+    if kind == "alpha0":
+        z = np.full((B, L, gate_heads, dk), -1e4)
+    elif kind == "tau1":
+        z = rng.standard_normal((B, L, gate_heads, dk)) - 3.0
+    elif kind == "mixed":
+        z = rng.standard_normal((B, L, gate_heads, dk))
+        gy, gx = np.divmod(np.arange(L), w.grid_w)
+        quad = (gy < w.grid_h // 2) & (gx < w.grid_w // 2)
+        z[:, quad] = -1e4
+    else:
+        raise ValueError(kind)
+    return np.ascontiguousarray(z, dtype=np.float32)

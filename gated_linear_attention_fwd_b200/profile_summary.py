@@ -6,9 +6,10 @@
     # DRAM bytes of one op call (ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --csv ...)
     # -> per-call traffic of the op, recorded in profiles/ncu_traffic.json with the hash of the
     #    op's sources (bench.py uses it only while the sources are unchanged)
-    python -m gated_linear_attention_fwd_b200.profile_summary traffic CSV --op fwd --calls N --workload W --command C
+    python -m gated_linear_attention_fwd_b200.profile_summary traffic CSV [CSV ...] --op fwd --calls N --workload W --command C
+    #    (several CSVs: one capture per scan order, each of N calls; the figure is their mean)
 
-Reads only the CSV it is given; runs nothing.
+Reads only the CSVs it is given; runs nothing.
 """
 import argparse
 import collections
@@ -80,11 +81,14 @@ def launches(args):
 def traffic(args):
     sys.path.insert(0, ROOT)
     import bench  # noqa: E402  (source lists and hash of the ops)
-    _, rows = _rows(args.csv)
     kernels = bench.OP_KERNELS[args.op]
+    # an entry "a | b" names the kernel that replaces the other in some scan orders
+    names = {n.strip() for k in kernels for n in k.split("|")}
+    rows = [r for c in args.csv for r in _rows(c)[1]]
+    calls = args.calls * len(args.csv)  # one capture per scan order, each of args.calls calls
     rd = wr = 0.0
     for r in rows:
-        if _short(r["Kernel Name"]).split("::")[-1] not in kernels:
+        if _short(r["Kernel Name"]).split("::")[-1] not in names:
             continue
         if r["Metric Name"] == "dram__bytes_read.sum":
             rd += _value(r)
@@ -96,9 +100,9 @@ def traffic(args):
     d = {k: v for k, v in d.items() if k in bench.OP_NAMES.values()}
     d[name] = {
         "source_sha": bench._src_hash(bench.OP_SOURCES[args.op]),
-        "dram_bytes_per_call": int((rd + wr) / args.calls),
-        "dram_read_bytes_per_call": int(rd / args.calls),
-        "dram_write_bytes_per_call": int(wr / args.calls),
+        "dram_bytes_per_call": int((rd + wr) / calls),
+        "dram_read_bytes_per_call": int(rd / calls),
+        "dram_write_bytes_per_call": int(wr / calls),
         "kernels": kernels,
         "workload": args.workload,
         "command": args.command,
@@ -123,7 +127,7 @@ def main():
     a.add_argument("--title", required=True)
     a.add_argument("--command", required=True)
     t = sub.add_parser("traffic")
-    t.add_argument("csv")
+    t.add_argument("csv", nargs="+", help="one capture per scan order; the figure is their mean per call")
     t.add_argument("--op", choices=sorted(bench_ops()), required=True)
     t.add_argument("--calls", type=int, required=True)
     t.add_argument("--workload", required=True)

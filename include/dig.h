@@ -65,7 +65,9 @@ enum {
   DIG_ERR_CUDA = 5,               /* a CUDA call failed (launch, attribute query)    */
   DIG_ERR_DEVICE_TIMEOUT = 6,     /* device status: a bounded inter-CTA wait ran out  */
   DIG_ERR_GATE_RANGE = 7          /* device status: a chunk's gate decay left the
-                                     exponent range of the chunked factorisation      */
+                                     exponent range of the chunked factorisation
+                                     (dig_gla_fwd_ext / dig_gla_bwd_ext only; the
+                                     plain entry points compute such chunks)          */
 };
 
 /* Scan orders (DiG scanning directions; layer l of the model uses mode l % 4).
@@ -102,7 +104,11 @@ size_t dig_gla_workspace_bytes(int B, int H, int gate_heads, int L, int d_k, int
  *   y      [B, L, H, d_v]   out_dtype    optional: Swish(r) * o / sqrt(mean(o^2)+eps) * gamma;
  *                                        written only when both r and y are non-NULL
  * The recurrence runs in the scan order `scan_mode` over the grid_h x grid_w
- * grid; no reordered copy of any tensor is written. */
+ * grid; no reordered copy of any tensor is written.
+ * Any finite z is computed: a chunk whose decay over half a chunk exceeds 2^115
+ * in some key channel (the range of the chunk factorisation in fp32) is
+ * recomputed exactly in fp32 token by token, inside the same kernels, and the
+ * backward does the same (strong gates; the device status stays DIG_OK). */
 dig_status dig_gla_fwd(const void *q, const void *k, const void *v, const float *z,
                        int gate_heads, float inv_tau, void *o,
                        const void *r, const float *gamma, float eps, void *y,
@@ -155,7 +161,9 @@ dig_status dig_gla_fwd_noalloc(const void *q, const void *k, const void *v, cons
  * scan order of each call).  d_v must be 64 or 72.  The call runs the fp32
  * kernels (64-token chunks); bf16 inputs are widened into the workspace, whose
  * size dig_gla_ext_workspace_bytes(..., dtype, 0) gives (zero-filled before the
- * first use).  Errors as dig_gla_fwd. */
+ * first use).  Errors as dig_gla_fwd, except that a chunk whose key or value
+ * gate decays beyond 2^115 over half a 64-token chunk is not recomputed: it
+ * sets DIG_ERR_GATE_RANGE in the device status word (dig_read_status). */
 dig_status dig_gla_fwd_ext(const void *q, const void *k, const void *v, const float *z, const float *zb,
                            int gate_heads, float inv_tau, const float *S0, void *o,
                            const void *r, const float *gamma, float eps, void *y, float *S_final,

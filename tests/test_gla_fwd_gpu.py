@@ -146,9 +146,19 @@ def test_workspace_is_reusable_across_calls():
     assert st == 0 and torch.equal(a, b) and torch.equal(b, c)
 
 
-def test_gate_out_of_range_is_reported_not_faulted():
-    w = inputs.custom(1, 1, 16, 16, 32, 64, dtype="bf16", inv_tau=1.0)
+@pytest.mark.parametrize("which", ["key", "value"])
+def test_ext_gate_out_of_range_is_reported_not_faulted(which):
+    """dig_gla_fwd computes strong key gates (tests/test_strong_gate_gpu.py); the
+    extended entry point has no strong-gate path and reports such a chunk in the
+    status word instead, for its key gate and for its value gate alike."""
+    dig = _dig()
+    w = inputs.custom(1, 1, 16, 16, 32, 64, dtype="f32", inv_tau=1.0)
     x = inputs.make_inputs(w, seed=99)
-    z = np.full_like(x["z"], -300.0)   # alpha = e^-300 per token: far outside the factorisation's range
-    _, _, st = run_fwd(w, x, 0, "f32", gate=z)
-    assert st == _dig().DIG_ERR_GATE_RANGE
+    strong = np.full_like(x["z"], -300.0)   # alpha = e^-300 per token: far outside the factorisation's range
+    z = strong if which == "key" else x["z"]
+    zb = np.full((w.B, w.L, 1, w.dv), -300.0 if which == "value" else 0.0, dtype=np.float32)
+    q, k, v = dev(x["q"]), dev(x["k"]), dev(x["v"])
+    o = torch.empty(w.B, w.L, w.H, w.dv, device="cuda")
+    ws = dig.new_ext_workspace(w.B, w.H, w.L, w.dk, w.dv, dtype=torch.float32)
+    dig.dig_gla_fwd_ext(q, k, v, dev(z), w.inv_tau, o, w.grid_h, w.grid_w, 0, ws, zb=dev(zb))
+    assert dig.dig_read_status(ws) == dig.DIG_ERR_GATE_RANGE
