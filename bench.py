@@ -99,7 +99,7 @@ OP_KERNELS = {  # this library's kernels per op on the bench workload (bf16, d_k
     "epi_bwd": ["epilogue_bwd_kernel"],
     "conv_bwd": ["srem_dwconv_bwd_kernel"],
     "gate_fwd": ["gate_proj_tc_kernel"],
-    "gate_bwd": ["gate_proj_bwd_kernel"],
+    "gate_bwd": ["gate_proj_bwd_tc_kernel"],
 }
 STEP_OPS = ("fwd", "bwd", "conv")  # the ops of one timed step
 _CHUNK_SRC = ["gla_chunk.cuh", "gla_common.cuh", "sm100.cuh", "dig_common.cuh", "gla.h"]
@@ -113,7 +113,8 @@ OP_SOURCES = {
     "conv_bwd": ["srem_bwd.cu", "srem.cuh", "gla_common.cuh", "sm100.cuh", "dig_common.cuh", "bwd_ops.h"],
     "gate_fwd": ["gate_proj_tc.cu", "gate_proj.cu", "gate_proj.h", "tma.cuh", "tma_tiles.cuh", "tmap.cu",
                  "gla_common.cuh", "sm100.cuh", "dig_common.cuh"],
-    "gate_bwd": ["gate_proj.cu", "gate_proj.h", "gla_common.cuh", "sm100.cuh", "dig_common.cuh"],
+    "gate_bwd": ["gate_proj_bwd_tc.cu", "gate_proj.cu", "gate_proj.h", "tma.cuh", "tma_tiles.cuh", "tmap.cu",
+                 "gla_common.cuh", "sm100.cuh", "dig_common.cuh"],
 }
 OP_NAMES = {"fwd": "dig_gla_fwd", "bwd": "dig_gla_bwd_saved", "conv": "dig_srem_reorient_dwconv",
             "epi_bwd": "dig_epilogue_bwd", "conv_bwd": "dig_srem_reorient_dwconv_bwd",

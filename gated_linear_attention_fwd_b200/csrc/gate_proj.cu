@@ -306,6 +306,16 @@ __global__ void __launch_bounds__(256) gate_proj_bwd_kernel(const TIN* __restric
 
 namespace {
 
+// a[0 .. na), b[0 .. nb), c[0 .. nc) = 0
+__global__ void __launch_bounds__(256) zero3_kernel(float* a, int na, float* b, int nb, float* c, int nc) {
+  griddep_wait();  // the kernels before this one have completed (they may read the buffers)
+  griddep_launch_dependents();
+  const int i = blockIdx.x * 256 + threadIdx.x;
+  if (i < na) a[i] = 0.f;
+  else if (i < na + nb) b[i - na] = 0.f;
+  else if (i < na + nb + nc) c[i - na - nb] = 0.f;
+}
+
 int resident_grid(const void* kern, size_t smem, long long work, int cap_per_sm) {
   int dev = 0, sms = 148, per_sm = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -370,14 +380,28 @@ cudaError_t launch_gate_proj_fwd(const void* x, const float* W1, const float* W2
                          : fwd_typed<float, 32>(x, W1, W2, b, z, u, rows, D, R, dk, s);
 }
 
+bool gate_proj_bwd_tc_eligible(long long rows, int D, int R, int dk, int tin);  // gate_proj_bwd_tc.cu
+cudaError_t launch_gate_proj_bwd_tc(const void* x, const float* W1, const float* W2, const float* u, const float* z,
+                                    const float* dla, float inv_tau, void* dx, float* dW1, float* dW2, float* db,
+                                    long long rows, int D, int R, int dk, int tout, uint32_t* status, cudaStream_t s,
+                                    bool* launched);
+
 cudaError_t launch_gate_proj_bwd(const void* x, const float* W1, const float* W2, const float* u, const float* z,
                                  const float* dla, float inv_tau, void* dx, float* dW1, float* dW2, float* db,
                                  long long rows, int D, int R, int dk, int tin, int tout, cudaStream_t s) {
   using bf = __nv_bfloat16;
-  cudaError_t e = cudaMemsetAsync(dW1, 0, (size_t)D * R * sizeof(float), s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(dW2, 0, (size_t)R * dk * sizeof(float), s);
-  if (e == cudaSuccess && db) e = cudaMemsetAsync(db, 0, (size_t)dk * sizeof(float), s);
+  // the weight gradients are sums of the blocks' atomics: zeroed first, by one kernel in
+  // the stream's dependent-launch chain
+  const int nw1 = D * R, nw2 = R * dk, nb = db ? dk : 0;
+  cudaError_t e = launch_pdl(zero3_kernel, dim3((nw1 + nw2 + nb + 255) / 256), dim3(256), 0, s, dW1, nw1, dW2, nw2,
+                             db, nb);
   if (e != cudaSuccess || rows == 0) return e;
+  if (gate_proj_bwd_tc_eligible(rows, D, R, dk, tin)) {  // bf16 x: dx and dW1 on the tensor cores
+    bool launched = false;
+    e = launch_gate_proj_bwd_tc(x, W1, W2, u, z, dla, inv_tau, dx, dW1, dW2, db, rows, D, R, dk, tout, nullptr, s,
+                                &launched);
+    if (e != cudaSuccess || launched) return e;
+  }
 #define DIG_GATE_BWD(TI, TO, RT) bwd_typed<TI, TO, RT>(x, W1, W2, u, z, dla, inv_tau, dx, dW1, dW2, db, rows, D, R, dk, s)
   if (R <= 16) {
     if (tin == DIG_BF16) return tout == DIG_BF16 ? DIG_GATE_BWD(bf, bf, 16) : DIG_GATE_BWD(bf, float, 16);

@@ -74,10 +74,13 @@ def test_gate_proj_workloads(index):
 
 
 @pytest.mark.parametrize("rows,D,R,dk", [(1, 8, 16, 32), (65, 24, 5, 6), (130, 16, 20, 3), (64, 384, 32, 128),
-                                         (7, 1024, 16, 36)])
+                                         (7, 1024, 16, 36),
+                                         # bf16: the tensor-core backward (D a multiple of 128 up to 384, R <= 16, d_k <= 32)
+                                         (1, 384, 16, 32), (130, 128, 16, 32), (300, 256, 8, 16), (1000, 384, 12, 28)])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_gate_proj_shapes(rows, D, R, dk, dtype):
-    """One token, ragged tiles, ranks padded to 16 and 32, the largest d_k."""
+    """One token, ragged tiles, ranks padded to 16 and 32, the largest d_k; for bf16 x the
+    last four shapes take the tensor-core backward (one and several tiles, 1-3 channel blocks)."""
     rng = np.random.default_rng(rows + D + R + dk)
     x = rng.standard_normal((rows, D))
     g = {"x": inputs.round_bf16(x) if dtype == "bf16" else x.astype(np.float32),
