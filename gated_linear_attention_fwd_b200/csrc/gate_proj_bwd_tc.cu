@@ -55,7 +55,7 @@ struct GbSmem {
 //          8 rows x 16 B; LBO 128, SBO 256), hi then lo
 //   dua    du terms [M = 128 tokens][K = 16] bf16 (same layout), hi then lo
 //   dub    du^T [N = 32: r hi, then r lo][K = 128 tokens] bf16, no swizzle (LBO 128, SBO 2048)
-//   dz     [128][d_k + 1] fp32;  us [128][17] fp32;  w2 [16][d_k] fp32
+//   dz     [128][d_k + 1] fp32;  us [128][20] fp32 (16-byte rows);  w2 W2^T [d_k][16] fp32
 //   stage  dx staging, 4 KB per warp (32 rows x 128 bytes)
 struct GbLayout {
   uint32_t x, w1, dua, dub, dz, us, w2, stage, total;
@@ -66,7 +66,7 @@ struct GbLayout {
     dub = dua + 2u * 4096u;
     dz = dub + 8192u;
     us = dz + (uint32_t)kBM * (dk + 1) * 4u;
-    w2 = us + (uint32_t)kBM * 17u * 4u;
+    w2 = us + (uint32_t)kBM * 20u * 4u;
     stage = (w2 + 16u * (uint32_t)dk * 4u + 127u) & ~127u;
     total = stage + 8u * 4096u;
   }
@@ -106,7 +106,6 @@ __global__ void __launch_bounds__(256, 1) gate_proj_bwd_tc_kernel(const __grid_c
                                                                   float* __restrict__ dW2, float* __restrict__ db,
                                                                   long long rows, int D, int R, int dk,
                                                                   uint32_t* status) {
-  constexpr int NE2 = 16 * kMaxDK / 32;  // dW2 entries per lane (warp partial sums over its tokens)
   constexpr int NLD = kMaxDK / 8;        // 16-byte loads of d log alpha (and of z) per thread and tile
   extern __shared__ uint8_t smem_raw[];
   __shared__ GbSmem sh;
@@ -167,7 +166,7 @@ __global__ void __launch_bounds__(256, 1) gate_proj_bwd_tc_kernel(const __grid_c
       *reinterpret_cast<__nv_bfloat16*>(sgen + lay.w1 + off) = __float2bfloat16_rn(0.f);
       *reinterpret_cast<__nv_bfloat16*>(sgen + lay.w1 + (uint32_t)(D / 8) * 256u + off) = __float2bfloat16_rn(0.f);
     }
-    for (int i = R * dk + tid; i < 16 * dk; i += 256) W2S[i] = 0.f;
+    for (int i = tid; i < dk * (16 - R); i += 256) W2S[(i / (16 - R)) * 16 + R + i % (16 - R)] = 0.f;
 #pragma unroll
     for (int j = 0; j < NW1; ++j) {
       const int q = tid + 256 * j;
@@ -185,21 +184,23 @@ __global__ void __launch_bounds__(256, 1) gate_proj_bwd_tc_kernel(const __grid_c
       }
     }
 #pragma unroll
-    for (int j = 0; j < NW2L; ++j)
-      if (tid + 256 * j < w24) reinterpret_cast<float4*>(W2S)[tid + 256 * j] = w2v[j];
+    for (int j = 0; j < NW2L; ++j) {  // W2[r][k .. k + 3] -> W2^T[k .. k + 3][r]
+      const int q = tid + 256 * j;
+      if (q < w24) {
+        const int r = (4 * q) / dk, k = 4 * q - r * dk;
+        W2S[(k + 0) * 16 + r] = w2v[j].x;
+        W2S[(k + 1) * 16 + r] = w2v[j].y;
+        W2S[(k + 2) * 16 + r] = w2v[j].z;
+        W2S[(k + 3) * 16 + r] = w2v[j].w;
+      }
+    }
   }
-  for (int i = tid; i < kBM * 17; i += 256) US[i] = 0.f;  // ranks past R stay zero
-  // dW2 entries e = lane + 32 i (r = e / d_k, k = e % d_k) and db[lane]: this warp's sums
-  // over its 16 tokens of every tile, added across the warps at the end
-  float g2[NE2], gb = 0.f;
-  int uo[NE2], zo[NE2];  // the entries' rank and channel (-1: past 16 d_k)
+  for (int i = tid; i < kBM * 20; i += 256) US[i] = 0.f;  // ranks past R stay zero
+  // dW2[r][lane] (r < 16) and db[lane]: this warp's sums over its 16 tokens of every
+  // tile, added across the warps at the end
+  float g2[16], gb = 0.f;  // lane k < d_k: dW2[r][k] for r = 0 .. 15 and db[k]
 #pragma unroll
-  for (int j = 0; j < NE2; ++j) {
-    g2[j] = 0.f;
-    const int e = lane + 32 * j;
-    uo[j] = e < 16 * dk ? e / dk : -1;
-    zo[j] = e < 16 * dk ? e - (e / dk) * dk : 0;
-  }
+  for (int j = 0; j < 16; ++j) g2[j] = 0.f;
   const uint32_t tmem = sh.tmem;
   const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
   uint8_t* stage = sgen + lay.stage + (uint32_t)warp * 4096u;  // this warp's dx staging: 32 rows x 128 bytes
@@ -232,7 +233,7 @@ __global__ void __launch_bounds__(256, 1) gate_proj_bwd_tc_kernel(const __grid_c
       const int n4 = nrow * dk / 4, u4 = nrow * R / 4;
       if (nrow < kBM) {  // the last, partial tile
         for (int idx = nrow * dk + tid; idx < kBM * dk; idx += 256) DZ[(idx / dk) * (dk + 1) + idx % dk] = 0.f;
-        for (int idx = nrow * 16 + tid; idx < kBM * 16; idx += 256) US[(idx >> 4) * 17 + (idx & 15)] = 0.f;
+        for (int idx = nrow * 16 + tid; idx < kBM * 16; idx += 256) US[(idx >> 4) * 20 + (idx & 15)] = 0.f;
       }
 #pragma unroll
       for (int j = 0; j < NLD; ++j) {
@@ -254,7 +255,7 @@ __global__ void __launch_bounds__(256, 1) gate_proj_bwd_tc_kernel(const __grid_c
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int idx = 4 * q + e, t = idx / R;
-            US[t * 17 + (idx - t * R)] = cv[e];
+            US[t * 20 + (idx - t * R)] = cv[e];
           }
         }
       }
@@ -268,8 +269,12 @@ __global__ void __launch_bounds__(256, 1) gate_proj_bwd_tc_kernel(const __grid_c
       for (int rr = 0; rr < 8; ++rr) du[rr] = 0.f;
       for (int k = 0; k < dk; ++k) {
         const float d = DZ[t * (dk + 1) + k];
-#pragma unroll
-        for (int rr = 0; rr < 8; ++rr) du[rr] = fmaf(d, W2S[(8 * h + rr) * dk + k], du[rr]);
+        const float4 w0 = *reinterpret_cast<const float4*>(W2S + k * 16 + 8 * h);
+        const float4 w1 = *reinterpret_cast<const float4*>(W2S + k * 16 + 8 * h + 4);
+        du[0] = fmaf(d, w0.x, du[0]); du[1] = fmaf(d, w0.y, du[1]);
+        du[2] = fmaf(d, w0.z, du[2]); du[3] = fmaf(d, w0.w, du[3]);
+        du[4] = fmaf(d, w1.x, du[4]); du[5] = fmaf(d, w1.y, du[5]);
+        du[6] = fmaf(d, w1.z, du[6]); du[7] = fmaf(d, w1.w, du[7]);
       }
       uint32_t hw[4], lw[4];
 #pragma unroll
@@ -294,14 +299,22 @@ __global__ void __launch_bounds__(256, 1) gate_proj_bwd_tc_kernel(const __grid_c
     // ---- dW2 += u^T dz and db += column sums of dz over this warp's 16 tokens (rows past
     // the end are zero); entry e = lane + 32 j: the lanes read one u value (broadcast) and
     // consecutive dz values of a row
+    if (lane < dk) {
 #pragma unroll 2
-    for (int tt = 0; tt < 16; ++tt) {
-      const float* ur = US + (16 * warp + tt) * 17;
-      const float* zr = DZ + (16 * warp + tt) * (dk + 1);
+      for (int tt = 0; tt < 16; ++tt) {
+        const int t = 16 * warp + tt;
+        const float zk = DZ[t * (dk + 1) + lane];
+        const float4* ur = reinterpret_cast<const float4*>(US + t * 20);  // the token's u (broadcast)
 #pragma unroll
-      for (int j = 0; j < NE2; ++j)
-        if (uo[j] >= 0) g2[j] = fmaf(ur[uo[j]], zr[zo[j]], g2[j]);
-      if (lane < dk) gb += zr[lane];
+        for (int q = 0; q < 4; ++q) {
+          const float4 u4 = ur[q];
+          g2[4 * q] = fmaf(u4.x, zk, g2[4 * q]);
+          g2[4 * q + 1] = fmaf(u4.y, zk, g2[4 * q + 1]);
+          g2[4 * q + 2] = fmaf(u4.z, zk, g2[4 * q + 2]);
+          g2[4 * q + 3] = fmaf(u4.w, zk, g2[4 * q + 3]);
+        }
+        gb += zk;
+      }
     }
     fence_async_smem();  // du terms (and, first time, W1^T) are visible to the tensor core
     tc_fence_before();
@@ -419,10 +432,11 @@ __global__ void __launch_bounds__(256, 1) gate_proj_bwd_tc_kernel(const __grid_c
     float* red = DZ;  // [8][16 * d_k + d_k], over the dz and u staging (contiguous, 25 KB)
     const int ne = 16 * dk + dk;
     __syncthreads();  // every warp is done with the dz staging
+    if (lane < dk) {
 #pragma unroll
-    for (int j = 0; j < NE2; ++j)
-      if (lane + 32 * j < 16 * dk) red[warp * ne + lane + 32 * j] = g2[j];
-    if (lane < dk) red[warp * ne + 16 * dk + lane] = gb;
+      for (int r = 0; r < 16; ++r) red[warp * ne + r * dk + lane] = g2[r];
+      red[warp * ne + 16 * dk + lane] = gb;
+    }
     __syncthreads();
     for (int q = tid; q < ne / 4; q += 256) {
       const int qr = (q + (int)blockIdx.x) % (ne / 4);  // rotated, as above
