@@ -44,7 +44,7 @@ def _short(name):
             depth -= 1
         elif depth == 0:
             out += ch
-    return out.strip()
+    return out.strip().replace("::::", "::")  # an anonymous namespace leaves an empty component
 
 
 def _value(r):
