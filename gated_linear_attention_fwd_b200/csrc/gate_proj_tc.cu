@@ -34,8 +34,8 @@ struct GpSmem {
 // Stages of the x ring: eight, six when D > 768 (the W1 terms then need the room).
 __host__ __device__ inline int ring_stages(int D) { return D > 768 ? 6 : kNS; }
 
-// Dynamic shared memory: the x ring (which first receives W1 and W2 as fp32 by bulk
-// copy), W1^T terms (D / 64 blocks of 16 rows x 128 bytes per term), W2 [16][d_k]
+// Dynamic shared memory: the x ring (whose last stages first receive W1 and W2 as
+// fp32 by bulk copy), W1^T terms (D / 64 blocks of 16 rows x 128 bytes per term), W2 [16][d_k]
 // and b [d_k] (fp32), and the output staging (z [128][d_k], u [128][R] fp32).
 struct GpLayout {
   uint32_t ring, w1, w2, bias, zst, ust, total;
@@ -103,20 +103,32 @@ __global__ void __launch_bounds__(256, 1) gate_proj_tc_kernel(const __grid_const
   griddep_wait();  // the kernels before this one have completed
   griddep_launch_dependents();
   const int ns = ring_stages(D);
-  // ---- W1 and W2 (fp32) into the still empty ring by two bulk copies, then W1^T as two
-  // bf16 terms (row n = output r, K-major, 128-byte swizzle), W2 and b into their places
+  // ---- W1 and W2 (fp32) into the ring's last stages by two bulk copies (the first x
+  // blocks go into the other stages at once), then W1^T as two bf16 terms (row n = output
+  // r, K-major, 128-byte swizzle), W2 and b into their places
   const uint32_t w1_bytes = (uint32_t)D * R * 4u, w2_off = (w1_bytes + 15u) & ~15u;
+  const int nraw = (int)((w2_off + (uint32_t)R * DK * 4u + kXB - 1) / kXB);  // stages the raw weights take
+  const uint32_t raw = lay.ring + (uint32_t)(ns - nraw) * kXB;
   if (tid == 0) {
     mbar_arrive_expect_tx(&sh.wbar, w1_bytes + (uint32_t)R * DK * 4u);
-    bulk_copy_g2s(sb + lay.ring, W1, w1_bytes, &sh.wbar);
-    bulk_copy_g2s(sb + lay.ring + w2_off, W2, (uint32_t)R * DK * 4u, &sh.wbar);
+    bulk_copy_g2s(sb + raw, W1, w1_bytes, &sh.wbar);
+    bulk_copy_g2s(sb + raw + w2_off, W2, (uint32_t)R * DK * 4u, &sh.wbar);
   }
+  auto tile_row = [&](int g) { return (int)((blockIdx.x + (long long)(g / nkb) * gridDim.x) * kBM); };
+  auto load = [&](int g) {
+    const int s = g % ns;
+    mbar_arrive_expect_tx(&sh.full[s], kXB);
+    tma_load_2d(sb + lay.ring + s * kXB, xmap, (g % nkb) * kKB, tile_row(g), &sh.full[s]);
+  };
+  int issued = 0;  // thread 0: blocks requested
+  if (tid == 0)
+    for (; issued < total && issued < ns - nraw; ++issued) load(issued);
   float* sW2 = reinterpret_cast<float*>(sgen + lay.w2);
   float* sB = reinterpret_cast<float*>(sgen + lay.bias);
   const float bv = (tid < DK && b != nullptr) ? __ldg(b + tid) : 0.f;
   const bool w_ok = mbar_wait(&sh.wbar, 0, kSpinLimitNs);
-  const float* rawW1 = reinterpret_cast<const float*>(sgen + lay.ring);
-  const float* rawW2 = reinterpret_cast<const float*>(sgen + lay.ring + w2_off);
+  const float* rawW1 = reinterpret_cast<const float*>(sgen + raw);
+  const float* rawW2 = reinterpret_cast<const float*>(sgen + raw + w2_off);
   for (int i = tid; i < 16 * D; i += 256) {  // element (k, n), i = 16 k + n
     const int k = i >> 4, n = i & 15;
     const float w = (n < R && w_ok) ? rawW1[k * R + n] : 0.f;
@@ -135,14 +147,7 @@ __global__ void __launch_bounds__(256, 1) gate_proj_tc_kernel(const __grid_const
   // every thread's reads of the raw weights precede the x copies into the ring
   fence_async_smem();
   __syncthreads();
-  auto tile_row = [&](int g) { return (int)((blockIdx.x + (long long)(g / nkb) * gridDim.x) * kBM); };
-  auto load = [&](int g) {
-    const int s = g % ns;
-    mbar_arrive_expect_tx(&sh.full[s], kXB);
-    tma_load_2d(sb + lay.ring + s * kXB, xmap, (g % nkb) * kKB, tile_row(g), &sh.full[s]);
-  };
-  int issued = 0;  // thread 0: blocks requested
-  if (tid == 0 && !sh.abort)
+  if (tid == 0 && !sh.abort)  // the raw weights are read: their stages take x blocks too
     for (; issued < total && issued < ns; ++issued) load(issued);
   fence_async_smem();
   tc_fence_before();
